@@ -1,0 +1,357 @@
+"""Benchmark: one MoE layer step (forward + backward) on B200, through libmoe's C ABI.
+
+Workload (default): T=8192 tokens, d=2048, E=128 experts, top-4, SwiGLU ffn=1024, bf16,
+seeded synthetic inputs (x ~ N(0,1), weights ~ N(0,0.02), dY ~ N(0,1)).  A step is
+moe_layer_fwd + moe_layer_bwd: router, routing metadata, permute, grouped SwiGLU GEMMs,
+combine, and the backward of each.  The expert weights (1.6 GB) exceed L2 (126 MB), so
+no L2 flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs one independent replica per GPU (weak scaling; the layer step has no
+data-path exchange), launched by torchrun.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOADS = {
+    # name: (T, d, E, k, f, skew, routing)
+    "e128_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router"),
+    "e8_fwd_bwd": (8192, 2048, 8, 4, 1024, False, "router"),
+    "e128_t16k_skew_fwd_bwd": (16384, 2048, 128, 4, 1024, True, "router"),
+    "e128_t16k_uniform_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "uniform"),
+    # a smaller case of the same kernels for profiler captures (still larger than L2)
+    "profile_e32_t4k": (4096, 2048, 32, 4, 1024, False, "router"),
+}
+DEFAULT = "e128_fwd_bwd"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            j = json.load(fh)
+        return dict(hbm=j["hbm_gbs"], bf16=j["bf16_tflops"], bf16_sus=j.get("bf16_tflops_sustained"),
+                    src="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) >= 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i] == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def make_inputs(name, seed):
+    from routing_grouped_expert_softmax_b200 import inputs as gen
+    T, d, E, k, f, skew, routing = WORKLOADS[name]
+    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=seed, skew=skew)
+    if routing == "uniform":
+        inp.extra["idx"], inp.extra["gate"] = gen.uniform_random_routing(T, E, k, seed=seed)
+    return inp
+
+
+def to_dev_bf16(a, torch):
+    from routing_grouped_expert_softmax_b200 import inputs as gen
+    return torch.from_numpy(gen.bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import routing_grouped_expert_softmax_b200 as moe
+    from routing_grouped_expert_softmax_b200 import build
+    ws_n, rank, local = dist_env()
+    if ws_n > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    torch.cuda.set_device(local)
+    build.build()
+    name = args.workload
+    T, d, E, k, f, skew, routing = WORKLOADS[name]
+    inp = make_inputs(name, seed=0)
+    cfg = moe.config(T, d, E, k, f, dtype="bf16")
+    st = torch.cuda.current_stream()
+    ws = moe.alloc_workspace(cfg)
+    saved = moe.alloc_saved(cfg, logits=False)
+    grads = moe.alloc_grads(cfg, router=(routing == "router"))
+    x = to_dev_bf16(inp.x, torch)
+    dy = to_dev_bf16(inp.dy, torch)
+    wr, wg, wu, wd = (to_dev_bf16(a, torch) for a in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down))
+    bias = torch.from_numpy(inp.bias).cuda() if inp.bias is not None else None
+    w = moe.layer_weights(wr, bias, wg, wu, wd)
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    fwd_fn = moe.moe_layer_fwd
+    if routing == "uniform":
+        saved["topk_idx"].copy_(torch.from_numpy(inp.extra["idx"]))
+        saved["topk_gate"].copy_(torch.from_numpy(inp.extra["gate"]))
+        fwd_fn = moe.moe_layer_fwd_routed
+    launches_per_step = count_launches(routing)
+
+    def step():
+        fwd_fn(cfg, w, x, y, saved, ws, st)
+        moe.moe_layer_bwd(cfg, w, x, dy, saved, grads, ws, st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_error(ws) == 0
+
+    def barrier():
+        if ws_n > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    # ---- headline: K whole steps, device-timed with CUDA events on the launching stream
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    with ClockSampler(local) as clk:
+        e0.record(st)
+        for _ in range(args.steps):
+            step()
+        e1.record(st)
+        barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = ms
+    if ws_n > 1:
+        t = torch.tensor([ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+
+    # ---- the grouped GEMMs alone (6 tcgen05 launches per step), same stream and inputs
+    g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    fwd_ms = bwd_ms = 0.0
+    for _ in range(args.steps):
+        g0.record(st)
+        moe.moe_grouped_swiglu_fwd(cfg, saved["x_perm"], saved["offsets"], wg, wu, wd, saved["hu"],
+                                   saved["a"], saved["y_perm"], ws, st)
+        g1.record(st)
+        moe.moe_grouped_swiglu_bwd(cfg, grads["dy_perm"], saved["x_perm"], saved["hu"], saved["a"],
+                                   saved["offsets"], wg, wu, wd, grads["dhu"], grads["dx_perm"],
+                                   grads["dw_gate"], grads["dw_up"], grads["dw_down"], ws, st)
+        g2.record(st)
+        g2.synchronize()
+        fwd_ms += g0.elapsed_time(g1)
+        bwd_ms += g1.elapsed_time(g2)
+    fwd_ms /= args.steps
+    bwd_ms /= args.steps
+
+    # ---- end to end through the public API with host buffers: x, dY in; y, dx out
+    hx = torch.from_numpy(gen_bits(inp.x)).pin_memory()
+    hdy = torch.from_numpy(gen_bits(inp.dy)).pin_memory()
+    hy = torch.empty(T * d, dtype=torch.int16).pin_memory()
+    hdx = torch.empty(T * d, dtype=torch.int16).pin_memory()
+    xi = x.view(torch.int16).view(-1)
+    dyi = dy.view(torch.int16).view(-1)
+    barrier()
+    e0.record(st)
+    for _ in range(args.steps):
+        xi.copy_(hx, non_blocking=True)
+        dyi.copy_(hdy, non_blocking=True)
+        step()
+        hy.copy_(y.view(torch.int16).view(-1), non_blocking=True)
+        hdx.copy_(grads["dx"].view(torch.int16).view(-1), non_blocking=True)
+    e1.record(st)
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if ws_n > 1:
+        t = torch.tensor([e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    assert moe.moe_get_error(ws) == 0
+
+    P = T * k
+    flops_fwd = 6.0 * P * d * f
+    flops_bwd = 12.0 * P * d * f
+    pk = peaks()
+    gemm_ms = fwd_ms + bwd_ms
+    achieved = (flops_fwd + flops_bwd) / (gemm_ms * 1e-3) / 1e12
+    peak = pk["bf16"]
+    out = {
+        "metric": "MoE-layer tokens/s (E=128,k=4,bf16 fwd+bwd) 1xB200; grouped-GEMM % TC peak",
+        "value": T * ws_n / (ms_max * 1e-3),
+        "unit": "tokens/s",
+        "n_gpus": ws_n,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_max,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+        "config": {"workload": name, "T": T, "d_model": d, "experts": E, "top_k": k, "ffn": f,
+                   "routing": "skewed (Zipf bias)" if skew else routing,
+                   "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+                   "l2": "no flush: 1.6 GB of expert weights per step exceed the 126 MB L2"},
+        "roofline": {"kernel": "grouped SwiGLU GEMMs (6 tcgen05 launches: fwd gate/up, fwd down, "
+                               "dgrad down, wgrad down, dgrad gate/up, wgrad gate/up)",
+                     "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "peak_source": f"{pk['src']} bf16 (burst)",
+                     "traffic": None,
+                     "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+                     "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
+                     "bwd_tflops": flops_bwd / (bwd_ms * 1e-3) / 1e12},
+        "e2e": {"value": T * ws_n / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": 2 * T * d * 2},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(inp, k, args.cpu_tokens)
+    if ws_n > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out))
+
+
+def gen_bits(a):
+    from routing_grouped_expert_softmax_b200 import inputs as gen
+    return gen.bf16_bits(a).view(np.int16).reshape(-1)
+
+
+def count_launches(routing):
+    """Kernels one step launches: forward (router 1, metadata 3, permute 1, grouped GEMMs 2,
+    combine 1) and backward (combine-bwd 1, grouped GEMMs 4, router transpose 1, router
+    weight-gradient 2, unpermute-sum 1)."""
+    fwd = (1 if routing == "router" else 0) + 3 + 1 + 2 + 1
+    bwd = 1 + 4 + (4 if routing == "router" else 1)
+    return fwd + bwd
+
+
+def cpu_baseline(inp, k, n_tokens):
+    """The CPU oracle (float64 NumPy, per-expert loops) on the first n_tokens tokens of the
+    same workload, forward + backward; tokens/s."""
+    from oracle import moe_ref as ref
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count()
+    xs, dys = inp.x[:n_tokens], inp.dy[:n_tokens]
+    t0 = time.perf_counter()
+    fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+    ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
+    dt = time.perf_counter() - t0
+    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n_tokens} tokens of the workload, full weights, fwd+bwd, float64",
+            "seconds": dt}
+
+
+def run_reference(args):
+    """The reference arm is the CPU oracle itself, timed on the host cores."""
+    ws_n, rank, local = dist_env()
+    if rank != 0:
+        return
+    name = args.workload
+    T, d, E, k, f, skew, routing = WORKLOADS[name]
+    inp = make_inputs(name, seed=0)
+    from oracle import moe_ref as ref
+    n = args.cpu_tokens
+    xs, dys = inp.x[:n], inp.dy[:n]
+    for _ in range(min(args.warmup, 1)):
+        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+        ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
+        times.append(time.perf_counter() - t0)
+    dt = float(np.mean(times))
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count()
+    v = n / dt
+    print(json.dumps({
+        "impl": "reference", "metric": "MoE-layer tokens/s (E=128,k=4,bf16 fwd+bwd) 1xB200; grouped-GEMM % TC peak",
+        "value": v, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic", "config": {"workload": name, "T": T, "d_model": d, "experts": E,
+                                                          "top_k": k, "ffn": f},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {n} tokens per step, full weights, fwd+bwd, float64"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
+    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

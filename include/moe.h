@@ -1,0 +1,248 @@
+/*
+ * moe.h -- C ABI of libmoe, a single-GPU MoE layer step for NVIDIA B200 (sm_100a).
+ *
+ * The step, forward and backward, as described in prose by the pages on Ai2's
+ * Olmo-core 3 training stack:
+ *   unite.ai, "Ai2 κυκλοφορεί το Olmo-Core 3, ανοιχτό σύνολο εκπαίδευσης για MoE
+ *     τρισεκατομμυρίων παραμέτρων", section "Παραλληλισμός, Ακρίβεια και Τεχνικές
+ *     Μνήμης" (parallelism, precision and memory techniques): routed rows are
+ *     written straight into the experts' input buffers; routing metadata stays on
+ *     the GPU so the CPU can queue work without waiting for a copy back; a grouped
+ *     GEMM runs the experts' many small matmuls together; MXFP8 for selected ops;
+ *   ettayeb.fr, "Olmo-core 3 ouvre l'entraînement des MoE à l'échelle du trillion
+ *     de paramètres", section "Trois parallélismes, trois optimisations de routage"
+ *     (the same three routing optimisations);
+ *   qidao123.com, "Ai2开源Olmo-core 3 ...", section "新闻原文": 8 -> 128 experts with
+ *     4 selected per token.
+ * The pages give no formulas.  This library computes: softmax router with top-k
+ * on the logits (ties to the lower expert index), gates renormalised over the k
+ * selected experts, a stable counting sort of the routed pairs by expert, a
+ * SwiGLU expert FFN y = (silu(x Wg) * (x Wu)) Wd without biases, and the
+ * gate-weighted sum of each token's k expert outputs.
+ *
+ * Conventions for every call
+ *   - Every pointer argument is a DEVICE pointer, allocated and owned by the
+ *     caller.  The library allocates nothing and keeps no pointer after a call.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream) and never synchronises the host, except moe_get_error.
+ *   - Row-major everywhere.  T tokens, d = model width, E experts, k experts per
+ *     token, f = expert FFN width, P = T*k routed pairs.  Pair i = t*k + j is
+ *     token t's j-th choice.
+ *   - Activations and weights have the element type cfg->dtype (MOE_BF16 or
+ *     MOE_F32).  Logits, gates and router gradients are always fp32; indices,
+ *     counts, offsets and slots int32.
+ *   - Return value: MOE_OK, or a host-detected error (invalid or unsupported
+ *     argument, CUDA launch failure); nothing is launched on a host error.
+ *     Errors found on the device (an expert index out of range, a timed-out
+ *     wait) are OR-ed into an error word inside the workspace and read back by
+ *     moe_get_error.
+ *   - Supported shapes: 1 <= E <= 256, 1 <= k <= min(E, 8), d and f multiples
+ *     of 128, T*k < 2^31.  T = 0 is valid and launches nothing.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *moe_stream_t; /* a cudaStream_t */
+
+enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape outside the supported set above */
+  MOE_ERR_WORKSPACE = 3,     /* workspace pointer missing */
+  MOE_ERR_CUDA = 4,          /* a CUDA call failed (launch, tensor map) */
+  /* device-side error bits, reported by moe_get_error (OR-ed together): */
+  MOE_ERR_DEVICE_INDEX = 16, /* an expert index outside [0, E) */
+  MOE_ERR_DEVICE_TIMEOUT = 32, /* a bounded wait inside a kernel gave up */
+  MOE_ERR_DEVICE_NAN = 64    /* a NaN router logit (its top-k is undefined) */
+};
+
+enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 };
+/* Precision of the grouped GEMMs: MOE_PREC_NATIVE multiplies in the storage
+ * type (bf16, or tf32 for fp32 storage) with fp32 accumulation; MOE_PREC_MXFP8
+ * quantises both operands of each grouped GEMM to E4M3 with one E8M0 scale per
+ * 32 elements along the reduction axis. */
+enum moe_prec { MOE_PREC_NATIVE = 0, MOE_PREC_MXFP8 = 1 };
+
+typedef struct moe_config {
+  int64_t T;     /* tokens */
+  int32_t d;     /* model width */
+  int32_t E;     /* experts */
+  int32_t k;     /* experts per token */
+  int32_t f;     /* expert FFN width */
+  int32_t dtype; /* enum moe_dtype */
+  int32_t prec;  /* enum moe_prec */
+} moe_config;
+
+/* Bytes of device workspace every call taking `ws` needs for this config.
+ * The workspace holds the error word and small scratch (per-block histograms,
+ * a transposed router weight, router-gradient partial sums).  Zero it once
+ * (cudaMemset) before its first use; the library keeps it consistent after. */
+MOE_API size_t moe_workspace_size(const moe_config *cfg);
+
+/* Synchronise `stream`, then report and clear the device error word in `ws`.
+ * *code receives 0 or an OR of MOE_ERR_DEVICE_* bits. */
+MOE_API int moe_get_error(void *ws, moe_stream_t stream, int32_t *code);
+
+/* ---------------------------------------------------------------- routing */
+
+/* Router forward.  logits z = x W_r (+ bias) in fp32; top-k on z, listed by
+ * descending logit with equal logits to the lower index; gates
+ * g_j = exp(z_j) / sum_j' exp(z_j') over the k selected logits (equal to the
+ * full softmax renormalised over the selection).
+ *   x [T,d] dtype; w_router [d,E] dtype; bias [E] fp32 or NULL;
+ *   logits [T,E] fp32 or NULL (not written); topk_idx [T,k] int32;
+ *   topk_gate [T,k] fp32; ws as from moe_workspace_size. */
+MOE_API int moe_route_topk(const moe_config *cfg, const void *x, const void *w_router,
+                   const float *bias, float *logits, int32_t *topk_idx,
+                   float *topk_gate, void *ws, moe_stream_t stream);
+
+/* The router's second half alone: top-k and renormalised gates from given
+ * fp32 logits [T,E].  Same selection and gate rule as moe_route_topk. */
+MOE_API int moe_topk_gating(const moe_config *cfg, const float *logits, int32_t *topk_idx,
+                    float *topk_gate, void *ws, moe_stream_t stream);
+
+/* GPU-resident routing metadata (stable counting sort of the P pairs by expert):
+ *   counts[e] = pairs routed to e; offsets[0..E] = exclusive scan of counts
+ *   (offsets[E] = P); slot_of_pair[i] = offsets[e] + number of pairs i' < i
+ *   with the same expert; pair_of_slot = its inverse.
+ *   topk_idx [T,k] int32 in; counts [E], offsets [E+1], slot_of_pair [P],
+ *   pair_of_slot [P] int32 out.  Indices outside [0, E) set
+ *   MOE_ERR_DEVICE_INDEX and leave the outputs undefined. */
+MOE_API int moe_build_offsets(const moe_config *cfg, const int32_t *topk_idx, int32_t *counts,
+                      int32_t *offsets, int32_t *slot_of_pair, int32_t *pair_of_slot,
+                      void *ws, moe_stream_t stream);
+
+/* Rowwise dispatch: x_perm[slot_of_pair[t*k+j]] = x[t] (a bit copy).
+ *   x [T,d] dtype; slot_of_pair [P]; x_perm [P,d] dtype. */
+MOE_API int moe_permute(const moe_config *cfg, const void *x, const int32_t *slot_of_pair,
+                void *x_perm, moe_stream_t stream);
+
+/* ------------------------------------------------------ grouped expert FFN */
+
+/* Grouped SwiGLU forward over the expert-contiguous rows of x_perm.  For each
+ * expert e and its rows R_e = [offsets[e], offsets[e+1]):
+ *   h = x_perm[R_e] Wg[e], u = x_perm[R_e] Wu[e], a = silu(h) * u,
+ *   y_perm[R_e] = a Wd[e].
+ *   x_perm [P,d]; offsets [E+1]; w_gate, w_up [E,d,f]; w_down [E,f,d];
+ *   hu [P,2f] receives h in columns [0,f) and u in [f,2f) (saved for the
+ *   backward); a [P,f]; y_perm [P,d].  All dtype; fp32 accumulation.
+ * The tile schedule is built on the device from offsets; the host never
+ * reads the counts. */
+MOE_API int moe_grouped_swiglu_fwd(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                           const void *w_gate, const void *w_up, const void *w_down,
+                           void *hu, void *a, void *y_perm, void *ws, moe_stream_t stream);
+
+/* Grouped SwiGLU backward.  Per expert e (rows R_e):
+ *   da = dy_perm Wd^T; dh = da * u * silu'(h); du = da * silu(h);
+ *   dhu = [dh | du] ([P,2f], written); dx_perm = dh Wg^T + du Wu^T;
+ *   dWd[e] = a^T dy_perm; dWg[e] = x_perm^T dh; dWu[e] = x_perm^T du.
+ * An expert with no rows gets zero weight gradients.
+ *   dy_perm, x_perm [P,d]; hu [P,2f] and a [P,f] from the forward;
+ *   dhu [P,2f] out; dx_perm [P,d] out; dw_gate, dw_up [E,d,f] out;
+ *   dw_down [E,f,d] out.  All dtype. */
+MOE_API int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, const void *x_perm,
+                           const void *hu, const void *a, const int32_t *offsets,
+                           const void *w_gate, const void *w_up, const void *w_down,
+                           void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
+                           void *dw_down, void *ws, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- combine */
+
+/* Gate-weighted unpermute: y[t] = sum_j topk_gate[t,j] * y_perm[slot_of_pair[t*k+j]],
+ * accumulated in fp32.  y_perm [P,d]; y [T,d] dtype. */
+MOE_API int moe_unpermute_combine(const moe_config *cfg, const void *y_perm,
+                          const int32_t *slot_of_pair, const float *topk_gate, void *y,
+                          moe_stream_t stream);
+
+/* Backward of the combine: dy_perm[slot(t,j)] = g[t,j] * dy[t];
+ * dgate[t,j] = <dy[t], y_perm[slot(t,j)]> (fp32).
+ *   dy [T,d]; y_perm [P,d]; dy_perm [P,d] out; dgate [T,k] fp32 out. */
+MOE_API int moe_combine_bwd(const moe_config *cfg, const void *dy, const void *y_perm,
+                    const int32_t *slot_of_pair, const float *topk_gate, void *dy_perm,
+                    float *dgate, moe_stream_t stream);
+
+/* Backward of the permute: dx[t] = sum_j dx_perm[slot(t,j)] (fp32 sum).
+ *   dx_perm [P,d]; dx [T,d] out. */
+MOE_API int moe_unpermute_sum(const moe_config *cfg, const void *dx_perm,
+                      const int32_t *slot_of_pair, void *dx, moe_stream_t stream);
+
+/* Router backward.  dz[t,S_j] = g_j (dgate_j - sum_j' g_j' dgate_j'), zero on
+ * unselected experts; dw_router = x^T dz ([d,E] fp32, overwritten);
+ * dx[t] += dz[t] W_r^T (dx [T,d] dtype, read and written). */
+MOE_API int moe_route_bwd(const moe_config *cfg, const float *dgate, const float *topk_gate,
+                  const int32_t *topk_idx, const void *x, const void *w_router, void *dx,
+                  float *dw_router, void *ws, moe_stream_t stream);
+
+/* ------------------------------------------------------------ whole layer */
+
+typedef struct moe_layer_weights {
+  const void *w_router; /* [d,E] dtype */
+  const float *bias;    /* [E] fp32 additive logit bias, or NULL */
+  const void *w_gate;   /* [E,d,f] */
+  const void *w_up;     /* [E,d,f] */
+  const void *w_down;   /* [E,f,d] */
+} moe_layer_weights;
+
+/* Buffers the forward fills and the backward reads (caller-owned). */
+typedef struct moe_layer_saved {
+  float *logits;          /* [T,E] fp32, or NULL */
+  int32_t *topk_idx;      /* [T,k] */
+  float *topk_gate;       /* [T,k] */
+  int32_t *counts;        /* [E] */
+  int32_t *offsets;       /* [E+1] */
+  int32_t *slot_of_pair;  /* [P] */
+  int32_t *pair_of_slot;  /* [P] */
+  void *x_perm;           /* [P,d] */
+  void *hu;               /* [P,2f] */
+  void *a;                /* [P,f] */
+  void *y_perm;           /* [P,d] */
+} moe_layer_saved;
+
+/* Outputs of the backward, plus its intermediates (caller-owned). */
+typedef struct moe_layer_grads {
+  void *dx;          /* [T,d] */
+  float *dw_router;  /* [d,E] fp32, or NULL to skip the router backward */
+  void *dw_gate;     /* [E,d,f] */
+  void *dw_up;       /* [E,d,f] */
+  void *dw_down;     /* [E,f,d] */
+  void *dy_perm;     /* [P,d] intermediate */
+  float *dgate;      /* [T,k] intermediate */
+  void *dhu;         /* [P,2f] intermediate */
+  void *dx_perm;     /* [P,d] intermediate */
+} moe_layer_grads;
+
+/* Whole forward: route_topk -> build_offsets -> permute -> grouped SwiGLU ->
+ * unpermute_combine, all enqueued on `stream` with no host synchronisation.
+ *   x [T,d]; y [T,d] out. */
+MOE_API int moe_layer_fwd(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
+                  const moe_layer_saved *saved, void *ws, moe_stream_t stream);
+
+/* Forward from given routing (e.g. uniform random routing with gates 1/k):
+ * skips the router; saved->topk_idx and saved->topk_gate are inputs. */
+MOE_API int moe_layer_fwd_routed(const moe_config *cfg, const moe_layer_weights *w, const void *x,
+                         void *y, const moe_layer_saved *saved, void *ws, moe_stream_t stream);
+
+/* Whole backward from dy [T,d]: combine_bwd -> grouped SwiGLU backward ->
+ * unpermute_sum (+ router backward when g->dw_router is not NULL). */
+MOE_API int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void *x,
+                  const void *dy, const moe_layer_saved *saved, const moe_layer_grads *g,
+                  void *ws, moe_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H */

@@ -1,0 +1,137 @@
+// Shared helpers for libmoe's kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+typedef __nv_bfloat16 bf16;
+
+// Layout of the small fixed part of the workspace (bytes).
+constexpr size_t WS_ERR = 0;          // int32 device error word
+constexpr size_t WS_FIXED = 256;      // everything else starts here
+
+constexpr int MAX_E = 256;
+constexpr int MAX_K = 8;
+constexpr int SCATTER_CHUNK = 1024;   // routed pairs per block in the metadata kernels
+
+struct Shape {
+  int64_t T;
+  int d, E, k, f;
+  int dtype;
+  int64_t P() const { return T * (int64_t)k; }
+  int es() const { return dtype == MOE_BF16 ? 2 : 4; }
+};
+
+inline Shape shape_of(const moe_config *c) {
+  Shape s;
+  s.T = c->T; s.d = c->d; s.E = c->E; s.k = c->k; s.f = c->f; s.dtype = c->dtype;
+  return s;
+}
+
+inline int *err_word(void *ws) { return reinterpret_cast<int *>(static_cast<char *>(ws) + WS_ERR); }
+
+// Workspace carve-up shared by the host launchers.
+struct WsLayout {
+  size_t block_counts;   // int32 [nblocks][E]
+  size_t w_rt;           // fp32 [E][d]   (transposed router weight)
+  size_t dwr_partial;    // fp32 [RB_SPLIT][E][d]
+  size_t wt;             // fp32 storage only: Wg^T, Wu^T [E][f][d] and Wd^T [E][d][f]
+  size_t total;
+};
+constexpr int RB_SPLIT = 16;          // token splits of the router weight-gradient reduction
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+inline WsLayout ws_layout(const Shape &s) {
+  WsLayout L;
+  size_t off = WS_FIXED;
+  int64_t nb = (s.P() + SCATTER_CHUNK - 1) / SCATTER_CHUNK;
+  L.block_counts = off; off = align_up(off + (size_t)nb * s.E * 4, 256);
+  L.w_rt = off;         off = align_up(off + (size_t)s.E * s.d * 4, 256);
+  L.dwr_partial = off;  off = align_up(off + (size_t)RB_SPLIT * s.E * s.d * 4, 256);
+  L.wt = off;
+  if (s.dtype == MOE_F32) off = align_up(off + (size_t)3 * s.E * s.d * s.f * 4, 256);
+  L.total = off;
+  return L;
+}
+
+template <typename T> __device__ __forceinline__ float to_f(T v);
+template <> __device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f<bf16>(bf16 v) { return __bfloat162float(v); }
+
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ bf16 from_f<bf16>(float v) { return __float2bfloat16_rn(v); }
+
+// 16-byte vector <-> fp32 lanes.  A uint4 holds 8 bf16 or 4 fp32.
+template <typename T> struct Vec;
+template <> struct Vec<bf16> {
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void load(const uint4 &v, float *o) {
+    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { float2 f = __bfloat1622float2(h[i]); o[2 * i] = f.x; o[2 * i + 1] = f.y; }
+  }
+  __device__ __forceinline__ static uint4 store(const float *o) {
+    uint4 v;
+    __nv_bfloat162 *h = reinterpret_cast<__nv_bfloat162 *>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[2 * i], o[2 * i + 1]);
+    return v;
+  }
+};
+template <> struct Vec<float> {
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void load(const uint4 &v, float *o) {
+    o[0] = __uint_as_float(v.x); o[1] = __uint_as_float(v.y);
+    o[2] = __uint_as_float(v.z); o[3] = __uint_as_float(v.w);
+  }
+  __device__ __forceinline__ static uint4 store(const float *o) {
+    return make_uint4(__float_as_uint(o[0]), __float_as_uint(o[1]), __float_as_uint(o[2]),
+                      __float_as_uint(o[3]));
+  }
+};
+
+__device__ __forceinline__ void set_error(int *err, int bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// ---- internal launchers (host side), implemented in routing.cu / rowops.cu / grouped_gemm.cu
+cudaError_t launch_route_topk(const Shape &s, const void *x, const void *w_r, const float *bias,
+                              float *logits, int32_t *idx, float *gate, int *err, cudaStream_t st);
+cudaError_t launch_topk_gating(const Shape &s, const float *logits, int32_t *idx, float *gate,
+                               int *err, cudaStream_t st);
+cudaError_t launch_build_offsets(const Shape &s, const int32_t *idx, int32_t *counts,
+                                 int32_t *offsets, int32_t *slot_of_pair, int32_t *pair_of_slot,
+                                 int32_t *block_counts, int *err, cudaStream_t st);
+cudaError_t launch_permute(const Shape &s, const void *x, const int32_t *slot_of_pair,
+                           void *x_perm, cudaStream_t st);
+cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const int32_t *sop,
+                                     const float *gate, void *y, cudaStream_t st);
+cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm,
+                               const int32_t *sop, const float *gate, void *dy_perm,
+                               float *dgate, cudaStream_t st);
+// dx[t] = sum_j dx_perm[slot(t,j)] (+ sum_j dz_j W_r^T[e_j] when w_rt != nullptr)
+cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int32_t *sop,
+                                 const float *dgate, const float *gate, const int32_t *idx,
+                                 const float *w_rt, bool accumulate, void *dx, cudaStream_t st);
+cudaError_t launch_router_transpose(const Shape &s, const void *w_r, float *w_rt, cudaStream_t st);
+cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
+                                const int32_t *idx, const void *x, float *partial,
+                                float *dw_r, cudaStream_t st);
+int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets,
+                       const void *w_gate, const void *w_up, const void *w_down, void *hu,
+                       void *a, void *y_perm, void *ws, cudaStream_t st);
+// dst[b][c][r] = src[b][r][c] (fp32)
+cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st);
+int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
+                       const void *a, const int32_t *offsets, const void *w_gate,
+                       const void *w_up, const void *w_down, void *dhu, void *dx_perm,
+                       void *dw_gate, void *dw_up, void *dw_down, int *err, cudaStream_t st);
+
+}  // namespace moe

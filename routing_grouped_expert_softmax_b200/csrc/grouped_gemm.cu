@@ -1,0 +1,716 @@
+// Grouped SwiGLU expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// Method: unite.ai "Ai2 κυκλοφορεί το Olmo-Core 3 ...", section "Παραλληλισμός,
+// Ακρίβεια και Τεχνικές Μνήμης": a grouped GEMM runs the experts' many small matmuls
+// together, with the matmuls scheduled from the device so that nothing waits on the
+// host; ettayeb.fr "Olmo-core 3 ouvre l'entraînement des MoE ...", section "Trois
+// parallélismes, trois optimisations de routage"; bigchange.ai "Olmo-core 3 открывает
+// стек обучения MoE от Ai2 ...", section "Три числа, три знаменателя" (the gains sit in
+// the feed-forward compute).
+//
+// One persistent kernel, one CTA per SM, 6 warps:
+//   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) K-blocks in shared
+//               memory (128-byte swizzle), one mbarrier per stage;
+//   warp 1      allocates TMEM; its lane 0 issues tcgen05.mma (128 x BN x 16 per
+//               instruction) into one of two TMEM accumulators and commits each stage
+//               back to the producer;
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31, i.e. one row per thread), apply the fused elementwise
+//               step and store to global memory, then release the accumulator.
+// The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered accumulator).
+//
+// Tile schedule.  Row-grouped GEMMs (forward and data-gradient) tile every expert's row
+// range [offsets[e], offsets[e+1]) in 128-row blocks; each CTA rebuilds the per-expert
+// block prefix from `offsets` on the device, so the host never learns the counts.
+// Rows of a block that belong to the next expert are computed and not stored.
+// Weight-gradient GEMMs reduce over one expert's rows; the last K-block of an expert
+// is zero-filled in shared memory past the expert's end before the MMA reads it.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "tc_ptx.cuh"
+
+namespace moe {
+namespace gg {
+
+enum Mode { FWD_GU = 0, FWD_DOWN = 1, DGRAD_DOWN = 2, DGRAD_GU = 3, WGRAD_DOWN = 4, WGRAD_GU = 5 };
+
+constexpr int BM = 128;
+constexpr int NUM_THREADS = 192;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any tile's time
+
+template <int MODE> struct ModeTraits {
+  static constexpr bool A_MN = (MODE == WGRAD_DOWN || MODE == WGRAD_GU);
+  static constexpr bool B_MN = (MODE == FWD_GU || MODE == FWD_DOWN || MODE == WGRAD_DOWN || MODE == WGRAD_GU);
+  static constexpr bool WGRAD = A_MN;
+};
+
+template <typename T> struct ElemTraits;
+template <> struct ElemTraits<bf16> {
+  static constexpr int ES = 2;
+  static constexpr uint32_t FMT = 1;  // BF16 in the instruction descriptor
+};
+template <> struct ElemTraits<float> {
+  static constexpr int ES = 4;
+  static constexpr uint32_t FMT = 2;  // TF32
+};
+
+template <typename T, int BN> struct Cfg {
+  static constexpr int ES = ElemTraits<T>::ES;
+  static constexpr int KBLK = 128 / ES;                 // K elements per stage (one 128-B swizzle row)
+  static constexpr int UMMA_K = 32 / ES;                // K per tcgen05.mma
+  static constexpr int BOX_MN = 128 / ES;               // MN elements per TMA box of an MN-major operand
+  static constexpr int BOX_BYTES = KBLK * 128;          // bytes of one [KBLK x BOX_MN] box
+  static constexpr int A_BYTES = BM * KBLK * ES;
+  static constexpr int B_BYTES = BN * KBLK * ES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int TMEM_COLS = 2 * BN;              // two accumulators
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 2048 /*bars etc*/;
+};
+
+struct Params {
+  const int32_t *offsets;
+  int E;
+  int P;       // rows of the row-grouped tensors
+  int K;       // reduction length (row-grouped modes)
+  int N;       // output columns
+  int M;       // output rows per expert (weight-gradient modes)
+  int f, d;
+  void *out0;
+  void *out1;
+  const void *aux;
+  int *err;
+  int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
+};
+
+__device__ __forceinline__ void note_fail(const Params &p, int role, int t, int kb, int site) {
+  if (p.where) atomicCAS(&p.where[role], 0, ((t + 1) << 12) | ((kb & 0x3FF) << 2) | (site & 3));
+}
+
+struct Tile {
+  int e, m_blk, n_blk;
+  int row0;       // first A row (row-grouped) or first K row (weight-gradient)
+  int rows;       // valid rows (row-grouped) or valid K rows (weight-gradient)
+  int num_kb;
+};
+
+// Shared control block placed after the stage ring.
+struct Ctrl {
+  uint64_t full[8];
+  uint64_t empty[8];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t tail;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
+};
+
+template <int MODE, int BN, int KBLK>
+__device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl) {
+  if constexpr (ModeTraits<MODE>::WGRAD) {
+    const int mt = p.M / BM, nt = p.N / BN;
+    tl.e = t / (mt * nt);
+    int r = t - tl.e * mt * nt;
+    tl.m_blk = r / nt;
+    tl.n_blk = r - tl.m_blk * nt;
+    int lo = p.offsets[tl.e], hi = p.offsets[tl.e + 1];
+    tl.row0 = lo;
+    tl.rows = hi - lo;
+    tl.num_kb = (tl.rows + KBLK - 1) / KBLK;
+  } else {
+    const int nt = p.N / BN;
+    int g = t / nt;
+    tl.n_blk = t - g * nt;
+    // largest e with prefix[e] <= g (prefix is non-decreasing, prefix[0] = 0)
+    int lo = 0, hi = p.E;  // invariant: prefix[lo] <= g < prefix[hi]
+    while (hi - lo > 1) {
+      int mid = (lo + hi) >> 1;
+      if (c.prefix[mid] <= g) lo = mid; else hi = mid;
+    }
+    tl.e = lo;
+    tl.m_blk = g - c.prefix[lo];
+    int off = p.offsets[lo], cnt = p.offsets[lo + 1] - off;
+    tl.row0 = off + tl.m_blk * BM;
+    tl.rows = min(BM, cnt - tl.m_blk * BM);
+    tl.num_kb = p.K / KBLK;
+  }
+  return true;
+}
+
+template <int MODE, int BN>
+__device__ __forceinline__ int total_tiles(const Params &p, const Ctrl &c) {
+  if constexpr (ModeTraits<MODE>::WGRAD) return p.E * (p.M / BM) * (p.N / BN);
+  else return c.prefix[p.E] * (p.N / BN);
+}
+
+// Store 32 consecutive values of one row.
+template <typename T>
+__device__ __forceinline__ void store32(T *dst, const float (&v)[32]) {
+  uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+  constexpr int N = Vec<T>::N;
+#pragma unroll
+  for (int i = 0; i < 32 / N; ++i) d4[i] = Vec<T>::store(&v[i * N]);
+}
+template <typename T>
+__device__ __forceinline__ void load32(const T *src, float (&v)[32]) {
+  const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+  constexpr int N = Vec<T>::N;
+#pragma unroll
+  for (int i = 0; i < 32 / N; ++i) Vec<T>::load(s4[i], &v[i * N]);
+}
+
+__device__ __forceinline__ float sigmoidf_(float h) { return 1.0f / (1.0f + __expf(-h)); }
+
+template <typename T, int BN, int MODE>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                        const __grid_constant__ CUtensorMap tmB0,
+                        const __grid_constant__ CUtensorMap tmB1, const Params p) {
+  using C = Cfg<T, BN>;
+  using MT = ModeTraits<MODE>;
+  // tf32 operands are only ever K-major: the fp32 forward reads pre-transposed weights
+  constexpr bool FWD_B_KMAJOR = (sizeof(T) == 4) && (MODE == FWD_GU || MODE == FWD_DOWN);
+  constexpr bool B_MN = MT::B_MN && !FWD_B_KMAJOR;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *ring = smem;                                   // STAGES x (A | B)
+  Ctrl &c = *reinterpret_cast<Ctrl *>(smem + C::STAGES * C::STAGE_BYTES);
+  volatile int *abort_flag = &c.abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ------------------------------------------------------------------ prologue
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(ptx::smem_u32(&c.full[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&c.empty[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
+      ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), 128);
+    }
+    ptx::mbar_init(ptx::smem_u32(&c.tail), 1);
+    ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
+    c.abort = 0;
+    ptx::fence_mbar_init();
+    ptx::tma_prefetch(&tmA);
+    ptx::tma_prefetch(&tmB0);
+    ptx::tma_prefetch(&tmB1);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  if (warp == 2 && !MT::WGRAD) {
+    // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
+    int cnt[8], s = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int e = lane * 8 + i;
+      int n = 0;
+      if (e < p.E) n = (p.offsets[e + 1] - p.offsets[e] + BM - 1) / BM;
+      cnt[i] = n;
+      s += n;
+    }
+    int incl = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - s;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      int e = lane * 8 + i;
+      if (e < p.E) c.prefix[e] = run;
+      run += cnt[i];
+    }
+    if (lane == 31) c.prefix[p.E] = incl;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = c.tmem_base;
+  const int ntiles = total_tiles<MODE, BN>(p, c);
+
+  if (warp == 0) {
+    // ================================================================ producer
+    int stage = 0;
+    uint32_t phase = 0, tail_phase = 0;
+    uint32_t armed = 0, armed_par = 0;  // per stage: a fill is in flight / its parity
+    bool tail_armed = false;
+    bool ok = true;
+    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+      Tile tl;
+      get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+      for (int kb = 0; kb < tl.num_kb && ok; ++kb) {
+        if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 0); break; }
+        const uint32_t a_dst = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
+        const uint32_t b_dst = a_dst + C::A_BYTES;
+        int valid = C::KBLK;
+        if constexpr (MT::WGRAD) valid = min(C::KBLK, tl.rows - kb * C::KBLK);
+        const bool tail = valid < C::KBLK;
+        const uint32_t bar = tail ? ptx::smem_u32(&c.tail) : ptx::smem_u32(&c.full[stage]);
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+          // ---- A
+          if constexpr (MT::A_MN) {
+#pragma unroll
+            for (int i = 0; i < BM / C::BOX_MN; ++i)
+              ptx::tma_load_2d(a_dst + i * C::BOX_BYTES, &tmA, bar, tl.m_blk * BM + i * C::BOX_MN,
+                               tl.row0 + kb * C::KBLK);
+          } else {
+            ptx::tma_load_2d(a_dst, &tmA, bar, kb * C::KBLK, tl.row0);
+          }
+          // ---- B
+          if constexpr (FWD_B_KMAJOR && MODE == FWD_GU) {
+            // Wg^T, Wu^T [E*f][d]: gate rows then up rows of the 256-row B tile
+            const int half = BN / 2;
+            ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.f + tl.n_blk * half);
+            ptx::tma_load_2d(b_dst + half * 128, &tmB1, bar, kb * C::KBLK, tl.e * p.f + tl.n_blk * half);
+          } else if constexpr (FWD_B_KMAJOR && MODE == FWD_DOWN) {
+            // Wd^T [E*d][f]
+            ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+          } else if constexpr (MODE == FWD_GU) {
+            const int half = BN / 2;
+#pragma unroll
+            for (int i = 0; i < half / C::BOX_MN; ++i) {
+              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * half + i * C::BOX_MN,
+                               tl.e * p.K + kb * C::KBLK);
+              ptx::tma_load_2d(b_dst + (half / C::BOX_MN + i) * C::BOX_BYTES, &tmB1, bar,
+                               tl.n_blk * half + i * C::BOX_MN, tl.e * p.K + kb * C::KBLK);
+            }
+          } else if constexpr (MODE == FWD_DOWN) {
+#pragma unroll
+            for (int i = 0; i < BN / C::BOX_MN; ++i)
+              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * BN + i * C::BOX_MN,
+                               tl.e * p.K + kb * C::KBLK);
+          } else if constexpr (MODE == DGRAD_DOWN) {
+            ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.f + tl.n_blk * BN);
+          } else if constexpr (MODE == DGRAD_GU) {
+            const int kb_half = p.f / C::KBLK;
+            if (kb < kb_half)
+              ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+            else
+              ptx::tma_load_2d(b_dst, &tmB1, bar, (kb - kb_half) * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+          } else {  // weight gradients: B is the MN-major activation gradient
+#pragma unroll
+            for (int i = 0; i < BN / C::BOX_MN; ++i)
+              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * BN + i * C::BOX_MN,
+                               tl.row0 + kb * C::KBLK);
+          }
+        }
+        if (tail) {
+          // Weight gradients only: K rows past the expert's end belong to another expert
+          // (or lie outside the tensor): zero them before the MMA reads the stage.
+          tail_armed = true;
+          ok = ptx::mbar_wait(ptx::smem_u32(&c.tail), tail_phase, abort_flag, WAIT_LIMIT_NS);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
+          tail_armed = false;
+          tail_phase ^= 1;
+          // In an MN-major box each K row is one 128-byte line: rows [valid, KBLK) are the
+          // byte range [valid*128, KBLK*128) of every box.
+          const int nbox_a = BM / C::BOX_MN, nbox_b = BN / C::BOX_MN;
+          const int line0 = valid * 8, lines = C::KBLK * 8;  // in 16-byte units
+          uint4 z = make_uint4(0, 0, 0, 0);
+          for (int b = 0; b < nbox_a + nbox_b; ++b) {
+            uint8_t *box = ring + stage * C::STAGE_BYTES + (b < nbox_a ? b * C::BOX_BYTES
+                                                                        : C::A_BYTES + (b - nbox_a) * C::BOX_BYTES);
+            for (int i = line0 + lane; i < lines; i += 32) reinterpret_cast<uint4 *>(box)[i] = z;
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
+        }
+        // this stage's full barrier completes (or has completed) the phase of this pass
+        armed |= 1u << stage;
+        if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
+        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+      }
+    }
+    // Drain: every TMA fill this warp issued must land before the CTA may exit.
+    if (lane == 0) {
+      for (int s = 0; s < C::STAGES; ++s)
+        if ((armed >> s) & 1u)
+          if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
+            note_fail(p, 0, 0, s, 2);
+      if (tail_armed && !ptx::mbar_wait(ptx::smem_u32(&c.tail), tail_phase, abort_flag, WAIT_LIMIT_NS))
+        note_fail(p, 0, 0, 0, 3);
+    }
+  } else if (warp == 1) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = (1u << 4) | (ElemTraits<T>::FMT << 7) | (ElemTraits<T>::FMT << 10) |
+                                 ((MT::A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
+                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+        Tile tl;
+        get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+        const int acc = it & 1;
+        const uint32_t aph = (it >> 1) & 1;
+        ok = ptx::mbar_wait(ptx::smem_u32(&c.tempty[acc]), aph ^ 1, abort_flag, WAIT_LIMIT_NS);
+        if (!ok) { note_fail(p, 1, t, 0, 0); break; }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        if (tl.num_kb == 0) {
+          ptx::mbar_arrive(ptx::smem_u32(&c.tfull[acc]));
+          continue;
+        }
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          ok = ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
+          if (!ok) { note_fail(p, 1, t, kb, 1); break; }
+          ptx::tc_fence_after();
+          const uint32_t a_addr = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
+          const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < C::KBLK / C::UMMA_K; ++kk) {
+            uint64_t adesc, bdesc;
+            if constexpr (MT::A_MN)
+              adesc = ptx::smem_desc_sw128(a_addr + kk * C::UMMA_K * 128, C::BOX_BYTES, 1024);
+            else
+              adesc = ptx::smem_desc_sw128(a_addr + kk * 32, 16, 1024);
+            if constexpr (B_MN)
+              bdesc = ptx::smem_desc_sw128(b_addr + kk * C::UMMA_K * 128, C::BOX_BYTES, 1024);
+            else
+              bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
+            const uint32_t accum = (kb | kk) ? 1u : 0u;
+            if constexpr (sizeof(T) == 2) ptx::mma_f16(d_tmem, adesc, bdesc, idesc, accum);
+            else ptx::mma_tf32(d_tmem, adesc, bdesc, idesc, accum);
+          }
+          ptx::tc_commit(ptx::smem_u32(&c.empty[stage]));
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+        ptx::tc_commit(ptx::smem_u32(&c.tfull[acc]));
+      }
+      // Drain: all MMAs issued here complete before TMEM is freed.
+      ptx::tc_commit(ptx::smem_u32(&c.drain));
+      if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, abort_flag, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
+    }
+    __syncwarp();
+  } else {
+    // ================================================================ epilogue
+    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    const int r = q * 32 + lane;          // tile row owned by this thread
+    int it = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+      Tile tl;
+      get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+      const int acc = it & 1;
+      const uint32_t aph = (it >> 1) & 1;
+      bool ok = ptx::mbar_wait(ptx::smem_u32(&c.tfull[acc]), aph, abort_flag, WAIT_LIMIT_NS);
+      if (!__all_sync(0xffffffffu, ok)) { if (lane == 0) note_fail(p, 2, t, 0, 0); break; }
+      ptx::tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
+
+      if constexpr (MODE == FWD_GU) {
+        // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
+        const bool valid = r < tl.rows;
+        const int64_t row = (int64_t)tl.row0 + r;
+        T *hu = static_cast<T *>(p.out0);
+        T *aa = static_cast<T *>(p.out1);
+#pragma unroll 1
+        for (int cc = 0; cc < BN / 2; cc += 32) {
+          float h[32], u[32];
+          ptx::tmem_ld32(taddr + cc, h);
+          ptx::tmem_ld32(taddr + BN / 2 + cc, u);
+          if (valid) {
+            const int col = tl.n_blk * (BN / 2) + cc;
+            store32(hu + row * 2 * p.f + col, h);
+            store32(hu + row * 2 * p.f + p.f + col, u);
+            float a[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) a[i] = h[i] * sigmoidf_(h[i]) * u[i];
+            store32(aa + row * p.f + col, a);
+          }
+        }
+      } else if constexpr (MODE == FWD_DOWN || MODE == DGRAD_GU) {
+        const bool valid = r < tl.rows;
+        const int64_t row = (int64_t)tl.row0 + r;
+        T *out = static_cast<T *>(p.out0);
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          float v[32];
+          ptx::tmem_ld32(taddr + cc, v);
+          if (valid) store32(out + row * p.N + tl.n_blk * BN + cc, v);
+        }
+      } else if constexpr (MODE == DGRAD_DOWN) {
+        // da -> (dh, du) through the SwiGLU derivative, using the saved h and u
+        const bool valid = r < tl.rows;
+        const int64_t row = (int64_t)tl.row0 + r;
+        const T *hu = static_cast<const T *>(p.aux);
+        T *dhu = static_cast<T *>(p.out0);
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          float da[32];
+          ptx::tmem_ld32(taddr + cc, da);
+          if (valid) {
+            const int col = tl.n_blk * BN + cc;
+            float h[32], u[32];
+            load32(hu + row * 2 * p.f + col, h);
+            load32(hu + row * 2 * p.f + p.f + col, u);
+            float dh[32], du[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              float s = sigmoidf_(h[i]);
+              dh[i] = da[i] * u[i] * s * (1.0f + h[i] * (1.0f - s));
+              du[i] = da[i] * h[i] * s;
+            }
+            store32(dhu + row * 2 * p.f + col, dh);
+            store32(dhu + row * 2 * p.f + p.f + col, du);
+          }
+        }
+      } else {  // weight gradients: row r of the [M x N] block of expert e
+        const int64_t mrow = (int64_t)tl.m_blk * BM + r;
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          float v[32];
+          if (tl.num_kb > 0) ptx::tmem_ld32(taddr + cc, v);
+          else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+          }
+          const int col = tl.n_blk * BN + cc;
+          if constexpr (MODE == WGRAD_DOWN) {
+            T *out = static_cast<T *>(p.out0);
+            store32(out + ((int64_t)tl.e * p.M + mrow) * p.N + col, v);
+          } else {
+            // N runs over [dh | du]: columns below f are dW_gate, the rest dW_up
+            T *out = static_cast<T *>(col < p.f ? p.out0 : p.out1);
+            const int cf = col < p.f ? col : col - p.f;
+            store32(out + ((int64_t)tl.e * p.M + mrow) * p.f + cf, v);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+    }
+  }
+
+  // ------------------------------------------------------------------ teardown
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0 && c.abort) set_error(p.err, MOE_ERR_DEVICE_TIMEOUT);
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2D row-major tensor [rows][cols], box [box_rows][box_cols], 128-byte swizzle.
+static bool make_tmap(CUtensorMap *m, const void *ptr, int es, uint64_t cols, uint64_t rows,
+                      uint32_t box_cols, uint32_t box_rows) {
+  auto enc = get_encode();
+  if (!enc) return false;
+  cuuint64_t gdim[2] = {cols, rows};
+  cuuint64_t gstride[1] = {cols * (uint64_t)es};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estride[2] = {1, 1};
+  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                   const_cast<void *>(ptr), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <typename T, int BN, int MODE>
+static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p,
+                  int64_t max_tiles, cudaStream_t st) {
+  using C = Cfg<T, BN>;
+  auto kern = grouped_gemm_kernel<T, BN, MODE>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    attr_set = true;
+  }
+  int64_t grid = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
+  kern<<<(unsigned)grid, NUM_THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+template <typename T>
+static int fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
+                    const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
+                    cudaStream_t st) {
+  int *err = err_word(ws);
+  if constexpr (sizeof(T) == 4) {
+    // tf32 MMAs take K-major operands only: stage Wg^T, Wu^T [E][f][d] and Wd^T [E][d][f]
+    WsLayout L = ws_layout(s);
+    char *w = static_cast<char *>(ws);
+    float *wgt = reinterpret_cast<float *>(w + L.wt), *wut = wgt + (size_t)s.E * s.d * s.f,
+          *wdt = wut + (size_t)s.E * s.d * s.f;
+    if (launch_transpose_batched(static_cast<const float *>(w_gate), wgt, s.E, s.d, s.f, st) ||
+        launch_transpose_batched(static_cast<const float *>(w_up), wut, s.E, s.d, s.f, st) ||
+        launch_transpose_batched(static_cast<const float *>(w_down), wdt, s.E, s.f, s.d, st))
+      return MOE_ERR_CUDA;
+    w_gate = wgt; w_up = wut; w_down = wdt;
+  }
+  constexpr int ES = sizeof(T);
+  constexpr int KBLK = 128 / ES, BOX_MN = 128 / ES;
+  const int64_t P = s.P();
+  CUtensorMap tA, tB0, tB1;
+  Params p{};
+  p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
+  const int64_t mblocks = (P + BM - 1) / BM + s.E;
+  // GEMM 1: [h | u] = x_perm [P,d] x [Wg | Wu] [d,f]; N tile = 128 gate + 128 up columns
+  {
+    constexpr int BN = 256;
+    if (!make_tmap(&tA, x_perm, ES, s.d, P, KBLK, BM)) return MOE_ERR_CUDA;
+    if constexpr (sizeof(T) == 4) {
+      if (!make_tmap(&tB0, w_gate, ES, s.d, (uint64_t)s.E * s.f, KBLK, BN / 2)) return MOE_ERR_CUDA;
+      if (!make_tmap(&tB1, w_up, ES, s.d, (uint64_t)s.E * s.f, KBLK, BN / 2)) return MOE_ERR_CUDA;
+    } else {
+      if (!make_tmap(&tB0, w_gate, ES, s.f, (uint64_t)s.E * s.d, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+      if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+    }
+    p.K = s.d; p.N = 2 * s.f; p.out0 = hu; p.out1 = a; p.aux = nullptr;
+    int rc = launch<T, BN, FWD_GU>(tA, tB0, tB1, p, mblocks * (p.N / BN), st);
+    if (rc) return rc;
+  }
+  // GEMM 2: y_perm = a [P,f] x Wd [f,d]
+  {
+    if (!make_tmap(&tA, a, ES, s.f, P, KBLK, BM)) return MOE_ERR_CUDA;
+    p.K = s.f; p.N = s.d; p.out0 = y_perm; p.out1 = nullptr;
+    int rc;
+    const int bn = (s.d % 256 == 0) ? 256 : 128;
+    bool ok;
+    if constexpr (sizeof(T) == 4)
+      ok = make_tmap(&tB0, w_down, ES, s.f, (uint64_t)s.E * s.d, KBLK, bn);
+    else
+      ok = make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, BOX_MN, KBLK);
+    if (!ok) return MOE_ERR_CUDA;
+    if (bn == 256)
+      rc = launch<T, 256, FWD_DOWN>(tA, tB0, tB0, p, mblocks * (p.N / 256), st);
+    else
+      rc = launch<T, 128, FWD_DOWN>(tA, tB0, tB0, p, mblocks * (p.N / 128), st);
+    if (rc) return rc;
+  }
+  return MOE_OK;
+}
+
+template <typename T>
+static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
+                    const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
+                    const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
+                    void *dw_down, int *err, cudaStream_t st) {
+  constexpr int ES = sizeof(T);
+  constexpr int KBLK = 128 / ES, BOX_MN = 128 / ES;
+  const int64_t P = s.P();
+  CUtensorMap tA, tB0, tB1;
+  Params p{};
+  p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
+  const int64_t mblocks = (P + BM - 1) / BM + s.E;
+  int rc;
+  // (1) da = dy_perm [P,d] x Wd^T [d,f]  -> SwiGLU backward -> dhu [P,2f]
+  {
+    if (!make_tmap(&tA, dy_perm, ES, s.d, P, KBLK, BM)) return MOE_ERR_CUDA;
+    p.K = s.d; p.N = s.f; p.out0 = dhu; p.aux = hu;
+    if (s.f % 256 == 0) {
+      if (!make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, KBLK, 256)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, DGRAD_DOWN>(tA, tB0, tB0, p, mblocks * (s.f / 256), st);
+    } else {
+      if (!make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, KBLK, 128)) return MOE_ERR_CUDA;
+      rc = launch<T, 128, DGRAD_DOWN>(tA, tB0, tB0, p, mblocks * (s.f / 128), st);
+    }
+    if (rc) return rc;
+  }
+  // (2) dWd[e] = a^T [f, rows_e] x dy_perm [rows_e, d]
+  {
+    if (!make_tmap(&tA, a, ES, s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+    p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
+    if (s.d % 256 == 0) {
+      if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st);
+    } else {
+      if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+      rc = launch<T, 128, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st);
+    }
+    if (rc) return rc;
+  }
+  // (3) dx_perm = dhu [P,2f] x [Wg | Wu]^T [2f,d]
+  {
+    if (!make_tmap(&tA, dhu, ES, 2 * s.f, P, KBLK, BM)) return MOE_ERR_CUDA;
+    p.K = 2 * s.f; p.N = s.d; p.out0 = dx_perm;
+    if (s.d % 256 == 0) {
+      if (!make_tmap(&tB0, w_gate, ES, s.f, (uint64_t)s.E * s.d, KBLK, 256)) return MOE_ERR_CUDA;
+      if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, KBLK, 256)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, DGRAD_GU>(tA, tB0, tB1, p, mblocks * (s.d / 256), st);
+    } else {
+      if (!make_tmap(&tB0, w_gate, ES, s.f, (uint64_t)s.E * s.d, KBLK, 128)) return MOE_ERR_CUDA;
+      if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, KBLK, 128)) return MOE_ERR_CUDA;
+      rc = launch<T, 128, DGRAD_GU>(tA, tB0, tB1, p, mblocks * (s.d / 128), st);
+    }
+    if (rc) return rc;
+  }
+  // (4) [dWg | dWu][e] = x_perm^T [d, rows_e] x dhu [rows_e, 2f]
+  {
+    if (!make_tmap(&tA, x_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+    if (!make_tmap(&tB0, dhu, ES, 2 * s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+    p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
+    if (s.f % 256 == 0)
+      rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st);
+    else
+      rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st);
+    if (rc) return rc;
+  }
+  return MOE_OK;
+}
+
+}  // namespace gg
+
+int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
+                       const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
+                       cudaStream_t st) {
+  if (s.dtype == MOE_BF16)
+    return gg::fwd_impl<bf16>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
+  return gg::fwd_impl<float>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
+}
+
+int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
+                       const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
+                       const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
+                       void *dw_down, int *err, cudaStream_t st) {
+  // The weight-gradient GEMMs reduce over tokens, which makes both operands MN-major;
+  // tf32 MMAs take K-major operands only, so the fp32 backward is not offered.
+  if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  return gg::bwd_impl<bf16>(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
+                            dw_gate, dw_up, dw_down, err, st);
+}
+
+}  // namespace moe

@@ -1,0 +1,277 @@
+// extern "C" entry points of libmoe: argument validation, workspace carve-up, and the
+// composition of the layer step.  Every step runs in this library's kernels; nothing
+// here touches the host copy of any tensor.
+#include <string.h>
+
+#include <initializer_list>
+
+#include "common.cuh"
+
+using namespace moe;
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_cfg(const moe_config *c) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->T < 0 || c->d <= 0 || c->f <= 0 || c->E <= 0 || c->k <= 0) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_BF16 && c->dtype != MOE_F32) return MOE_ERR_INVALID_ARG;
+  if (c->prec != MOE_PREC_NATIVE && c->prec != MOE_PREC_MXFP8) return MOE_ERR_INVALID_ARG;
+  if (c->E > MAX_E || c->k > MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
+  if (c->d % 128 || c->f % 128) return MOE_ERR_UNSUPPORTED;
+  if (c->T * (int64_t)c->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
+  if (c->prec == MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// All pointers non-null and 16-byte aligned (rows are moved as 16-byte vectors / TMA tiles).
+int check_ptrs(std::initializer_list<const void *> ps) {
+  for (const void *p : ps)
+    if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+// Pointers that only need to be non-null and 4-byte aligned (index and fp32 arrays).
+int check_ptrs4(std::initializer_list<const void *> ps) {
+  for (const void *p : ps)
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 3u)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+int cuda_rc(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+cudaStream_t S(moe_stream_t s) { return static_cast<cudaStream_t>(s); }
+
+#define RETURN_IF(x)        \
+  do {                      \
+    int _rc = (x);          \
+    if (_rc) return _rc;    \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_config *cfg) {
+  if (!cfg || cfg->T < 0 || cfg->E <= 0 || cfg->d <= 0 || cfg->k <= 0) return 0;
+  return ws_layout(shape_of(cfg)).total;
+}
+
+int moe_get_error(void *ws, moe_stream_t stream, int32_t *code) {
+  if (!ws || !code) return MOE_ERR_INVALID_ARG;
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, err_word(ws), sizeof(int32_t), cudaMemcpyDeviceToHost, S(stream));
+  if (e == cudaSuccess) e = cudaMemsetAsync(err_word(ws), 0, sizeof(int32_t), S(stream));
+  if (e == cudaSuccess) e = cudaStreamSynchronize(S(stream));
+  if (e != cudaSuccess) return MOE_ERR_CUDA;
+  *code = h;
+  return MOE_OK;
+}
+
+int moe_route_topk(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
+                   float *logits, int32_t *topk_idx, float *topk_gate, void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs4({x, w_router, topk_idx, topk_gate}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  return cuda_rc(launch_route_topk(s, x, w_router, bias, logits, topk_idx, topk_gate, err_word(ws), S(stream)));
+}
+
+int moe_topk_gating(const moe_config *cfg, const float *logits, int32_t *topk_idx, float *topk_gate,
+                    void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs4({logits, topk_idx, topk_gate}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  return cuda_rc(launch_topk_gating(shape_of(cfg), logits, topk_idx, topk_gate, err_word(ws), S(stream)));
+}
+
+int moe_build_offsets(const moe_config *cfg, const int32_t *topk_idx, int32_t *counts, int32_t *offsets,
+                      int32_t *slot_of_pair, int32_t *pair_of_slot, void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  RETURN_IF(check_ptrs4({counts, offsets}));
+  if (cfg->T > 0) RETURN_IF(check_ptrs4({topk_idx, slot_of_pair, pair_of_slot}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  WsLayout L = ws_layout(s);
+  int32_t *bc = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.block_counts);
+  return cuda_rc(launch_build_offsets(s, topk_idx, counts, offsets, slot_of_pair, pair_of_slot, bc,
+                                      err_word(ws), S(stream)));
+}
+
+int moe_permute(const moe_config *cfg, const void *x, const int32_t *slot_of_pair, void *x_perm,
+                moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs({x, x_perm}));
+  RETURN_IF(check_ptrs4({slot_of_pair}));
+  return cuda_rc(launch_permute(shape_of(cfg), x, slot_of_pair, x_perm, S(stream)));
+}
+
+int moe_grouped_swiglu_fwd(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                           const void *w_gate, const void *w_up, const void *w_down, void *hu, void *a,
+                           void *y_perm, void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs({x_perm, w_gate, w_up, w_down, hu, a, y_perm}));
+  RETURN_IF(check_ptrs4({offsets}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  return launch_grouped_fwd(shape_of(cfg), x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws,
+                            S(stream));
+}
+
+int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, const void *x_perm, const void *hu,
+                           const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
+                           const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
+                           void *dw_down, void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  RETURN_IF(check_ptrs({w_gate, w_up, w_down, dw_gate, dw_up, dw_down}));
+  RETURN_IF(check_ptrs4({offsets}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  if (cfg->T == 0) {
+    // no routed rows: every expert's weight gradient is zero
+    size_t wb = (size_t)s.E * s.d * s.f * s.es();
+    cudaError_t e = cudaMemsetAsync(dw_gate, 0, wb, S(stream));
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_up, 0, wb, S(stream));
+    if (e == cudaSuccess) e = cudaMemsetAsync(dw_down, 0, wb, S(stream));
+    return cuda_rc(e);
+  }
+  RETURN_IF(check_ptrs({dy_perm, x_perm, hu, a, dhu, dx_perm}));
+  return launch_grouped_bwd(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
+                            dw_gate, dw_up, dw_down, err_word(ws), S(stream));
+}
+
+int moe_unpermute_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_of_pair,
+                          const float *topk_gate, void *y, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs({y_perm, y}));
+  RETURN_IF(check_ptrs4({slot_of_pair, topk_gate}));
+  return cuda_rc(launch_unpermute_combine(shape_of(cfg), y_perm, slot_of_pair, topk_gate, y, S(stream)));
+}
+
+int moe_combine_bwd(const moe_config *cfg, const void *dy, const void *y_perm, const int32_t *slot_of_pair,
+                    const float *topk_gate, void *dy_perm, float *dgate, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs({dy, y_perm, dy_perm}));
+  RETURN_IF(check_ptrs4({slot_of_pair, topk_gate, dgate}));
+  return cuda_rc(launch_combine_bwd(shape_of(cfg), dy, y_perm, slot_of_pair, topk_gate, dy_perm, dgate,
+                                    S(stream)));
+}
+
+int moe_unpermute_sum(const moe_config *cfg, const void *dx_perm, const int32_t *slot_of_pair, void *dx,
+                      moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(check_ptrs({dx_perm, dx}));
+  RETURN_IF(check_ptrs4({slot_of_pair}));
+  return cuda_rc(launch_unpermute_sum(shape_of(cfg), dx_perm, slot_of_pair, nullptr, nullptr, nullptr,
+                                      nullptr, false, dx, S(stream)));
+}
+
+int moe_route_bwd(const moe_config *cfg, const float *dgate, const float *topk_gate, const int32_t *topk_idx,
+                  const void *x, const void *w_router, void *dx, float *dw_router, void *ws,
+                  moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  RETURN_IF(check_ptrs4({w_router, dw_router}));
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  if (cfg->T > 0) {
+    RETURN_IF(check_ptrs4({dgate, topk_gate, topk_idx}));
+    RETURN_IF(check_ptrs({x, dx}));
+  }
+  WsLayout L = ws_layout(s);
+  char *w = static_cast<char *>(ws);
+  float *w_rt = reinterpret_cast<float *>(w + L.w_rt);
+  float *part = reinterpret_cast<float *>(w + L.dwr_partial);
+  RETURN_IF(cuda_rc(launch_router_transpose(s, w_router, w_rt, S(stream))));
+  RETURN_IF(cuda_rc(launch_router_wgrad(s, dgate, topk_gate, topk_idx, x, part, dw_router, S(stream))));
+  return cuda_rc(launch_unpermute_sum(s, nullptr, nullptr, dgate, topk_gate, topk_idx, w_rt, true, dx,
+                                      S(stream)));
+}
+
+static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
+                            const moe_layer_saved *sv, void *ws, moe_stream_t stream, bool route) {
+  RETURN_IF(check_cfg(cfg));
+  if (!w || !sv) return MOE_ERR_INVALID_ARG;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down}));
+  RETURN_IF(check_ptrs4({sv->counts, sv->offsets}));
+  if (route) RETURN_IF(check_ptrs4({w->w_router}));
+  if (cfg->T > 0) {
+    RETURN_IF(check_ptrs({x, y, sv->x_perm, sv->hu, sv->a, sv->y_perm}));
+    RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, sv->pair_of_slot}));
+  }
+  cudaStream_t st = S(stream);
+  int *err = err_word(ws);
+  WsLayout L = ws_layout(s);
+  int32_t *bc = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.block_counts);
+  if (route && cfg->T > 0)
+    RETURN_IF(cuda_rc(launch_route_topk(s, x, w->w_router, w->bias, sv->logits, sv->topk_idx, sv->topk_gate,
+                                        err, st)));
+  RETURN_IF(cuda_rc(launch_build_offsets(s, sv->topk_idx, sv->counts, sv->offsets, sv->slot_of_pair,
+                                         sv->pair_of_slot, bc, err, st)));
+  if (cfg->T == 0) return MOE_OK;
+  RETURN_IF(cuda_rc(launch_permute(s, x, sv->slot_of_pair, sv->x_perm, st)));
+  RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, sv->hu, sv->a,
+                               sv->y_perm, ws, st));
+  return cuda_rc(launch_unpermute_combine(s, sv->y_perm, sv->slot_of_pair, sv->topk_gate, y, st));
+}
+
+int moe_layer_fwd(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
+                  const moe_layer_saved *saved, void *ws, moe_stream_t stream) {
+  return layer_fwd_common(cfg, w, x, y, saved, ws, stream, true);
+}
+
+int moe_layer_fwd_routed(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
+                         const moe_layer_saved *saved, void *ws, moe_stream_t stream) {
+  return layer_fwd_common(cfg, w, x, y, saved, ws, stream, false);
+}
+
+int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void *x, const void *dy,
+                  const moe_layer_saved *sv, const moe_layer_grads *g, void *ws, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (!w || !sv || !g) return MOE_ERR_INVALID_ARG;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  Shape s = shape_of(cfg);
+  cudaStream_t st = S(stream);
+  int *err = err_word(ws);
+  const bool router = g->dw_router != nullptr;
+  RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down, g->dw_gate, g->dw_up, g->dw_down}));
+  RETURN_IF(check_ptrs4({sv->offsets}));
+  if (router) RETURN_IF(check_ptrs4({w->w_router, g->dw_router}));
+  if (cfg->T > 0) {
+    RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->hu, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
+    RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, g->dgate}));
+  }
+  if (cfg->T == 0) {
+    size_t wb = (size_t)s.E * s.d * s.f * s.es();
+    cudaError_t e = cudaMemsetAsync(g->dw_gate, 0, wb, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g->dw_up, 0, wb, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(g->dw_down, 0, wb, st);
+    if (e == cudaSuccess && router) e = cudaMemsetAsync(g->dw_router, 0, (size_t)s.d * s.E * 4, st);
+    return cuda_rc(e);
+  }
+  RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
+                                       g->dgate, st)));
+  RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, sv->hu, sv->a, sv->offsets, w->w_gate, w->w_up,
+                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, err, st));
+  if (!router)
+    return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, nullptr, nullptr, nullptr, nullptr,
+                                        false, g->dx, st));
+  WsLayout L = ws_layout(s);
+  char *wsc = static_cast<char *>(ws);
+  float *w_rt = reinterpret_cast<float *>(wsc + L.w_rt);
+  float *part = reinterpret_cast<float *>(wsc + L.dwr_partial);
+  RETURN_IF(cuda_rc(launch_router_transpose(s, w->w_router, w_rt, st)));
+  RETURN_IF(cuda_rc(launch_router_wgrad(s, g->dgate, sv->topk_gate, sv->topk_idx, x, part, g->dw_router, st)));
+  // dx = sum_j dx_perm[slot(t,j)] + dz W_r^T in one pass
+  return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, g->dgate, sv->topk_gate, sv->topk_idx,
+                                      w_rt, false, g->dx, st));
+}
+
+}  // extern "C"

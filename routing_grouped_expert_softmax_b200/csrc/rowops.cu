@@ -1,0 +1,388 @@
+// Row-wise, HBM-bound steps of the layer: rowwise dispatch (permute), gate-weighted
+// unpermute-combine, their backwards, and the router backward.
+//
+// Method: unite.ai "Ai2 κυκλοφορεί το Olmo-Core 3 ...", section "Παραλληλισμός,
+// Ακρίβεια και Τεχνικές Μνήμης" and ettayeb.fr "Olmo-core 3 ouvre l'entraînement des
+// MoE ...", section "Trois parallélismes, trois optimisations de routage": routed rows
+// are placed straight into each expert's contiguous input buffer.  The combine is the
+// inverse step, weighting each of a token's k expert outputs by its gate.
+//
+// Every kernel gives one warp to one token and moves its rows as 16-byte vectors
+// (8 bf16 or 4 fp32 per lane per access), so each row access is fully coalesced.
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int ROW_THREADS = 256;
+constexpr int ROW_WARPS = ROW_THREADS / 32;
+
+// Broadcast the k slots (and optionally gates) of token t to every lane.
+__device__ __forceinline__ int64_t lane_slot(const int32_t *sop, int64_t t, int k) {
+  int lane = threadIdx.x & 31;
+  return lane < k ? (int64_t)sop[t * k + lane] : 0;
+}
+
+// x_perm[slot(t,j)] = x[t]
+__global__ void __launch_bounds__(ROW_THREADS) permute_kernel(const uint4 *__restrict__ x,
+                                                              const int32_t *__restrict__ sop,
+                                                              uint4 *__restrict__ x_perm,
+                                                              int64_t T, int k, int nv) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int64_t my_slot = lane_slot(sop, t, k);
+  int64_t slot[MAX_K];
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j) slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+  const uint4 *src = x + t * nv;
+  for (int v0 = 0; v0 < nv; v0 += 32 * 4) {
+    uint4 buf[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      int v = v0 + u * 32 + lane;
+      if (v < nv) buf[u] = __ldg(src + v);
+    }
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+      if (j < k) {
+        uint4 *dst = x_perm + slot[j] * nv;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          int v = v0 + u * 32 + lane;
+          if (v < nv) dst[v] = buf[u];
+        }
+      }
+    }
+  }
+}
+
+// y[t] = sum_j g[t,j] * y_perm[slot(t,j)]   (fp32 accumulation)
+template <typename T>
+__global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__restrict__ y_perm,
+                                                              const int32_t *__restrict__ sop,
+                                                              const float *__restrict__ gate,
+                                                              uint4 *__restrict__ y, int64_t Tn,
+                                                              int k, int nv) {
+  constexpr int N = Vec<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+  if (t >= Tn) return;
+  int64_t my_slot = lane_slot(sop, t, k);
+  float my_g = lane < k ? gate[t * k + lane] : 0.f;
+  for (int v0 = 0; v0 < nv; v0 += 64) {
+    float acc[2][N];
+#pragma unroll
+    for (int u = 0; u < 2; ++u)
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+      if (j < k) {
+        int64_t slot = __shfl_sync(0xffffffffu, my_slot, j);
+        float g = __shfl_sync(0xffffffffu, my_g, j);
+        const uint4 *src = y_perm + slot * nv;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          int v = v0 + u * 32 + lane;
+          if (v < nv) {
+            float f[N];
+            Vec<T>::load(__ldg(src + v), f);
+#pragma unroll
+            for (int i = 0; i < N; ++i) acc[u][i] = fmaf(g, f[i], acc[u][i]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      int v = v0 + u * 32 + lane;
+      if (v < nv) y[t * nv + v] = Vec<T>::store(acc[u]);
+    }
+  }
+}
+
+// dy_perm[slot(t,j)] = g[t,j] dy[t];  dgate[t,j] = <dy[t], y_perm[slot(t,j)]>
+template <typename T>
+__global__ void __launch_bounds__(ROW_THREADS) combine_bwd_kernel(
+    const uint4 *__restrict__ dy, const uint4 *__restrict__ y_perm, const int32_t *__restrict__ sop,
+    const float *__restrict__ gate, uint4 *__restrict__ dy_perm, float *__restrict__ dgate,
+    int64_t Tn, int k, int nv) {
+  constexpr int N = Vec<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+  if (t >= Tn) return;
+  int64_t my_slot = lane_slot(sop, t, k);
+  float my_g = lane < k ? gate[t * k + lane] : 0.f;
+  int64_t slot[MAX_K];
+  float g[MAX_K], dot[MAX_K];
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j) {
+    slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    g[j] = __shfl_sync(0xffffffffu, my_g, j);
+    dot[j] = 0.f;
+  }
+  for (int v = lane; v < nv; v += 32) {
+    float fd[N];
+    Vec<T>::load(__ldg(dy + t * nv + v), fd);
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+      if (j < k) {
+        float fy[N], o[N];
+        Vec<T>::load(__ldg(y_perm + slot[j] * nv + v), fy);
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+          dot[j] = fmaf(fd[i], fy[i], dot[j]);
+          o[i] = g[j] * fd[i];
+        }
+        dy_perm[slot[j] * nv + v] = Vec<T>::store(o);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j) {
+    if (j < k) {
+      float s = dot[j];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) dgate[t * k + j] = s;
+    }
+  }
+}
+
+// dz_j = g_j (dg_j - sum_j' g_j' dg_j') for token t, computed by every lane.
+__device__ __forceinline__ void token_dz(const float *dgate, const float *gate, int64_t t, int k,
+                                         float (&dz)[MAX_K]) {
+  float inner = 0.f;
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j)
+    if (j < k) inner = fmaf(gate[t * k + j], dgate[t * k + j], inner);
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j)
+    dz[j] = (j < k) ? gate[t * k + j] * (dgate[t * k + j] - inner) : 0.f;
+}
+
+// dx[t] = [dx[t]] + sum_j dx_perm[slot(t,j)] + sum_j dz_j W_r^T[e_j]
+// (dx_perm / w_rt may each be null; accumulate reads the old dx)
+template <typename T>
+__global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
+    const uint4 *__restrict__ dx_perm, const int32_t *__restrict__ sop,
+    const float *__restrict__ dgate, const float *__restrict__ gate, const int32_t *__restrict__ idx,
+    const float *__restrict__ w_rt, bool accumulate, uint4 *__restrict__ dx, int64_t Tn, int k,
+    int nv, int d) {
+  constexpr int N = Vec<T>::N;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
+  if (t >= Tn) return;
+  int64_t slot[MAX_K];
+  int e[MAX_K];
+  float dz[MAX_K];
+  if (dx_perm) {
+    int64_t my_slot = lane_slot(sop, t, k);
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+  }
+  if (w_rt) {
+    token_dz(dgate, gate, t, k, dz);
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) e[j] = (j < k) ? idx[t * k + j] : 0;
+  }
+  for (int v = lane; v < nv; v += 32) {
+    float acc[N];
+    if (accumulate) {
+      Vec<T>::load(dx[t * nv + v], acc);
+    } else {
+#pragma unroll
+      for (int i = 0; i < N; ++i) acc[i] = 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+      if (j < k) {
+        if (dx_perm) {
+          float f[N];
+          Vec<T>::load(__ldg(dx_perm + slot[j] * nv + v), f);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[i] += f[i];
+        }
+        if (w_rt) {
+          const float *wr = w_rt + (int64_t)e[j] * d + (int64_t)v * N;
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[i] = fmaf(dz[j], __ldg(wr + i), acc[i]);
+        }
+      }
+    }
+    dx[t * nv + v] = Vec<T>::store(acc);
+  }
+}
+
+// w_rt[e][i] = W_r[i][e] (fp32), 32x32 tiles through shared memory.
+template <typename T>
+__global__ void router_transpose_kernel(const T *__restrict__ w_r, float *__restrict__ w_rt, int d,
+                                        int E) {
+  __shared__ float tile[32][33];
+  int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    int i = i0 + r, e = e0 + threadIdx.x;
+    tile[r][threadIdx.x] = (i < d && e < E) ? to_f(w_r[(int64_t)i * E + e]) : 0.f;
+  }
+  __syncthreads();
+  for (int r = threadIdx.y; r < 32; r += blockDim.y) {
+    int e = e0 + r, i = i0 + threadIdx.x;
+    if (e < E && i < d) w_rt[(int64_t)e * d + i] = tile[threadIdx.x][r];
+  }
+}
+
+// Router weight gradient, stage 1: partial[s][e][c] = sum over tokens of split s of
+// dz[t,e] x[t,c].  Thread c owns one column: no atomics, fixed summation order.
+constexpr int RW_COLS = 128;
+template <typename T>
+__global__ void __launch_bounds__(RW_COLS) router_wgrad_partial_kernel(
+    const float *__restrict__ dgate, const float *__restrict__ gate, const int32_t *__restrict__ idx,
+    const T *__restrict__ x, float *__restrict__ partial, int64_t Tn, int d, int E, int k) {
+  extern __shared__ float acc[];  // [E][RW_COLS]
+  const int c = blockIdx.x * RW_COLS + threadIdx.x;
+  for (int i = threadIdx.x; i < E * RW_COLS; i += RW_COLS) acc[i] = 0.f;
+  __syncthreads();
+  const int64_t per = (Tn + RB_SPLIT - 1) / RB_SPLIT;
+  const int64_t tb = (int64_t)blockIdx.y * per;
+  const int64_t te = min(Tn, tb + per);
+  if (c < d) {
+    for (int64_t t = tb; t < te; ++t) {
+      float dz[MAX_K];
+      token_dz(dgate, gate, t, k, dz);
+      float xv = to_f(x[t * d + c]);
+#pragma unroll
+      for (int j = 0; j < MAX_K; ++j)
+        if (j < k) acc[idx[t * k + j] * RW_COLS + threadIdx.x] += dz[j] * xv;
+    }
+  }
+  __syncthreads();
+  float *out = partial + (int64_t)blockIdx.y * E * d;
+  if (c < d)
+    for (int e = 0; e < E; ++e) out[(int64_t)e * d + c] = acc[e * RW_COLS + threadIdx.x];
+}
+
+// Stage 2: dW_r[c][e] = sum_s partial[s][e][c], in split order.
+__global__ void router_wgrad_reduce_kernel(const float *__restrict__ partial, float *__restrict__ dw_r,
+                                           int d, int E) {
+  int64_t n = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= (int64_t)d * E) return;
+  int e = (int)(n / d), c = (int)(n % d);
+  float s = 0.f;
+  for (int sp = 0; sp < RB_SPLIT; ++sp) s += partial[(int64_t)sp * E * d + n];
+  dw_r[(int64_t)c * E + e] = s;
+}
+
+// dst[b][c][r] = src[b][r][c], 32x32 tiles through shared memory.
+__global__ void transpose_batched_kernel(const float *__restrict__ src, float *__restrict__ dst, int R,
+                                         int C) {
+  __shared__ float tile[32][33];
+  const int64_t b = blockIdx.z;
+  const float *s = src + b * R * C;
+  float *d = dst + b * R * C;
+  int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int r = r0 + i, c = c0 + threadIdx.x;
+    if (r < R && c < C) tile[i][threadIdx.x] = s[(int64_t)r * C + c];
+  }
+  __syncthreads();
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    int c = c0 + i, r = r0 + threadIdx.x;
+    if (r < R && c < C) d[(int64_t)c * R + r] = tile[threadIdx.x][i];
+  }
+}
+
+cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st) {
+  dim3 grid((C + 31) / 32, (R + 31) / 32, B), block(32, 8);
+  transpose_batched_kernel<<<grid, block, 0, st>>>(src, dst, R, C);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------ launchers
+static unsigned row_grid(int64_t T) { return (unsigned)((T + ROW_WARPS - 1) / ROW_WARPS); }
+
+cudaError_t launch_permute(const Shape &s, const void *x, const int32_t *sop, void *x_perm,
+                           cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  int nv = s.d * s.es() / 16;
+  permute_kernel<<<row_grid(s.T), ROW_THREADS, 0, st>>>(static_cast<const uint4 *>(x), sop,
+                                                        static_cast<uint4 *>(x_perm), s.T, s.k, nv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const int32_t *sop,
+                                     const float *gate, void *y, cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  int nv = s.d * s.es() / 16;
+  auto yp = static_cast<const uint4 *>(y_perm);
+  auto yo = static_cast<uint4 *>(y);
+  if (s.dtype == MOE_BF16)
+    combine_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv);
+  else
+    combine_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm, const int32_t *sop,
+                               const float *gate, void *dy_perm, float *dgate, cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  int nv = s.d * s.es() / 16;
+  auto a = static_cast<const uint4 *>(dy);
+  auto b = static_cast<const uint4 *>(y_perm);
+  auto o = static_cast<uint4 *>(dy_perm);
+  if (s.dtype == MOE_BF16)
+    combine_bwd_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, b, sop, gate, o, dgate, s.T, s.k, nv);
+  else
+    combine_bwd_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, b, sop, gate, o, dgate, s.T, s.k, nv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int32_t *sop,
+                                 const float *dgate, const float *gate, const int32_t *idx,
+                                 const float *w_rt, bool accumulate, void *dx, cudaStream_t st) {
+  if (s.T == 0) return cudaSuccess;
+  int nv = s.d * s.es() / 16;
+  auto a = static_cast<const uint4 *>(dx_perm);
+  auto o = static_cast<uint4 *>(dx);
+  if (s.dtype == MOE_BF16)
+    unpermute_sum_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w_rt,
+                                                                      accumulate, o, s.T, s.k, nv, s.d);
+  else
+    unpermute_sum_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w_rt,
+                                                                       accumulate, o, s.T, s.k, nv, s.d);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_transpose(const Shape &s, const void *w_r, float *w_rt, cudaStream_t st) {
+  dim3 grid((s.d + 31) / 32, (s.E + 31) / 32), block(32, 8);
+  if (s.dtype == MOE_BF16)
+    router_transpose_kernel<bf16><<<grid, block, 0, st>>>(static_cast<const bf16 *>(w_r), w_rt, s.d, s.E);
+  else
+    router_transpose_kernel<float><<<grid, block, 0, st>>>(static_cast<const float *>(w_r), w_rt, s.d, s.E);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
+                                const int32_t *idx, const void *x, float *partial, float *dw_r,
+                                cudaStream_t st) {
+  size_t smem = (size_t)s.E * RW_COLS * sizeof(float);
+  dim3 grid((s.d + RW_COLS - 1) / RW_COLS, RB_SPLIT);
+  cudaError_t e;
+  if (s.dtype == MOE_BF16) {
+    e = cudaFuncSetAttribute(router_wgrad_partial_kernel<bf16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    router_wgrad_partial_kernel<bf16><<<grid, RW_COLS, smem, st>>>(
+        dgate, gate, idx, static_cast<const bf16 *>(x), partial, s.T, s.d, s.E, s.k);
+  } else {
+    e = cudaFuncSetAttribute(router_wgrad_partial_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    router_wgrad_partial_kernel<float><<<grid, RW_COLS, smem, st>>>(
+        dgate, gate, idx, static_cast<const float *>(x), partial, s.T, s.d, s.E, s.k);
+  }
+  int64_t n = (int64_t)s.d * s.E;
+  router_wgrad_reduce_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(partial, dw_r, s.d, s.E);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

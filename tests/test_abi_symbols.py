@@ -1,0 +1,74 @@
+"""The C-ABI library loads and exports every symbol include/moe.h declares; host-side
+argument validation rejects bad calls before any CUDA call (CPU only, no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import routing_grouped_expert_softmax_b200 as moe
+from routing_grouped_expert_softmax_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+\w+\s+(moe_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    moe_build.build()
+    return moe.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(moe.EXPORTED) == names
+
+
+def test_workspace_size_is_host_only(lib):
+    cfg = moe.config(8192, 2048, 128, 4, 1024)
+    ws = moe.moe_workspace_size(cfg)
+    assert ws >= 256 and ws % 256 == 0
+    assert moe.moe_workspace_size(moe.config(0, 128, 8, 2, 256)) >= 256
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=-1), dict(d=0), dict(E=0), dict(k=0), dict(f=-5), dict(dtype=7), dict(prec=9),
+])
+def test_invalid_config_rejected(lib, bad):
+    base = dict(T=16, d=128, E=8, k=2, f=128, dtype=moe.MOE_BF16, prec=moe.MOE_PREC_NATIVE)
+    base.update(bad)
+    cfg = moe.MoeConfig(**base)
+    rc = lib.moe_permute(ctypes.byref(cfg), 16, 16, 16, None)
+    assert rc == moe.MOE_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bad", [dict(E=257), dict(k=9), dict(k=9, E=8), dict(d=192), dict(f=200),
+                                 dict(prec=moe.MOE_PREC_MXFP8)])
+def test_unsupported_config_rejected(lib, bad):
+    base = dict(T=16, d=128, E=8, k=2, f=128, dtype=moe.MOE_BF16, prec=moe.MOE_PREC_NATIVE)
+    base.update(bad)
+    cfg = moe.MoeConfig(**base)
+    assert lib.moe_permute(ctypes.byref(cfg), 16, 16, 16, None) == moe.MOE_ERR_UNSUPPORTED
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    cfg = moe.config(16, 128, 8, 2, 128)
+    assert lib.moe_permute(ctypes.byref(cfg), None, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute(ctypes.byref(cfg), 16, 16, 24, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_build_offsets(ctypes.byref(cfg), 16, 16, 16, 16, 16, None, None) == moe.MOE_ERR_WORKSPACE
+    code = ctypes.c_int32()
+    assert lib.moe_get_error(None, None, ctypes.byref(code)) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_empty_batch_launches_nothing(lib):
+    # T = 0 returns MOE_OK before any launch, so it is valid even without a GPU
+    cfg = moe.config(0, 128, 8, 2, 128)
+    assert lib.moe_permute(ctypes.byref(cfg), None, None, None, None) == moe.MOE_OK
+    assert lib.moe_unpermute_combine(ctypes.byref(cfg), None, None, None, None, None) == moe.MOE_OK

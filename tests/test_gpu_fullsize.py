@@ -1,0 +1,151 @@
+"""Parity at the benchmark's full sizes, in the launch configuration bench.py times
+(moe_layer_fwd + moe_layer_bwd on one stream):
+
+  * E=8:   T=8192, d=2048, k=4, ffn=1024 (near-uniform load)
+  * E=128: T=8192, d=2048, k=4, ffn=1024
+  * E=128: T=16384 with the Zipf-like logit bias, and with uniform random routing
+
+The whole-tensor oracle is too slow here, so the checks are (a) properties that hold at
+any size (routing and metadata invariants, exact permute), (b) oracle values computed one
+token at a time (y and dx of sampled tokens) or one expert at a time (the weight
+gradients of sampled experts), each from the oracle's own routing of those tokens.
+"""
+import numpy as np
+import pytest
+
+import routing_grouped_expert_softmax_b200 as moe
+from oracle import moe_ref as ref
+from routing_grouped_expert_softmax_b200 import inputs as gen
+from tests.gpu_util import dev, dev_f32, host, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-2
+TOL_COMBINE = 1e-2
+
+CONFIGS = {
+    "e8": dict(T=8192, d=2048, E=8, k=4, f=1024, skew=False, routing="router"),
+    "e128": dict(T=8192, d=2048, E=128, k=4, f=1024, skew=False, routing="router"),
+    "e128_t16k_skew": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=True, routing="router"),
+    "e128_t16k_uniform": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=False, routing="uniform"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    import torch
+    assert torch.cuda.is_available()
+    from routing_grouped_expert_softmax_b200 import build
+    build.build()
+
+
+def _token_oracle(inp, t, idx_t, g_t, router):
+    """Oracle y[t] and dx[t] of one token from its routing (experts idx_t, gates g_t)."""
+    x = inp.x[t:t + 1].astype(np.float64)
+    dY = inp.dy[t].astype(np.float64)
+    y = np.zeros(inp.d)
+    dx = np.zeros(inp.d)
+    dg = np.zeros(len(idx_t))
+    for j, e in enumerate(idx_t):
+        h, u, a, ye = ref.expert_swiglu(x, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+        y += g_t[j] * ye[0]
+        dg[j] = dY @ ye[0]
+        da = (g_t[j] * dY)[None, :] @ inp.w_down[e].astype(np.float64).T
+        dh, du = ref.swiglu_bwd(da, h, u)
+        dx += (dh @ inp.w_gate[e].astype(np.float64).T + du @ inp.w_up[e].astype(np.float64).T)[0]
+    if router:
+        dz = ref.gate_logit_grad(dg[None, :], np.asarray(g_t)[None, :], np.asarray(idx_t)[None, :], inp.E)
+        dx += (dz @ inp.w_r.astype(np.float64).T)[0]
+    return y, dx
+
+
+def _expert_oracle(inp, e, idx, gate):
+    """Oracle weight gradients of expert e from the routing of every token."""
+    pairs = np.nonzero(idx.ravel() == e)[0]           # pair order = the stable slot order
+    toks = pairs // inp.k
+    g = gate.ravel()[pairs].astype(np.float64)
+    X = inp.x[toks].astype(np.float64)
+    h, u, a, _ = ref.expert_swiglu(X, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+    dy = g[:, None] * inp.dy[toks].astype(np.float64)
+    da = dy @ inp.w_down[e].astype(np.float64).T
+    dh, du = ref.swiglu_bwd(da, h, u)
+    return X.T @ dh, X.T @ du, a.T @ dy
+
+
+@pytest.mark.parametrize("name", list(CONFIGS))
+def test_fullsize(name):
+    import torch
+    c = CONFIGS[name]
+    T, d, E, k, f = c["T"], c["d"], c["E"], c["k"], c["f"]
+    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=0, skew=c["skew"])
+    cfg = moe.config(T, d, E, k, f, dtype="bf16")
+    ws = moe.alloc_workspace(cfg)
+    saved = moe.alloc_saved(cfg)
+    router = c["routing"] == "router"
+    grads = moe.alloc_grads(cfg, router=router)
+    w = [dev(a, "bf16") for a in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down)]
+    bias = dev_f32(inp.bias) if inp.bias is not None else None
+    wts = moe.layer_weights(w[0], bias, w[1], w[2], w[3])
+    x = dev(inp.x, "bf16")
+    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+    if router:
+        moe.moe_layer_fwd(cfg, wts, x, y, saved, ws)
+    else:
+        ridx, rgate = gen.uniform_random_routing(T, E, k, seed=0)
+        saved["topk_idx"].copy_(torch.from_numpy(ridx))
+        saved["topk_gate"].copy_(torch.from_numpy(rgate))
+        moe.moe_layer_fwd_routed(cfg, wts, x, y, saved, ws)
+    moe.moe_layer_bwd(cfg, wts, x, dev(inp.dy, "bf16"), saved, grads, ws)
+    assert moe.moe_get_error(ws) == 0
+
+    # (a) invariants at any size
+    gi = host(saved["topk_idx"]).astype(np.int64)
+    gg = host(saved["topk_gate"])
+    counts, offsets = host(saved["counts"]), host(saved["offsets"])
+    sop, pos = host(saved["slot_of_pair"]).astype(np.int64), host(saved["pair_of_slot"]).astype(np.int64)
+    assert gi.min() >= 0 and gi.max() < E
+    assert all(len(set(r)) == k for r in gi[:: max(1, T // 512)])
+    np.testing.assert_allclose(gg.sum(axis=1), 1.0, atol=1e-5)
+    assert np.all(np.diff(gg, axis=1) <= 1e-7)
+    assert counts.sum() == T * k and offsets[0] == 0 and np.array_equal(offsets[1:], np.cumsum(counts))
+    assert np.array_equal(counts, np.bincount(gi.ravel(), minlength=E))
+    assert np.array_equal(pos[sop], np.arange(T * k))
+    assert np.array_equal(pos, np.argsort(gi.ravel(), kind="stable"))
+    xp = host(saved["x_perm"])
+    rows = np.random.default_rng(1).choice(T * k, size=256, replace=False)
+    assert np.array_equal(xp[rows], inp.x[pos[rows] // k])
+    load = counts / counts.mean()
+    print(f"{name}: max/mean expert load {load.max():.3f}, empty experts {(counts == 0).sum()}")
+
+    # (b) oracle routing, then sampled tokens
+    if router:
+        z, p, ridx, rgate = ref.route(inp.x, inp.w_r, k, inp.bias)
+        bound = d * 2.0 ** -24 * (np.abs(inp.x.astype(np.float64)) @ np.abs(inp.w_r.astype(np.float64)))
+        zs = np.sort(z, axis=1)[:, ::-1]
+        clear = (zs[:, k - 1] - zs[:, k]) > 2 * bound.max(axis=1)
+        assert clear.mean() > 0.99
+        assert np.array_equal(gi[clear], ridx[clear])
+        print(f"{name}: {(~clear).sum()} near-tie tokens of {T}; "
+              f"routing flips among them: {(gi[~clear] != ridx[~clear]).any(axis=1).sum()}")
+    else:
+        ridx, rgate, clear = ridx.astype(np.int64), rgate.astype(np.float64), np.ones(T, bool)
+    rng = np.random.default_rng(2)
+    toks = rng.choice(np.nonzero(clear)[0], size=24, replace=False)
+    gy, gdx = host(y), host(grads["dx"])
+    ys, dxs = [], []
+    for t in toks:
+        yt, dxt = _token_oracle(inp, t, ridx[t], rgate[t], router)
+        ys.append(yt)
+        dxs.append(dxt)
+    assert rel_err(gy[toks], np.array(ys)) <= TOL_COMBINE
+    assert rel_err(gdx[toks], np.array(dxs)) <= TOL
+
+    # sampled experts' weight gradients (only experts all of whose tokens route clearly)
+    touch = (ridx[:, :, None] == np.arange(E)).any(axis=1) | (gi[:, :, None] == np.arange(E)).any(axis=1)
+    owners = [e for e in range(E) if clear[touch[:, e]].all()]
+    picks = [owners[0], owners[len(owners) // 2], owners[-1]] if E > 8 else owners[:1]
+    for e in picks:
+        dwg, dwu, dwd = _expert_oracle(inp, e, ridx, rgate)
+        assert rel_err(host(grads["dw_gate"][e]), dwg) <= TOL, e
+        assert rel_err(host(grads["dw_up"][e]), dwu) <= TOL, e
+        assert rel_err(host(grads["dw_down"][e]), dwd) <= TOL, e
