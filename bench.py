@@ -63,7 +63,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
         except (FileNotFoundError, OSError):
@@ -74,7 +74,10 @@ class ClockSampler:
         for line in self.proc.stdout:
             parts = [s.strip() for s in line.split(",")]
             if len(parts) >= 7:
-                self.samples.append(parts)
+                self.samples.append((time.time(), parts))
+
+    def window(self, t0, t1):
+        self.t0, self.t1 = t0, t1
 
     def __exit__(self, *a):
         if self.proc:
@@ -85,14 +88,22 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        t0, t1 = getattr(self, "t0", 0.0), getattr(self, "t1", 1e30)
+        rows = [p for (t, p) in self.samples if t0 <= t <= t1 + 0.15]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[0]) for r in rows) if v is not None]
+        mx = [v for v in (num(r[1]) for r in rows) if v is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4) if s[3 + i] == "Active"})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[3 + i] == "Active"})
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+                "reasons": reasons, "samples": len(rows)}
 
 
 def dist_env():
@@ -152,25 +163,30 @@ def run_ours(args):
         fwd_fn(cfg, w, x, y, saved, ws, st)
         moe.moe_layer_bwd(cfg, w, x, dy, saved, grads, ws, st)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    assert moe.moe_get_error(ws) == 0
-
     def barrier():
         if ws_n > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
+    clk = ClockSampler(local)
+    clk.__enter__()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert moe.moe_get_error(ws) == 0
+    time.sleep(0.3)     # let the sampler start reporting before the timed region
+
     # ---- headline: K whole steps, device-timed with CUDA events on the launching stream
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
-    with ClockSampler(local) as clk:
-        e0.record(st)
-        for _ in range(args.steps):
-            step()
-        e1.record(st)
-        barrier()
+    t_start = time.time()
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    barrier()
+    clk.window(t_start, time.time())
+    clk.__exit__()
     ms = e0.elapsed_time(e1) / args.steps
     ms_max = ms
     if ws_n > 1:
@@ -308,10 +324,14 @@ def run_reference(args):
     T, d, E, k, f, skew, routing = WORKLOADS[name]
     inp = make_inputs(name, seed=0)
     from oracle import moe_ref as ref
-    n = args.cpu_tokens
+    # size each step's token sample so that the K timed steps take about two minutes
+    probe = 16
+    t0 = time.perf_counter()
+    fwd = ref.layer_fwd(inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+    ref.layer_bwd(fwd, inp.dy[:probe], inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
+    t_probe = time.perf_counter() - t0
+    n = int(max(4, min(args.cpu_tokens, probe * (120.0 / max(args.steps, 1)) / max(t_probe, 1e-3))))
     xs, dys = inp.x[:n], inp.dy[:n]
-    for _ in range(min(args.warmup, 1)):
-        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
@@ -340,11 +360,11 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
-    ap.add_argument("--cpu-tokens", type=int, default=32)
+    ap.add_argument("--cpu-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

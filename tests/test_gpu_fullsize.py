@@ -39,6 +39,13 @@ def _gpu():
     build.build()
 
 
+def clear_tokens(z, delta, k):
+    """Tokens whose top-(k+1) logits are pairwise separated by more than 2*delta."""
+    zs = np.sort(z, axis=1)[:, ::-1][:, :k + 1]
+    gaps = -np.diff(zs, axis=1)
+    return np.all(gaps > 2 * delta[:, None], axis=1)
+
+
 def _token_oracle(inp, t, idx_t, g_t, router):
     """Oracle y[t] and dx[t] of one token from its routing (experts idx_t, gates g_t)."""
     x = inp.x[t:t + 1].astype(np.float64)
@@ -120,9 +127,13 @@ def test_fullsize(name):
     # (b) oracle routing, then sampled tokens
     if router:
         z, p, ridx, rgate = ref.route(inp.x, inp.w_r, k, inp.bias)
+        # the logits are checked against the rigorous fp32 dot-product bound ...
         bound = d * 2.0 ** -24 * (np.abs(inp.x.astype(np.float64)) @ np.abs(inp.w_r.astype(np.float64)))
-        zs = np.sort(z, axis=1)[:, ::-1]
-        clear = (zs[:, k - 1] - zs[:, k]) > 2 * bound.max(axis=1)
+        zg = host(saved["logits"])
+        assert np.all(np.abs(zg - z) <= bound + 2.0 ** -24 * np.abs(z) + 1e-30)
+        # ... and a token's routing is fixed wherever every gap among its k+1 largest oracle
+        # logits exceeds twice that token's largest logit error: then the order must agree
+        clear = clear_tokens(z, np.max(np.abs(zg - z), axis=1), k)
         assert clear.mean() > 0.99
         assert np.array_equal(gi[clear], ridx[clear])
         print(f"{name}: {(~clear).sum()} near-tie tokens of {T}; "
