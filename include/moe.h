@@ -125,6 +125,23 @@ MOE_API int moe_build_offsets(const moe_config *cfg, const int32_t *topk_idx, in
                       int32_t *offsets, int32_t *slot_of_pair, int32_t *pair_of_slot,
                       void *ws, moe_stream_t stream);
 
+/* moe_build_offsets without a workspace, for callers that cannot allocate device memory
+ * (for example a program that gives all GPU memory to its own pool at start-up, or a C
+ * caller with no allocator of its own).  Same outputs as moe_build_offsets.
+ * (The pages have no counterpart: this is a calling convention, not a step of the method.)
+ *   Scratch: a fixed 256 KiB array inside the library, held on every GPU that loads the
+ *   library until the process exits; it must hold ceil(T*k/1024) * E int32 histogram
+ *   entries, so larger shapes return MOE_ERR_UNSUPPORTED (e.g. T*k = 262144 at E = 256).
+ *   The first call made with a given device current looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call shares the one array: calls whose work can overlap on the GPU (different
+ *   streams, different host threads) race and must be ordered by the caller.
+ *   An expert index outside [0, E) leaves the outputs undefined and is not reported.
+ *   Allocates nothing (no cudaMalloc, cudaFree or allocating library call). */
+MOE_API int moe_build_offsets_noalloc(const moe_config *cfg, const int32_t *topk_idx,
+                                      int32_t *counts, int32_t *offsets, int32_t *slot_of_pair,
+                                      int32_t *pair_of_slot, moe_stream_t stream);
+
 /* Rowwise dispatch: x_perm[slot_of_pair[t*k+j]] = x[t] (a bit copy).
  *   x [T,d] dtype; slot_of_pair [P]; x_perm [P,d] dtype. */
 MOE_API int moe_permute(const moe_config *cfg, const void *x, const int32_t *slot_of_pair,

@@ -33,7 +33,7 @@ MOE_PREC_MXFP8 = 1
 
 EXPORTED = [
     "moe_workspace_size", "moe_get_error", "moe_route_topk", "moe_topk_gating",
-    "moe_build_offsets", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
+    "moe_build_offsets", "moe_build_offsets_noalloc", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
     "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd",
 ]
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
             "moe_route_topk": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]),
             "moe_topk_gating": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
             "moe_build_offsets": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
+            "moe_build_offsets_noalloc": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P]),
             "moe_permute": (ctypes.c_int, [_CFG, _P, _P, _P, _P]),
             "moe_grouped_swiglu_fwd": (ctypes.c_int, [_CFG] + [_P] * 10),
             "moe_grouped_swiglu_bwd": (ctypes.c_int, [_CFG] + [_P] * 15),
@@ -167,6 +168,14 @@ def moe_topk_gating(cfg, logits, topk_idx, topk_gate, ws, stream=None):
 def moe_build_offsets(cfg, topk_idx, counts, offsets, slot_of_pair, pair_of_slot, ws, stream=None):
     _call("moe_build_offsets", ctypes.byref(cfg), ptr(topk_idx), ptr(counts), ptr(offsets),
           ptr(slot_of_pair), ptr(pair_of_slot), ptr(ws), stream_handle(stream))
+
+
+def moe_build_offsets_noalloc(cfg, topk_idx, counts, offsets, slot_of_pair, pair_of_slot,
+                              stream=None):
+    """moe_build_offsets with its scratch inside the library: for callers that cannot
+    allocate a workspace.  Calls that may overlap on the GPU must be ordered."""
+    _call("moe_build_offsets_noalloc", ctypes.byref(cfg), ptr(topk_idx), ptr(counts), ptr(offsets),
+          ptr(slot_of_pair), ptr(pair_of_slot), stream_handle(stream))
 
 
 def moe_permute(cfg, x, slot_of_pair, x_perm, stream=None):
