@@ -41,6 +41,8 @@ struct WsLayout {
   size_t w_rt;           // fp32 [E][d]   (transposed router weight)
   size_t dwr_partial;    // fp32 [RB_SPLIT][E][d]
   size_t wt;             // fp32 storage only: Wg^T, Wu^T [E][f][d] and Wd^T [E][d][f]
+  size_t dz_slot;        // fp32 [P]: router logit gradient of the pair in each slot
+  size_t rg_partial;     // fp32 [P/64 + E][d]: per-chunk router weight-gradient sums
   size_t total;
 };
 constexpr int RB_SPLIT = 16;          // token splits of the router weight-gradient reduction
@@ -56,6 +58,8 @@ inline WsLayout ws_layout(const Shape &s) {
   L.dwr_partial = off;  off = align_up(off + (size_t)RB_SPLIT * s.E * s.d * 4, 256);
   L.wt = off;
   if (s.dtype == MOE_F32) off = align_up(off + (size_t)3 * s.E * s.d * s.f * 4, 256);
+  L.dz_slot = off;      off = align_up(off + (size_t)s.P() * 4, 256);
+  L.rg_partial = off;   off = align_up(off + (size_t)((s.P() + 63) / 64 + s.E) * s.d * 4, 256);
   L.total = off;
   return L;
 }
@@ -121,6 +125,10 @@ cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int3
                                  const float *dgate, const float *gate, const int32_t *idx,
                                  const float *w_rt, bool accumulate, void *dx, cudaStream_t st);
 cudaError_t launch_router_transpose(const Shape &s, const void *w_r, float *w_rt, cudaStream_t st);
+// dW_r from the expert-contiguous rows x_perm and the slot maps (layer backward)
+cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, const int32_t *pos,
+                                        const int32_t *offsets, const float *dgate, const float *gate,
+                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st);
 cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
                                 const int32_t *idx, const void *x, float *partial,
                                 float *dw_r, cudaStream_t st);

@@ -244,6 +244,7 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down, g->dw_gate, g->dw_up, g->dw_down}));
   RETURN_IF(check_ptrs4({sv->offsets}));
   if (router) RETURN_IF(check_ptrs4({w->w_router, g->dw_router}));
+  if (router && cfg->T > 0) RETURN_IF(check_ptrs4({sv->pair_of_slot}));
   if (cfg->T > 0) {
     RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->hu, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
     RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, g->dgate}));
@@ -266,9 +267,11 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   WsLayout L = ws_layout(s);
   char *wsc = static_cast<char *>(ws);
   float *w_rt = reinterpret_cast<float *>(wsc + L.w_rt);
-  float *part = reinterpret_cast<float *>(wsc + L.dwr_partial);
   RETURN_IF(cuda_rc(launch_router_transpose(s, w->w_router, w_rt, st)));
-  RETURN_IF(cuda_rc(launch_router_wgrad(s, g->dgate, sv->topk_gate, sv->topk_idx, x, part, g->dw_router, st)));
+  RETURN_IF(cuda_rc(launch_router_wgrad_grouped(s, sv->x_perm, sv->pair_of_slot, sv->offsets, g->dgate,
+                                                sv->topk_gate, reinterpret_cast<float *>(wsc + L.dz_slot),
+                                                reinterpret_cast<float *>(wsc + L.rg_partial), g->dw_router,
+                                                st)));
   // dx = sum_j dx_perm[slot(t,j)] + dz W_r^T in one pass
   return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, g->dgate, sv->topk_gate, sv->topk_idx,
                                       w_rt, false, g->dx, st));

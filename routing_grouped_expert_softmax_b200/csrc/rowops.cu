@@ -204,9 +204,15 @@ __global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
           for (int i = 0; i < N; ++i) acc[i] += f[i];
         }
         if (w_rt) {
-          const float *wr = w_rt + (int64_t)e[j] * d + (int64_t)v * N;
+          const float4 *wr = reinterpret_cast<const float4 *>(w_rt + (int64_t)e[j] * d + (int64_t)v * N);
 #pragma unroll
-          for (int i = 0; i < N; ++i) acc[i] = fmaf(dz[j], __ldg(wr + i), acc[i]);
+          for (int i = 0; i < N / 4; ++i) {
+            float4 q = __ldg(wr + i);
+            acc[4 * i] = fmaf(dz[j], q.x, acc[4 * i]);
+            acc[4 * i + 1] = fmaf(dz[j], q.y, acc[4 * i + 1]);
+            acc[4 * i + 2] = fmaf(dz[j], q.z, acc[4 * i + 2]);
+            acc[4 * i + 3] = fmaf(dz[j], q.w, acc[4 * i + 3]);
+          }
         }
       }
     }
@@ -294,6 +300,133 @@ __global__ void transpose_batched_kernel(const float *__restrict__ src, float *_
 cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st) {
   dim3 grid((C + 31) / 32, (R + 31) / 32, B), block(32, 8);
   transpose_batched_kernel<<<grid, block, 0, st>>>(src, dst, R, C);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------------------
+// Router weight gradient from the expert-contiguous rows (layer backward):
+//   dW_r[c][e] = sum over slots s of expert e of dz(s) * x_perm[s][c],
+// where dz(s) is the logit gradient of the pair in slot s.  The rows of every expert are
+// cut into chunks of RG_ROWS; chunk q covers rows of one expert only, so its partial sum
+// belongs to that expert; a second kernel adds an expert's chunks in order.
+// ---------------------------------------------------------------------------------------
+constexpr int RG_ROWS = 64;
+constexpr int RG_THREADS = 128;  // x 2 columns = 256 columns per block
+
+// dz_slot[s] = g (dg - sum_j' g_j' dg_j') of the pair in slot s
+__global__ void router_dz_slot_kernel(const int32_t *__restrict__ pos, const float *__restrict__ dgate,
+                                      const float *__restrict__ gate, float *__restrict__ dz_slot,
+                                      int64_t P, int k) {
+  int64_t s = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (s >= P) return;
+  int64_t p = pos[s];
+  int64_t t = p / k;
+  float inner = 0.f;
+  for (int j = 0; j < k; ++j) inner = fmaf(gate[t * k + j], dgate[t * k + j], inner);
+  dz_slot[s] = gate[p] * (dgate[p] - inner);
+}
+
+// Exclusive prefix over experts of ceil(count_e / RG_ROWS), one warp; returns the total.
+__device__ int chunk_prefix(const int32_t *offsets, int E, int *prefix) {
+  const int lane = threadIdx.x & 31;
+  int cnt[8], sum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int e = lane * 8 + i;
+    cnt[i] = (e < E) ? (offsets[e + 1] - offsets[e] + RG_ROWS - 1) / RG_ROWS : 0;
+    sum += cnt[i];
+  }
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  int run = incl - sum;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    int e = lane * 8 + i;
+    if (e < E) prefix[e] = run;
+    run += cnt[i];
+  }
+  if (lane == 31) prefix[E] = incl;
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(RG_THREADS) router_wgrad_grouped_kernel(
+    const T *__restrict__ x_perm, const float *__restrict__ dz_slot, const int32_t *__restrict__ offsets,
+    float *__restrict__ partial, int E, int d) {
+  __shared__ int prefix[MAX_E + 1];
+  if (threadIdx.x < 32) chunk_prefix(offsets, E, prefix);
+  __syncthreads();
+  const int q = blockIdx.x;
+  if (q >= prefix[E]) return;
+  int lo = 0, hi = E;  // prefix[lo] <= q < prefix[hi]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= q) lo = mid; else hi = mid;
+  }
+  const int e = lo;
+  const int r0 = offsets[e] + (q - prefix[e]) * RG_ROWS;
+  const int r1 = min(offsets[e + 1], r0 + RG_ROWS);
+  const int c = (blockIdx.y * RG_THREADS + threadIdx.x) * 2;
+  if (c >= d) return;
+  float a0 = 0.f, a1 = 0.f;
+  int r = r0;
+  for (; r + 4 <= r1; r += 4) {
+    float z[4], x0[4], x1[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      z[u] = dz_slot[r + u];
+      x0[u] = to_f(x_perm[(int64_t)(r + u) * d + c]);
+      x1[u] = to_f(x_perm[(int64_t)(r + u) * d + c + 1]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      a0 = fmaf(z[u], x0[u], a0);
+      a1 = fmaf(z[u], x1[u], a1);
+    }
+  }
+  for (; r < r1; ++r) {
+    float z = dz_slot[r];
+    a0 = fmaf(z, to_f(x_perm[(int64_t)r * d + c]), a0);
+    a1 = fmaf(z, to_f(x_perm[(int64_t)r * d + c + 1]), a1);
+  }
+  partial[(int64_t)q * d + c] = a0;
+  partial[(int64_t)q * d + c + 1] = a1;
+}
+
+// dW_r[c][e] = sum of expert e's chunk partials, in chunk order (0 for an empty expert).
+__global__ void router_wgrad_grouped_reduce_kernel(const float *__restrict__ partial,
+                                                   const int32_t *__restrict__ offsets,
+                                                   float *__restrict__ dw_r, int E, int d) {
+  __shared__ int prefix[MAX_E + 1];
+  if (threadIdx.x < 32) chunk_prefix(offsets, E, prefix);
+  __syncthreads();
+  const int e = blockIdx.y;
+  const int c = blockIdx.x * blockDim.x + threadIdx.x;
+  if (c >= d) return;
+  float s = 0.f;
+  for (int q = prefix[e]; q < prefix[e + 1]; ++q) s += partial[(int64_t)q * d + c];
+  dw_r[(int64_t)c * E + e] = s;
+}
+
+cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, const int32_t *pos,
+                                        const int32_t *offsets, const float *dgate, const float *gate,
+                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st) {
+  const int64_t P = s.P();
+  router_dz_slot_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(pos, dgate, gate, dz_slot, P, s.k);
+  const int64_t max_chunks = (P + RG_ROWS - 1) / RG_ROWS + s.E;
+  dim3 grid((unsigned)max_chunks, (unsigned)((s.d / 2 + RG_THREADS - 1) / RG_THREADS));
+  if (s.dtype == MOE_BF16)
+    router_wgrad_grouped_kernel<bf16><<<grid, RG_THREADS, 0, st>>>(static_cast<const bf16 *>(x_perm), dz_slot,
+                                                                   offsets, partial, s.E, s.d);
+  else
+    router_wgrad_grouped_kernel<float><<<grid, RG_THREADS, 0, st>>>(static_cast<const float *>(x_perm), dz_slot,
+                                                                    offsets, partial, s.E, s.d);
+  dim3 g2((unsigned)((s.d + 255) / 256), (unsigned)s.E);
+  router_wgrad_grouped_reduce_kernel<<<g2, 256, 0, st>>>(partial, offsets, dw_r, s.E, s.d);
   return cudaGetLastError();
 }
 
