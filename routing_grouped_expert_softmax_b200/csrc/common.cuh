@@ -108,6 +108,9 @@ __device__ __forceinline__ void set_error(int *err, int bit) {
 // ---- internal launchers (host side), implemented in routing.cu / rowops.cu / grouped_gemm.cu
 cudaError_t launch_route_topk(const Shape &s, const void *x, const void *w_r, const float *bias,
                               float *logits, int32_t *idx, float *gate, int *err, cudaStream_t st);
+// tensor-core router (bf16, E % 8 == 0) with the top-k fused into its epilogue
+int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float *bias, float *logits,
+                     int32_t *idx, float *gate, int *err, cudaStream_t st);
 cudaError_t launch_topk_gating(const Shape &s, const float *logits, int32_t *idx, float *gate,
                                int *err, cudaStream_t st);
 cudaError_t launch_build_offsets(const Shape &s, const int32_t *idx, int32_t *counts,

@@ -8,15 +8,16 @@
 // стек обучения MoE от Ai2 ...", section "Три числа, три знаменателя" (the gains sit in
 // the feed-forward compute).
 //
-// One persistent kernel, one CTA per SM, 6 warps:
+// One persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) K-blocks in shared
 //               memory (128-byte swizzle), one mbarrier per stage;
 //   warp 1      allocates TMEM; its lane 0 issues tcgen05.mma (128 x BN x 16 per
 //               instruction) into one of two TMEM accumulators and commits each stage
 //               back to the producer;
-//   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
-//               32*(w%4)..+31, i.e. one row per thread), apply the fused elementwise
-//               step and store to global memory, then release the accumulator.
+//   warps 2..9  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
+//               32*(w%4)..+31, i.e. one row per thread; two warps per lane quarter split
+//               the columns), apply the fused elementwise step and store to global
+//               memory, then release the accumulator.
 // The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered accumulator).
 //
 // Tile schedule.  Row-grouped GEMMs (forward and data-gradient) tile every expert's row
@@ -34,15 +35,17 @@
 namespace moe {
 namespace gg {
 
-enum Mode { FWD_GU = 0, FWD_DOWN = 1, DGRAD_DOWN = 2, DGRAD_GU = 3, WGRAD_DOWN = 4, WGRAD_GU = 5 };
+enum Mode { FWD_GU = 0, FWD_DOWN = 1, DGRAD_DOWN = 2, DGRAD_GU = 3, WGRAD_DOWN = 4, WGRAD_GU = 5, ROUTER = 6 };
 
 constexpr int BM = 128;
-constexpr int NUM_THREADS = 192;
+constexpr int EPI_WARPS = 8;
+constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;  // producer warp, MMA warp, epilogue warps
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any tile's time
 
 template <int MODE> struct ModeTraits {
   static constexpr bool A_MN = (MODE == WGRAD_DOWN || MODE == WGRAD_GU);
-  static constexpr bool B_MN = (MODE == FWD_GU || MODE == FWD_DOWN || MODE == WGRAD_DOWN || MODE == WGRAD_GU);
+  static constexpr bool B_MN = (MODE == FWD_GU || MODE == FWD_DOWN || MODE == WGRAD_DOWN || MODE == WGRAD_GU ||
+                                MODE == ROUTER);
   static constexpr bool WGRAD = A_MN;
 };
 
@@ -65,7 +68,7 @@ template <typename T, int BN> struct Cfg {
   static constexpr int A_BYTES = BM * KBLK * ES;
   static constexpr int B_BYTES = BN * KBLK * ES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
   static constexpr int TMEM_COLS = 2 * BN;              // two accumulators
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 2048 /*bars etc*/;
 };
@@ -80,7 +83,9 @@ struct Params {
   int f, d;
   void *out0;
   void *out1;
+  void *out2;
   const void *aux;
+  int k;       // router: experts per token
   int *err;
   int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
 };
@@ -111,7 +116,14 @@ struct Ctrl {
 
 template <int MODE, int BN, int KBLK>
 __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl) {
-  if constexpr (ModeTraits<MODE>::WGRAD) {
+  if constexpr (MODE == ROUTER) {
+    tl.e = 0;
+    tl.m_blk = t;
+    tl.n_blk = 0;
+    tl.row0 = t * BM;
+    tl.rows = min(BM, p.P - t * BM);
+    tl.num_kb = p.K / KBLK;
+  } else if constexpr (ModeTraits<MODE>::WGRAD) {
     const int mt = p.M / BM, nt = p.N / BN;
     tl.e = t / (mt * nt);
     int r = t - tl.e * mt * nt;
@@ -143,7 +155,8 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
 
 template <int MODE, int BN>
 __device__ __forceinline__ int total_tiles(const Params &p, const Ctrl &c) {
-  if constexpr (ModeTraits<MODE>::WGRAD) return p.E * (p.M / BM) * (p.N / BN);
+  if constexpr (MODE == ROUTER) return (p.P + BM - 1) / BM;
+  else if constexpr (ModeTraits<MODE>::WGRAD) return p.E * (p.M / BM) * (p.N / BN);
   else return c.prefix[p.E] * (p.N / BN);
 }
 
@@ -164,6 +177,17 @@ __device__ __forceinline__ void load32(const T *src, float (&v)[32]) {
 }
 
 __device__ __forceinline__ float sigmoidf_(float h) { return 1.0f / (1.0f + __expf(-h)); }
+
+// Router order: numbers before NaN, larger first, then the lower expert index; an empty
+// slot (index INT_MAX) loses to everything.
+__device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
+  if (ai == INT_MAX) return false;
+  if (bi == INT_MAX) return true;
+  const bool an = av != av, bn = bv != bv;
+  if (an != bn) return bn;
+  if (an) return ai < bi;
+  return av > bv || (av == bv && ai < bi);
+}
 
 template <typename T, int BN, int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -191,7 +215,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
-      ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), 128);
+      ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), 32 * EPI_WARPS);
     }
     ptx::mbar_init(ptx::smem_u32(&c.tail), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
@@ -205,7 +229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == 2 && !MT::WGRAD) {
+  if (warp == 2 && !MT::WGRAD && MODE != ROUTER) {
     // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
     int cnt[8], s = 0;
 #pragma unroll
@@ -286,6 +310,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ptx::tma_load_2d(b_dst + (half / C::BOX_MN + i) * C::BOX_BYTES, &tmB1, bar,
                                tl.n_blk * half + i * C::BOX_MN, tl.e * p.K + kb * C::KBLK);
             }
+          } else if constexpr (MODE == ROUTER) {
+            // W_r [d][E], MN-major; columns past E read as zeros
+#pragma unroll
+            for (int i = 0; i < BN / C::BOX_MN; ++i)
+              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, i * C::BOX_MN, kb * C::KBLK);
           } else if constexpr (MODE == FWD_DOWN) {
 #pragma unroll
             for (int i = 0; i < BN / C::BOX_MN; ++i)
@@ -401,7 +430,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue
-    const int q = warp & 3;               // TMEM lane quarter this warp may access
+    // EPI_WARPS warps: warp w reads TMEM lane quarter w % 4 (one tile row per thread);
+    // the two warps of a quarter split the accumulator's columns in halves.
+    const int q = warp & 3;
+    const int half = (warp - 2) >> 2;     // 0 or 1
     const int r = q * 32 + lane;          // tile row owned by this thread
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
@@ -414,14 +446,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 
-      if constexpr (MODE == FWD_GU) {
+      if constexpr (MODE == ROUTER) {
+        // One token per thread: z = x W_r (+ b) for all E experts, then top-k by an
+        // insertion network over the logits in expert order (a later equal logit never
+        // displaces an earlier one: ties go to the lower index), then the softmax of the
+        // k selected logits.  The first warp of each lane quarter does the work.
+        if (half == 0) {
+          const bool valid = r < tl.rows;
+          const int64_t row = (int64_t)tl.row0 + r;
+          const float *bias = static_cast<const float *>(p.aux);
+          float *logits = static_cast<float *>(p.out2);
+          float tv[MAX_K];
+          int ti[MAX_K];
+#pragma unroll
+          for (int j = 0; j < MAX_K; ++j) { tv[j] = 0.f; ti[j] = INT_MAX; }
+          bool nan_seen = false;
+#pragma unroll 1
+          for (int c0 = 0; c0 < p.E; c0 += 32) {
+            float v[32];
+            ptx::tmem_ld32(taddr + c0, v);
+            if (valid) {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                const int e = c0 + i;
+                if (e < p.E) {
+                  float z = v[i] + (bias ? __ldg(bias + e) : 0.f);
+                  v[i] = z;
+                  nan_seen |= (z != z);
+                  float cv = z;
+                  int ci = e;
+#pragma unroll
+                  for (int j = 0; j < MAX_K; ++j) {
+                    bool take = j < p.k && topk_better(cv, ci, tv[j], ti[j]);
+                    float sv = tv[j];
+                    int si = ti[j];
+                    if (take) { tv[j] = cv; ti[j] = ci; cv = sv; ci = si; }
+                  }
+                }
+              }
+              if (logits) {
+                if (c0 + 32 <= p.E) {
+                  store32(logits + row * p.E + c0, v);
+                } else {
+#pragma unroll
+                  for (int i = 0; i < 32; ++i)
+                    if (c0 + i < p.E) logits[row * p.E + c0 + i] = v[i];
+                }
+              }
+            }
+          }
+          if (valid) {
+            if (nan_seen) set_error(p.err, MOE_ERR_DEVICE_NAN);
+            int32_t *idx = static_cast<int32_t *>(p.out0);
+            float *gate = static_cast<float *>(p.out1);
+            float ex[MAX_K], sum = 0.f;
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j)
+              if (j < p.k) { ex[j] = expf(tv[j] - tv[0]); sum += ex[j]; }
+            const float inv = 1.0f / sum;
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j)
+              if (j < p.k) { idx[row * p.k + j] = ti[j]; gate[row * p.k + j] = ex[j] * inv; }
+          }
+        }
+      } else if constexpr (MODE == FWD_GU) {
         // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
         const bool valid = r < tl.rows;
         const int64_t row = (int64_t)tl.row0 + r;
         T *hu = static_cast<T *>(p.out0);
         T *aa = static_cast<T *>(p.out1);
 #pragma unroll 1
-        for (int cc = 0; cc < BN / 2; cc += 32) {
+        for (int cc = half * (BN / 4); cc < (half + 1) * (BN / 4); cc += 32) {
           float h[32], u[32];
           ptx::tmem_ld32(taddr + cc, h);
           ptx::tmem_ld32(taddr + BN / 2 + cc, u);
@@ -440,41 +535,60 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int64_t row = (int64_t)tl.row0 + r;
         T *out = static_cast<T *>(p.out0);
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
+        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
           ptx::tmem_ld32(taddr + cc, v);
           if (valid) store32(out + row * p.N + tl.n_blk * BN + cc, v);
         }
       } else if constexpr (MODE == DGRAD_DOWN) {
-        // da -> (dh, du) through the SwiGLU derivative, using the saved h and u
+        // da -> (dh, du) through the SwiGLU derivative, using the saved h and u.  The
+        // loads of the next chunk's h, u are issued before this chunk's math.
         const bool valid = r < tl.rows;
         const int64_t row = (int64_t)tl.row0 + r;
         const T *hu = static_cast<const T *>(p.aux);
         T *dhu = static_cast<T *>(p.out0);
-#pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
+        constexpr int NV = 32 / Vec<T>::N;   // 16-byte vectors per 32 values
+        const int c0 = half * (BN / 2), c1 = (half + 1) * (BN / 2);
+        uint4 hv[2][NV], uv[2][NV];
+        auto issue = [&](int buf, int cc) {
+          const uint4 *hs = reinterpret_cast<const uint4 *>(hu + row * 2 * p.f + tl.n_blk * BN + cc);
+          const uint4 *us = reinterpret_cast<const uint4 *>(hu + row * 2 * p.f + p.f + tl.n_blk * BN + cc);
+#pragma unroll
+          for (int i = 0; i < NV; ++i) { hv[buf][i] = __ldg(hs + i); uv[buf][i] = __ldg(us + i); }
+        };
+        if (valid) issue(0, c0);
+#pragma unroll
+        for (int j = 0; j < (BN / 2) / 32; ++j) {
+          const int cc = c0 + j * 32;
           float da[32];
           ptx::tmem_ld32(taddr + cc, da);
           if (valid) {
+            if (cc + 32 < c1) issue((j + 1) & 1, cc + 32);
             const int col = tl.n_blk * BN + cc;
-            float h[32], u[32];
-            load32(hu + row * 2 * p.f + col, h);
-            load32(hu + row * 2 * p.f + p.f + col, u);
-            float dh[32], du[32];
+            uint4 *dh_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + col);
+            uint4 *du_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + p.f + col);
+            constexpr int VN = Vec<T>::N;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              float s = sigmoidf_(h[i]);
-              dh[i] = da[i] * u[i] * s * (1.0f + h[i] * (1.0f - s));
-              du[i] = da[i] * h[i] * s;
+            for (int i = 0; i < NV; ++i) {   // one 16-byte vector of h, u at a time
+              float h[VN], u[VN], dh[VN], du[VN];
+              Vec<T>::load(hv[j & 1][i], h);
+              Vec<T>::load(uv[j & 1][i], u);
+#pragma unroll
+              for (int v = 0; v < VN; ++v) {
+                const float g = da[i * VN + v];
+                const float s = sigmoidf_(h[v]);
+                dh[v] = g * u[v] * s * (1.0f + h[v] * (1.0f - s));
+                du[v] = g * h[v] * s;
+              }
+              dh_dst[i] = Vec<T>::store(dh);
+              du_dst[i] = Vec<T>::store(du);
             }
-            store32(dhu + row * 2 * p.f + col, dh);
-            store32(dhu + row * 2 * p.f + p.f + col, du);
           }
         }
       } else {  // weight gradients: row r of the [M x N] block of expert e
         const int64_t mrow = (int64_t)tl.m_blk * BM + r;
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
+        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
           if (tl.num_kb > 0) ptx::tmem_ld32(taddr + cc, v);
           else {
@@ -692,7 +806,31 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   return MOE_OK;
 }
 
+// Router on the tensor cores: logits = x [T,d] x W_r [d,E] (bf16 in, fp32 out) with the
+// top-k and gates fused into the epilogue.  Needs E % 8 == 0 (16-byte TMA row pitch).
+static int router_impl(const Shape &s, const void *x, const void *w_r, const float *bias, float *logits,
+                       int32_t *idx, float *gate, int *err, cudaStream_t st) {
+  constexpr int ES = 2, KBLK = 64, BOX_MN = 64;
+  CUtensorMap tA, tB;
+  if (!make_tmap(&tA, x, ES, s.d, s.T, KBLK, BM)) return MOE_ERR_CUDA;
+  if (!make_tmap(&tB, w_r, ES, s.E, s.d, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+  Params p{};
+  p.E = s.E; p.P = (int)s.T; p.K = s.d; p.d = s.d; p.f = s.f; p.k = s.k;
+  p.out0 = idx; p.out1 = gate; p.out2 = logits; p.aux = bias; p.err = err; p.where = err + 1;
+  const int64_t tiles = (s.T + BM - 1) / BM;
+  const int bn = s.E <= 64 ? 64 : s.E <= 128 ? 128 : 256;
+  p.N = bn;
+  if (bn == 64) return launch<bf16, 64, ROUTER>(tA, tB, tB, p, tiles, st);
+  if (bn == 128) return launch<bf16, 128, ROUTER>(tA, tB, tB, p, tiles, st);
+  return launch<bf16, 256, ROUTER>(tA, tB, tB, p, tiles, st);
+}
+
 }  // namespace gg
+
+int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float *bias, float *logits,
+                     int32_t *idx, float *gate, int *err, cudaStream_t st) {
+  return gg::router_impl(s, x, w_r, bias, logits, idx, gate, err, st);
+}
 
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,

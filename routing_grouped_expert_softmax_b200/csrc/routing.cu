@@ -224,6 +224,11 @@ static cudaError_t route_dispatch(const Shape &s, const void *x, const void *w_r
 cudaError_t launch_route_topk(const Shape &s, const void *x, const void *w_r, const float *bias,
                               float *logits, int32_t *idx, float *gate, int *err, cudaStream_t st) {
   if (s.T == 0) return cudaSuccess;
+  if (s.dtype == MOE_BF16 && s.E % 8 == 0) {
+    // the tensor-core router; its host-side failures come back as a CUDA error
+    return launch_router_tc(s, x, w_r, bias, logits, idx, gate, err, st) == MOE_OK ? cudaSuccess
+                                                                                   : cudaErrorLaunchFailure;
+  }
   if (s.dtype == MOE_BF16) return route_dispatch<bf16>(s, x, w_r, bias, logits, idx, gate, err, st);
   return route_dispatch<float>(s, x, w_r, bias, logits, idx, gate, err, st);
 }

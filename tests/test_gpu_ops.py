@@ -66,6 +66,8 @@ def test_topk_gating_bit_exact(T, E, k, kind):
     (1000, 256, 64, 4, "bf16", True),
     (333, 384, 128, 4, "bf16", False),
     (129, 128, 256, 8, "bf16", True),
+    (300, 256, 36, 4, "bf16", False),     # E not a multiple of 8: the CUDA-core router
+    (8192, 2048, 8, 4, "bf16", False),    # E below one 64-column MMA tile
 ])
 def test_route_topk(T, d, E, k, dtype, bias):
     import torch
