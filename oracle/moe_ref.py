@@ -341,6 +341,15 @@ def layer_bwd_routed(fwd, dY, w_gate, w_up, w_down):
 # scale per block of 32 consecutive elements along the reduction axis.
 # ---------------------------------------------------------------------------
 
+def bf16_rne(v):
+    """Round to bf16 (nearest, ties to even) through fp32, as a GEMM output stored in bf16
+    after fp32 accumulation: the bf16 tensors the MXFP8 GEMMs quantise."""
+    f = np.asarray(v, F64).astype(np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return (u.astype(np.uint32) << 16).view(np.float32).astype(F64)
+
+
 MX_BLOCK = 32
 E4M3_EMAX = 8          # exponent of the largest normal E4M3 value, 448 = 1.75 * 2^8
 E4M3_MAX = 448.0
@@ -456,7 +465,8 @@ def grouped_swiglu_mx(x_perm, offsets, w_gate, w_up, w_down):
 
     GEMM 1: x_perm (K = d, along rows' columns) with W_gate/W_up (K = d, along
     their rows).  GEMM 2: a (K = f) with W_down (K = f).  Products and sums in
-    float64 on the dequantised values.
+    float64 on the dequantised values.  The MXFP8 GEMMs output bf16, so GEMM 2
+    quantises a as stored: bf16(a).  Returns h, u, a unrounded.
     """
     xq = mx_quantize(x_perm, axis=1)[2]
     wgq = mx_quantize(w_gate, axis=1)[2]
@@ -476,7 +486,7 @@ def grouped_swiglu_mx(x_perm, offsets, w_gate, w_up, w_down):
         h[lo:hi] = xq[lo:hi] @ wgq[e]
         u[lo:hi] = xq[lo:hi] @ wuq[e]
         a[lo:hi] = silu(h[lo:hi]) * u[lo:hi]
-    aq = mx_quantize(a, axis=1)[2]
+    aq = mx_quantize(bf16_rne(a), axis=1)[2]
     for e in range(w_gate.shape[0]):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi > lo:
@@ -489,7 +499,9 @@ def grouped_swiglu_bwd_mx(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_dow
 
     dgrad GEMMs reduce over the feature axis (dy: K = d with W_down^T; [dh|du]:
     K = 2f with [W_gate|W_up]^T); weight-gradient GEMMs reduce over the tokens
-    of one expert (blocks of 32 rows inside each expert, zero-padded).
+    of one expert (blocks of 32 rows inside each expert, zero-padded).  [dh|du]
+    is the bf16 output of the first GEMM's epilogue, so both GEMMs that read it
+    quantise bf16([dh|du]).  Returns dh, du unrounded.
     """
     dy_perm = np.asarray(dy_perm, F64)
     x_perm = np.asarray(x_perm, F64)
@@ -505,7 +517,7 @@ def grouped_swiglu_bwd_mx(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_dow
             continue
         da = dyq_k[lo:hi] @ wdq_t[e].T
         dh[lo:hi], du[lo:hi] = swiglu_bwd(da, h[lo:hi], u[lo:hi])
-    dhu = np.concatenate([dh, du], axis=1)
+    dhu = bf16_rne(np.concatenate([dh, du], axis=1))
     dhuq_k = mx_quantize(dhu, axis=1)[2]
     wgu = np.concatenate([np.asarray(w_gate, F64), np.asarray(w_up, F64)], axis=2)  # [E, d, 2f]
     wguq_t = mx_quantize(wgu, axis=2)[2]
