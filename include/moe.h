@@ -75,6 +75,9 @@ enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1 };
  * quantises both operands of each grouped GEMM to E4M3 with one E8M0 scale per
  * 32 elements along the reduction axis. */
 enum moe_prec { MOE_PREC_NATIVE = 0, MOE_PREC_MXFP8 = 1 };
+/* MOE_PREC_MXFP8 needs dtype MOE_BF16 (bf16 storage, outputs and gradients stay bf16).
+ * The quantised operands live in the workspace, which is then much larger (about
+ * 2*(P + 127*E)*(3d + 3f) + 4*E*d*f bytes). */
 
 typedef struct moe_config {
   int64_t T;     /* tokens */
@@ -175,6 +178,25 @@ MOE_API int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, c
                            const void *w_gate, const void *w_up, const void *w_down,
                            void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
                            void *dw_down, void *ws, moe_stream_t stream);
+
+/* MXFP8 quantisation (OCP Microscaling v1.0, as the pages' "MXFP8" is read here):
+ * E4M3 codes with one E8M0 scale byte per 32 elements, X = 2^(floor(log2 amax) - 8)
+ * clamped to [2^-127, 2^127] (amax = 0 gives 2^-127), v / X rounded to nearest even and
+ * saturated to +-448; scale byte = 127 + log2 X.  src is bf16 [rows][cols].
+ *   rows variant: blocks of 32 consecutive columns; codes [R'][cols], scales [R'][cols/32].
+ *   cols variant: blocks of 32 consecutive rows;    codes [R'][cols], scales [R'/32][cols].
+ * offsets == NULL: R' = rows (for the cols variant, a partial last block reads zeros).
+ * offsets != NULL ([E+1], as from moe_build_offsets): the rows are E expert groups and are
+ *   written into buffers padded to 128 rows per expert; padded row 128*pre[e] + i holds
+ *   src row offsets[e] + i for i < count_e and zeros after, pre[e] = sum_{e'<e}
+ *   ceil(count_e'/128); the buffers must hold rows_bound >= rows + 127*E rows.
+ * cols must be a multiple of 32 (of 128 for the rows variant with offsets). */
+MOE_API int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int32_t *offsets,
+                                 int32_t E, int64_t rows_bound, uint8_t *codes, uint8_t *scales,
+                                 moe_stream_t stream);
+MOE_API int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, const int32_t *offsets,
+                                 int32_t E, int64_t rows_bound, uint8_t *codes, uint8_t *scales,
+                                 moe_stream_t stream);
 
 /* ---------------------------------------------------------------- combine */
 

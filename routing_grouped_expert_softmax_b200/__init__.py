@@ -35,7 +35,8 @@ EXPORTED = [
     "moe_workspace_size", "moe_get_error", "moe_route_topk", "moe_topk_gating",
     "moe_build_offsets", "moe_build_offsets_noalloc", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
-    "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd",
+    "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd", "moe_mx_quantize_rows",
+    "moe_mx_quantize_cols",
 ]
 
 
@@ -100,6 +101,10 @@ def lib() -> ctypes.CDLL:
             "moe_combine_bwd": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
             "moe_unpermute_sum": (ctypes.c_int, [_CFG, _P, _P, _P, _P]),
             "moe_route_bwd": (ctypes.c_int, [_CFG] + [_P] * 9),
+            "moe_mx_quantize_rows": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, ctypes.c_int32,
+                                                    ctypes.c_int64, _P, _P, _P]),
+            "moe_mx_quantize_cols": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, ctypes.c_int32,
+                                                    ctypes.c_int64, _P, _P, _P]),
             "moe_layer_fwd": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
                                              ctypes.POINTER(LayerSaved), _P, _P]),
             "moe_layer_fwd_routed": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
@@ -214,6 +219,16 @@ def moe_unpermute_sum(cfg, dx_perm, slot_of_pair, dx, stream=None):
 def moe_route_bwd(cfg, dgate, topk_gate, topk_idx, x, w_router, dx, dw_router, ws, stream=None):
     _call("moe_route_bwd", ctypes.byref(cfg), ptr(dgate), ptr(topk_gate), ptr(topk_idx), ptr(x),
           ptr(w_router), ptr(dx), ptr(dw_router), ptr(ws), stream_handle(stream))
+
+
+def moe_mx_quantize_rows(src, rows, cols, offsets, E, rows_bound, codes, scales, stream=None):
+    _call("moe_mx_quantize_rows", ptr(src), rows, cols, ptr(offsets), E, rows_bound, ptr(codes),
+          ptr(scales), stream_handle(stream))
+
+
+def moe_mx_quantize_cols(src, rows, cols, offsets, E, rows_bound, codes, scales, stream=None):
+    _call("moe_mx_quantize_cols", ptr(src), rows, cols, ptr(offsets), E, rows_bound, ptr(codes),
+          ptr(scales), stream_handle(stream))
 
 
 def _struct(cls, fields, d):

@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmoe.so")
-SOURCES = ["routing.cu", "rowops.cu", "grouped_gemm.cu", "moe_abi.cu", "noalloc.cu"]
+SOURCES = ["routing.cu", "rowops.cu", "grouped_gemm.cu", "quant.cu", "moe_abi.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "-Xptxas", "-warn-spills", "--expt-relaxed-constexpr"]

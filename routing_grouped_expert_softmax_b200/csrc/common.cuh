@@ -23,17 +23,22 @@ struct Shape {
   int64_t T;
   int d, E, k, f;
   int dtype;
+  int prec = MOE_PREC_NATIVE;
+  // rows of an expert buffer padded to 128 rows per expert (MXFP8 operands), upper bound
+  int64_t Ppad() const { return P() + 127 * (int64_t)E; }
   int64_t P() const { return T * (int64_t)k; }
   int es() const { return dtype == MOE_BF16 ? 2 : 4; }
 };
 
 inline Shape shape_of(const moe_config *c) {
   Shape s;
-  s.T = c->T; s.d = c->d; s.E = c->E; s.k = c->k; s.f = c->f; s.dtype = c->dtype;
+  s.T = c->T; s.d = c->d; s.E = c->E; s.k = c->k; s.f = c->f; s.dtype = c->dtype; s.prec = c->prec;
   return s;
 }
 
 inline int *err_word(void *ws) { return reinterpret_cast<int *>(static_cast<char *>(ws) + WS_ERR); }
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Workspace carve-up shared by the host launchers.
 struct WsLayout {
@@ -43,11 +48,17 @@ struct WsLayout {
   size_t wt;             // fp32 storage only: Wg^T, Wu^T [E][f][d] and Wd^T [E][d][f]
   size_t dz_slot;        // fp32 [P]: router logit gradient of the pair in each slot
   size_t rg_partial;     // fp32 [P/64 + E][d]: per-chunk router weight-gradient sums
+  // MXFP8 operands (codes, then scales), present when prec == MOE_PREC_MXFP8:
+  //   *_r: blocks along the row (K-major use), *_t: blocks down the rows (token axis)
+  size_t xq_r, aq_r, dyq_r, dhuq_r, xq_t, aq_t, dyq_t, dhuq_t;  // activations, Ppad rows
+  size_t wgu_c, wd_c, wd_r, wgu_r;                              // weights
   size_t total;
 };
+// bytes of an MXFP8 operand [rows][cols] with scales along the row / down the rows
+inline size_t mx_bytes_r(int64_t rows, int64_t cols) { return align_up((size_t)(rows * cols + rows * (cols / 32)), 256); }
+inline size_t mx_bytes_t(int64_t rows, int64_t cols) { return align_up((size_t)(rows * cols + (rows / 32) * cols), 256); }
 constexpr int RB_SPLIT = 16;          // token splits of the router weight-gradient reduction
 
-inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 inline WsLayout ws_layout(const Shape &s) {
   WsLayout L;
@@ -60,6 +71,23 @@ inline WsLayout ws_layout(const Shape &s) {
   if (s.dtype == MOE_F32) off = align_up(off + (size_t)3 * s.E * s.d * s.f * 4, 256);
   L.dz_slot = off;      off = align_up(off + (size_t)s.P() * 4, 256);
   L.rg_partial = off;   off = align_up(off + (size_t)((s.P() + 63) / 64 + s.E) * s.d * 4, 256);
+  L.xq_r = L.aq_r = L.dyq_r = L.dhuq_r = L.xq_t = L.aq_t = L.dyq_t = L.dhuq_t = 0;
+  L.wgu_c = L.wd_c = L.wd_r = L.wgu_r = 0;
+  if (s.prec == MOE_PREC_MXFP8) {
+    const int64_t R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
+    L.xq_r = off;   off += mx_bytes_r(R, s.d);
+    L.aq_r = off;   off += mx_bytes_r(R, s.f);
+    L.dyq_r = off;  off += mx_bytes_r(R, s.d);
+    L.dhuq_r = off; off += mx_bytes_r(R, 2 * s.f);
+    L.xq_t = off;   off += mx_bytes_t(R, s.d);
+    L.aq_t = off;   off += mx_bytes_t(R, s.f);
+    L.dyq_t = off;  off += mx_bytes_t(R, s.d);
+    L.dhuq_t = off; off += mx_bytes_t(R, 2 * s.f);
+    L.wgu_c = off;  off += mx_bytes_t(ed, 2 * s.f);
+    L.wd_c = off;   off += mx_bytes_t(ef, s.d);
+    L.wd_r = off;   off += mx_bytes_r(ef, s.d);
+    L.wgu_r = off;  off += mx_bytes_r(ed, 2 * s.f);
+  }
   L.total = off;
   return L;
 }
@@ -140,9 +168,19 @@ int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offset
                        void *a, void *y_perm, void *ws, cudaStream_t st);
 // dst[b][c][r] = src[b][r][c] (fp32)
 cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st);
+// MXFP8 quantisers (quant.cu).  offsets != nullptr: source rows are expert groups written
+// into buffers padded to 128 rows per expert (rows_bound: rows the buffer holds).
+cudaError_t launch_mx_quant_rows(const void *src, int64_t R, int K, const int32_t *offsets, int E, int64_t rows_bound,
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st);
+cudaError_t launch_mx_quant_cols(const void *src, int64_t R, int C, const int32_t *offsets, int E, int64_t rows_bound,
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st);
+cudaError_t launch_mx_quant_cols_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
+                                    uint8_t *scales, cudaStream_t st);
+cudaError_t launch_mx_quant_rows_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
+                                    uint8_t *scales, cudaStream_t st);
 int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                        const void *a, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *dhu, void *dx_perm,
-                       void *dw_gate, void *dw_up, void *dw_down, int *err, cudaStream_t st);
+                       void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st);
 
 }  // namespace moe

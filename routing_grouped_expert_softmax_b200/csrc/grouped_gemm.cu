@@ -49,17 +49,30 @@ template <int MODE> struct ModeTraits {
   static constexpr bool WGRAD = A_MN;
 };
 
+// MXFP8 operand tag: E4M3 codes with E8M0 scales per 32 K-elements (outputs stay bf16).
+struct e4m3 {
+  uint8_t v;
+};
+
 template <typename T> struct ElemTraits;
 template <> struct ElemTraits<bf16> {
   static constexpr int ES = 2;
   static constexpr uint32_t FMT = 1;  // BF16 in the instruction descriptor
+  using Out = bf16;
 };
 template <> struct ElemTraits<float> {
   static constexpr int ES = 4;
   static constexpr uint32_t FMT = 2;  // TF32
+  using Out = float;
+};
+template <> struct ElemTraits<e4m3> {
+  static constexpr int ES = 1;
+  static constexpr uint32_t FMT = 0;  // E4M3 in the block-scaled instruction descriptor
+  using Out = bf16;
 };
 
 template <typename T, int BN> struct Cfg {
+  static constexpr bool MX = (ElemTraits<T>::ES == 1);
   static constexpr int ES = ElemTraits<T>::ES;
   static constexpr int KBLK = 128 / ES;                 // K elements per stage (one 128-B swizzle row)
   static constexpr int UMMA_K = 32 / ES;                // K per tcgen05.mma
@@ -69,8 +82,10 @@ template <typename T, int BN> struct Cfg {
   static constexpr int B_BYTES = BN * KBLK * ES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
-  static constexpr int TMEM_COLS = 2 * BN;              // two accumulators
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align slack*/ + 2048 /*bars etc*/;
+  // two accumulators; MXFP8 adds 8 columns of scale factors (A: 4, B: 4) after them
+  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
+  static constexpr int SF_BYTES = MX ? 1024 : 0;        // per stage: 512-byte scale blocks of A and B
+  static constexpr int SMEM_BYTES = STAGES * (STAGE_BYTES + SF_BYTES) + 1024 /*align slack*/ + 2048 /*bars etc*/;
 };
 
 struct Params {
@@ -86,6 +101,11 @@ struct Params {
   void *out2;
   const void *aux;
   int k;       // router: experts per token
+  // MXFP8 scale factors: K-major operands [rows][K/32] (ld = K/32), MN-major operands
+  // [K/32][MN] (ld = MN)
+  const uint8_t *sfa;
+  const uint8_t *sfb;
+  int sfa_ld, sfb_ld;
   int *err;
   int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
 };
@@ -96,6 +116,7 @@ __device__ __forceinline__ void note_fail(const Params &p, int role, int t, int 
 
 struct Tile {
   int e, m_blk, n_blk;
+  int orow0;      // first output row (row-grouped modes)
   int row0;       // first A row (row-grouped) or first K row (weight-gradient)
   int rows;       // valid rows (row-grouped) or valid K rows (weight-gradient)
   int num_kb;
@@ -114,13 +135,13 @@ struct Ctrl {
   int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
 };
 
-template <int MODE, int BN, int KBLK>
+template <int MODE, int BN, int KBLK, bool MX>
 __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl) {
   if constexpr (MODE == ROUTER) {
     tl.e = 0;
     tl.m_blk = t;
     tl.n_blk = 0;
-    tl.row0 = t * BM;
+    tl.row0 = tl.orow0 = t * BM;
     tl.rows = min(BM, p.P - t * BM);
     tl.num_kb = p.K / KBLK;
   } else if constexpr (ModeTraits<MODE>::WGRAD) {
@@ -130,9 +151,16 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.m_blk = r / nt;
     tl.n_blk = r - tl.m_blk * nt;
     int lo = p.offsets[tl.e], hi = p.offsets[tl.e + 1];
-    tl.row0 = lo;
     tl.rows = hi - lo;
-    tl.num_kb = (tl.rows + KBLK - 1) / KBLK;
+    if constexpr (MX) {
+      // quantised operands live in expert buffers padded to 128 rows (zeros past the end)
+      tl.row0 = c.prefix[tl.e] * BM;
+      tl.num_kb = c.prefix[tl.e + 1] - c.prefix[tl.e];
+    } else {
+      tl.row0 = lo;
+      tl.num_kb = (tl.rows + KBLK - 1) / KBLK;
+    }
+    tl.orow0 = 0;
   } else {
     const int nt = p.N / BN;
     int g = t / nt;
@@ -146,7 +174,8 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.e = lo;
     tl.m_blk = g - c.prefix[lo];
     int off = p.offsets[lo], cnt = p.offsets[lo + 1] - off;
-    tl.row0 = off + tl.m_blk * BM;
+    tl.orow0 = off + tl.m_blk * BM;
+    tl.row0 = MX ? g * BM : tl.orow0;   // quantised A: expert buffers padded to 128 rows
     tl.rows = min(BM, cnt - tl.m_blk * BM);
     tl.num_kb = p.K / KBLK;
   }
@@ -178,6 +207,32 @@ __device__ __forceinline__ void load32(const T *src, float (&v)[32]) {
 
 __device__ __forceinline__ float sigmoidf_(float h) { return 1.0f / (1.0f + __expf(-h)); }
 
+// MXFP8 scale blocks in shared memory: 128 rows (or columns) x 4 K-blocks in 512 bytes,
+// row m's four scales forming the 32-bit word at byte 16*(m%32) + 4*(m/32).  Lane l of the
+// producer warp builds the 16 bytes at 16*l (rows l, l+32, l+64, l+96).
+// K-major operand: scales [rows][ld], the stage's four bytes of row m at (rowbase+m)*ld + 4*kb.
+__device__ __forceinline__ void sf_gather_kmajor(const uint8_t *sf, int64_t rowbase, int ld, int kb, uint8_t *dst,
+                                                 int lane) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    w[i] = __ldg(reinterpret_cast<const uint32_t *>(sf + (rowbase + lane + 32 * i) * ld + 4 * kb));
+  *reinterpret_cast<uint4 *>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+// MN-major operand: scales [K/32][ld], K-block kblk+kc of column colbase+m at (kblk+kc)*ld + colbase + m.
+__device__ __forceinline__ void sf_gather_mnmajor(const uint8_t *sf, int64_t kblk, int ld, int64_t colbase,
+                                                  uint8_t *dst, int lane) {
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int kc = 0; kc < 4; ++kc) v |= (uint32_t)__ldg(sf + (kblk + kc) * ld + colbase + lane + 32 * i) << (8 * kc);
+    w[i] = v;
+  }
+  *reinterpret_cast<uint4 *>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
 // Router order: numbers before NaN, larger first, then the lower expert index; an empty
 // slot (index INT_MAX) loses to everything.
 __device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
@@ -202,7 +257,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ring = smem;                                   // STAGES x (A | B)
-  Ctrl &c = *reinterpret_cast<Ctrl *>(smem + C::STAGES * C::STAGE_BYTES);
+  uint8_t *sf_ring = smem + C::STAGES * C::STAGE_BYTES;   // MXFP8: STAGES x (SFA | SFB)
+  Ctrl &c = *reinterpret_cast<Ctrl *>(smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES));
   volatile int *abort_flag = &c.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -210,7 +266,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // ------------------------------------------------------------------ prologue
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      ptx::mbar_init(ptx::smem_u32(&c.full[s]), 1);
+      // MXFP8: a second arrival once the producer warp has written the stage's scales
+      ptx::mbar_init(ptx::smem_u32(&c.full[s]), C::MX ? 2 : 1);
       ptx::mbar_init(ptx::smem_u32(&c.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -229,7 +286,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == 2 && !MT::WGRAD && MODE != ROUTER) {
+  if (warp == 2 && (!MT::WGRAD || C::MX) && MODE != ROUTER) {
     // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
     int cnt[8], s = 0;
 #pragma unroll
@@ -270,7 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     bool ok = true;
     for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+      get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
       for (int kb = 0; kb < tl.num_kb && ok; ++kb) {
         if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -278,7 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t a_dst = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
         const uint32_t b_dst = a_dst + C::A_BYTES;
         int valid = C::KBLK;
-        if constexpr (MT::WGRAD) valid = min(C::KBLK, tl.rows - kb * C::KBLK);
+        if constexpr (MT::WGRAD && !C::MX) valid = min(C::KBLK, tl.rows - kb * C::KBLK);
         const bool tail = valid < C::KBLK;
         const uint32_t bar = tail ? ptx::smem_u32(&c.tail) : ptx::smem_u32(&c.full[stage]);
         if (lane == 0) {
@@ -293,7 +350,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tma_load_2d(a_dst, &tmA, bar, kb * C::KBLK, tl.row0);
           }
           // ---- B
-          if constexpr (FWD_B_KMAJOR && MODE == FWD_GU) {
+          if constexpr (C::MX && MODE == FWD_GU) {
+            // quantised [Wg | Wu] with gate and up interleaved in 64-column chunks
+            ptx::tma_load_2d(b_dst, &tmB0, bar, tl.n_blk * BN, tl.e * p.K + kb * C::KBLK);
+          } else if constexpr (C::MX && MODE == DGRAD_GU) {
+            // quantised [Wg | Wu] rows (K = 2f), one tensor
+            ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+          } else if constexpr (FWD_B_KMAJOR && MODE == FWD_GU) {
             // Wg^T, Wu^T [E*f][d]: gate rows then up rows of the 256-row B tile
             const int half = BN / 2;
             ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.f + tl.n_blk * half);
@@ -334,6 +397,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * BN + i * C::BOX_MN,
                                tl.row0 + kb * C::KBLK);
           }
+        }
+        if constexpr (C::MX) {
+          // this stage's scales: A then B, 512 bytes each
+          uint8_t *sfa_s = sf_ring + stage * C::SF_BYTES;
+          uint8_t *sfb_s = sfa_s + 512;
+          if constexpr (MT::A_MN)
+            sf_gather_mnmajor(p.sfa, (tl.row0 + kb * C::KBLK) / 32, p.sfa_ld, (int64_t)tl.m_blk * BM, sfa_s, lane);
+          else
+            sf_gather_kmajor(p.sfa, tl.row0, p.sfa_ld, kb, sfa_s, lane);
+          if constexpr (MODE == FWD_GU)
+            sf_gather_mnmajor(p.sfb, ((int64_t)tl.e * p.K + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN,
+                              sfb_s, lane);
+          else if constexpr (MODE == FWD_DOWN)
+            sf_gather_mnmajor(p.sfb, ((int64_t)tl.e * p.K + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN,
+                              sfb_s, lane);
+          else if constexpr (MODE == DGRAD_DOWN)
+            sf_gather_kmajor(p.sfb, (int64_t)tl.e * p.f + tl.n_blk * BN, p.sfb_ld, kb, sfb_s, lane);
+          else if constexpr (MODE == DGRAD_GU)
+            sf_gather_kmajor(p.sfb, (int64_t)tl.e * p.d + tl.n_blk * BN, p.sfb_ld, kb, sfb_s, lane);
+          else
+            sf_gather_mnmajor(p.sfb, (tl.row0 + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN, sfb_s, lane);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
         }
         if (tail) {
           // Weight gradients only: K rows past the expert's end belong to another expert
@@ -379,13 +466,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t idesc = (1u << 4) | (ElemTraits<T>::FMT << 7) | (ElemTraits<T>::FMT << 10) |
                                  ((MT::A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
                                  ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+      // block-scaled E4M3 x E4M3 (formats 0), UE8M0 scales (bit 23); per-MMA scale-byte ids
+      // go in bits 5:4 (B) and 30:29 (A)
+      constexpr uint32_t idesc_mx = ((MT::A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
+                                    ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24);
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
         Tile tl;
-        get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+        get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         ok = ptx::mbar_wait(ptx::smem_u32(&c.tempty[acc]), aph ^ 1, abort_flag, WAIT_LIMIT_NS);
@@ -402,6 +493,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
           const uint32_t b_addr = a_addr + C::A_BYTES;
+          uint32_t sfa_t = 0, sfb_t = 0;
+          if constexpr (C::MX) {
+            // scales of this stage into TMEM columns 2*BN (A) and 2*BN + 4 (B)
+            sfa_t = tmem_base + 2 * BN;
+            sfb_t = sfa_t + 4;
+            const uint32_t sf_s = ptx::smem_u32(sf_ring + stage * C::SF_BYTES);
+            ptx::tmem_cp_32x128b_x4(sfa_t, ptx::smem_desc_sf(sf_s));
+            ptx::tmem_cp_32x128b_x4(sfb_t, ptx::smem_desc_sf(sf_s + 512));
+          }
 #pragma unroll
           for (int kk = 0; kk < C::KBLK / C::UMMA_K; ++kk) {
             uint64_t adesc, bdesc;
@@ -414,7 +514,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             else
               bdesc = ptx::smem_desc_sw128(b_addr + kk * 32, 16, 1024);
             const uint32_t accum = (kb | kk) ? 1u : 0u;
-            if constexpr (sizeof(T) == 2) ptx::mma_f16(d_tmem, adesc, bdesc, idesc, accum);
+            if constexpr (C::MX)
+              ptx::mma_mxf8(d_tmem, adesc, bdesc, idesc_mx | ((uint32_t)kk << 4) | ((uint32_t)kk << 29),
+                            sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30), accum);
+            else if constexpr (sizeof(T) == 2) ptx::mma_f16(d_tmem, adesc, bdesc, idesc, accum);
             else ptx::mma_tf32(d_tmem, adesc, bdesc, idesc, accum);
           }
           ptx::tc_commit(ptx::smem_u32(&c.empty[stage]));
@@ -430,6 +533,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else {
     // ================================================================ epilogue
+    using OutT = typename ElemTraits<T>::Out;
     // EPI_WARPS warps: warp w reads TMEM lane quarter w % 4 (one tile row per thread);
     // the two warps of a quarter split the accumulator's columns in halves.
     const int q = warp & 3;
@@ -438,7 +542,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int it = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK>(t, p, c, tl);
+      get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       bool ok = ptx::mbar_wait(ptx::smem_u32(&c.tfull[acc]), aph, abort_flag, WAIT_LIMIT_NS);
@@ -453,7 +557,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // k selected logits.  The first warp of each lane quarter does the work.
         if (half == 0) {
           const bool valid = r < tl.rows;
-          const int64_t row = (int64_t)tl.row0 + r;
+          const int64_t row = (int64_t)tl.orow0 + r;
           const float *bias = static_cast<const float *>(p.aux);
           float *logits = static_cast<float *>(p.out2);
           float tv[MAX_K];
@@ -512,9 +616,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if constexpr (MODE == FWD_GU) {
         // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
         const bool valid = r < tl.rows;
-        const int64_t row = (int64_t)tl.row0 + r;
-        T *hu = static_cast<T *>(p.out0);
-        T *aa = static_cast<T *>(p.out1);
+        const int64_t row = (int64_t)tl.orow0 + r;
+        OutT *hu = static_cast<OutT *>(p.out0);
+        OutT *aa = static_cast<OutT *>(p.out1);
 #pragma unroll 1
         for (int cc = half * (BN / 4); cc < (half + 1) * (BN / 4); cc += 32) {
           float h[32], u[32];
@@ -532,8 +636,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       } else if constexpr (MODE == FWD_DOWN || MODE == DGRAD_GU) {
         const bool valid = r < tl.rows;
-        const int64_t row = (int64_t)tl.row0 + r;
-        T *out = static_cast<T *>(p.out0);
+        const int64_t row = (int64_t)tl.orow0 + r;
+        OutT *out = static_cast<OutT *>(p.out0);
 #pragma unroll 1
         for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
@@ -544,10 +648,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // da -> (dh, du) through the SwiGLU derivative, using the saved h and u.  The
         // loads of the next chunk's h, u are issued before this chunk's math.
         const bool valid = r < tl.rows;
-        const int64_t row = (int64_t)tl.row0 + r;
-        const T *hu = static_cast<const T *>(p.aux);
-        T *dhu = static_cast<T *>(p.out0);
-        constexpr int NV = 32 / Vec<T>::N;   // 16-byte vectors per 32 values
+        const int64_t row = (int64_t)tl.orow0 + r;
+        const OutT *hu = static_cast<const OutT *>(p.aux);
+        OutT *dhu = static_cast<OutT *>(p.out0);
+        constexpr int NV = 32 / Vec<OutT>::N;   // 16-byte vectors per 32 values
         const int c0 = half * (BN / 2), c1 = (half + 1) * (BN / 2);
         uint4 hv[2][NV], uv[2][NV];
         auto issue = [&](int buf, int cc) {
@@ -567,12 +671,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const int col = tl.n_blk * BN + cc;
             uint4 *dh_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + col);
             uint4 *du_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + p.f + col);
-            constexpr int VN = Vec<T>::N;
+            constexpr int VN = Vec<OutT>::N;
 #pragma unroll
             for (int i = 0; i < NV; ++i) {   // one 16-byte vector of h, u at a time
               float h[VN], u[VN], dh[VN], du[VN];
-              Vec<T>::load(hv[j & 1][i], h);
-              Vec<T>::load(uv[j & 1][i], u);
+              Vec<OutT>::load(hv[j & 1][i], h);
+              Vec<OutT>::load(uv[j & 1][i], u);
 #pragma unroll
               for (int v = 0; v < VN; ++v) {
                 const float g = da[i * VN + v];
@@ -580,8 +684,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 dh[v] = g * u[v] * s * (1.0f + h[v] * (1.0f - s));
                 du[v] = g * h[v] * s;
               }
-              dh_dst[i] = Vec<T>::store(dh);
-              du_dst[i] = Vec<T>::store(du);
+              dh_dst[i] = Vec<OutT>::store(dh);
+              du_dst[i] = Vec<OutT>::store(du);
             }
           }
         }
@@ -597,11 +701,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const int col = tl.n_blk * BN + cc;
           if constexpr (MODE == WGRAD_DOWN) {
-            T *out = static_cast<T *>(p.out0);
+            OutT *out = static_cast<OutT *>(p.out0);
             store32(out + ((int64_t)tl.e * p.M + mrow) * p.N + col, v);
           } else {
             // N runs over [dh | du]: columns below f are dW_gate, the rest dW_up
-            T *out = static_cast<T *>(col < p.f ? p.out0 : p.out1);
+            OutT *out = static_cast<OutT *>(col < p.f ? p.out0 : p.out1);
             const int cf = col < p.f ? col : col - p.f;
             store32(out + ((int64_t)tl.e * p.M + mrow) * p.f + cf, v);
           }
@@ -644,7 +748,9 @@ static bool make_tmap(CUtensorMap *m, const void *ptr, int es, uint64_t cols, ui
   cuuint64_t gstride[1] = {cols * (uint64_t)es};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estride[2] = {1, 1};
-  CUresult r = enc(m, es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+  const CUtensorMapDataType dt = es == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  CUresult r = enc(m, dt, 2,
                    const_cast<void *>(ptr), gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -825,6 +931,105 @@ static int router_impl(const Shape &s, const void *x, const void *w_r, const flo
   return launch<bf16, 256, ROUTER>(tA, tB, tB, p, tiles, st);
 }
 
+// ------------------------------------------------------------------ MXFP8 path
+struct MxOp {
+  uint8_t *codes, *scales;
+};
+static MxOp mx_r(void *ws, size_t off, int64_t rows, int64_t cols) {
+  uint8_t *b = static_cast<uint8_t *>(ws) + off;
+  return {b, b + rows * cols};
+}
+
+// Forward with both operands of both GEMMs quantised to MXFP8 (blocks along K).
+static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
+                       const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
+                       cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
+  const MxOp xq = mx_r(ws, L.xq_r, R, s.d), aq = mx_r(ws, L.aq_r, R, s.f);
+  const MxOp wgu = mx_r(ws, L.wgu_c, ed, 2 * s.f), wd = mx_r(ws, L.wd_c, ef, s.d);
+  if (launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st) ||
+      launch_mx_quant_cols_gu(w_gate, w_up, ed, s.f, wgu.codes, wgu.scales, st) ||
+      launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st))
+    return MOE_ERR_CUDA;
+  int *err = err_word(ws);
+  Params p{};
+  p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
+  const int64_t mblocks = (P + BM - 1) / BM + s.E;
+  CUtensorMap tA, tB;
+  // GEMM 1: [h | u] tiles of 64 gate + 64 up columns
+  if (!make_tmap(&tA, xq.codes, 1, s.d, R, 128, BM) || !make_tmap(&tB, wgu.codes, 1, 2 * s.f, ed, 128, 128))
+    return MOE_ERR_CUDA;
+  p.K = s.d; p.N = 2 * s.f; p.out0 = hu; p.out1 = a;
+  p.sfa = xq.scales; p.sfa_ld = s.d / 32; p.sfb = wgu.scales; p.sfb_ld = 2 * s.f;
+  int rc = launch<e4m3, 128, FWD_GU>(tA, tB, tB, p, mblocks * (p.N / 128), st);
+  if (rc) return rc;
+  // GEMM 2: y_perm = a Wd
+  if (launch_mx_quant_rows(a, P, s.f, offsets, s.E, R, aq.codes, aq.scales, st)) return MOE_ERR_CUDA;
+  if (!make_tmap(&tA, aq.codes, 1, s.f, R, 128, BM) || !make_tmap(&tB, wd.codes, 1, s.d, ef, 128, 128))
+    return MOE_ERR_CUDA;
+  p.K = s.f; p.N = s.d; p.out0 = y_perm; p.out1 = nullptr;
+  p.sfa = aq.scales; p.sfa_ld = s.f / 32; p.sfb = wd.scales; p.sfb_ld = s.d;
+  return launch<e4m3, 128, FWD_DOWN>(tA, tB, tB, p, mblocks * (p.N / 128), st);
+}
+
+// Backward with every GEMM operand quantised to MXFP8 along that GEMM's own K.
+static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu, const void *a,
+                       const int32_t *offsets, const void *w_gate, const void *w_up, const void *w_down, void *dhu,
+                       void *dx_perm, void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st) {
+  const WsLayout L = ws_layout(s);
+  const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
+  const MxOp dyq = mx_r(ws, L.dyq_r, R, s.d), dhuq = mx_r(ws, L.dhuq_r, R, 2 * s.f);
+  const MxOp xqt = mx_r(ws, L.xq_t, R, s.d), aqt = mx_r(ws, L.aq_t, R, s.f);
+  const MxOp dyqt = mx_r(ws, L.dyq_t, R, s.d), dhuqt = mx_r(ws, L.dhuq_t, R, 2 * s.f);
+  const MxOp wdr = mx_r(ws, L.wd_r, ef, s.d), wgur = mx_r(ws, L.wgu_r, ed, 2 * s.f);
+  int *err = err_word(ws);
+  Params p{};
+  p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
+  const int64_t mblocks = (P + BM - 1) / BM + s.E;
+  CUtensorMap tA, tB;
+  int rc;
+  // (1) da = dy Wd^T -> SwiGLU backward -> dhu
+  if (launch_mx_quant_rows(dy_perm, P, s.d, offsets, s.E, R, dyq.codes, dyq.scales, st) ||
+      launch_mx_quant_rows(w_down, ef, s.d, nullptr, s.E, ef, wdr.codes, wdr.scales, st))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tA, dyq.codes, 1, s.d, R, 128, BM) || !make_tmap(&tB, wdr.codes, 1, s.d, ef, 128, 128))
+    return MOE_ERR_CUDA;
+  p.K = s.d; p.N = s.f; p.out0 = dhu; p.aux = hu;
+  p.sfa = dyq.scales; p.sfa_ld = s.d / 32; p.sfb = wdr.scales; p.sfb_ld = s.d / 32;
+  rc = launch<e4m3, 128, DGRAD_DOWN>(tA, tB, tB, p, mblocks * (s.f / 128), st);
+  if (rc) return rc;
+  // (2) dWd = a^T dy, K = the tokens of each expert
+  if (launch_mx_quant_cols(a, P, s.f, offsets, s.E, R, aqt.codes, aqt.scales, st) ||
+      launch_mx_quant_cols(dy_perm, P, s.d, offsets, s.E, R, dyqt.codes, dyqt.scales, st))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tA, aqt.codes, 1, s.f, R, 128, 128) || !make_tmap(&tB, dyqt.codes, 1, s.d, R, 128, 128))
+    return MOE_ERR_CUDA;
+  p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
+  p.sfa = aqt.scales; p.sfa_ld = s.f; p.sfb = dyqt.scales; p.sfb_ld = s.d;
+  rc = launch<e4m3, 128, WGRAD_DOWN>(tA, tB, tB, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st);
+  if (rc) return rc;
+  // (3) dx_perm = [dh | du] [Wg | Wu]^T
+  if (launch_mx_quant_rows(dhu, P, 2 * s.f, offsets, s.E, R, dhuq.codes, dhuq.scales, st) ||
+      launch_mx_quant_rows_gu(w_gate, w_up, ed, s.f, wgur.codes, wgur.scales, st))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tA, dhuq.codes, 1, 2 * s.f, R, 128, BM) || !make_tmap(&tB, wgur.codes, 1, 2 * s.f, ed, 128, 128))
+    return MOE_ERR_CUDA;
+  p.K = 2 * s.f; p.N = s.d; p.out0 = dx_perm;
+  p.sfa = dhuq.scales; p.sfa_ld = 2 * s.f / 32; p.sfb = wgur.scales; p.sfb_ld = 2 * s.f / 32;
+  rc = launch<e4m3, 128, DGRAD_GU>(tA, tB, tB, p, mblocks * (s.d / 128), st);
+  if (rc) return rc;
+  // (4) [dWg | dWu] = x^T [dh | du], K = the tokens of each expert
+  if (launch_mx_quant_cols(x_perm, P, s.d, offsets, s.E, R, xqt.codes, xqt.scales, st) ||
+      launch_mx_quant_cols(dhu, P, 2 * s.f, offsets, s.E, R, dhuqt.codes, dhuqt.scales, st))
+    return MOE_ERR_CUDA;
+  if (!make_tmap(&tA, xqt.codes, 1, s.d, R, 128, 128) || !make_tmap(&tB, dhuqt.codes, 1, 2 * s.f, R, 128, 128))
+    return MOE_ERR_CUDA;
+  p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
+  p.sfa = xqt.scales; p.sfa_ld = s.d; p.sfb = dhuqt.scales; p.sfb_ld = 2 * s.f;
+  return launch<e4m3, 128, WGRAD_GU>(tA, tB, tB, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st);
+}
+
 }  // namespace gg
 
 int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float *bias, float *logits,
@@ -835,6 +1040,8 @@ int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
                        cudaStream_t st) {
+  if (s.prec == MOE_PREC_MXFP8)
+    return gg::mx_fwd_impl(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
   if (s.dtype == MOE_BF16)
     return gg::fwd_impl<bf16>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
   return gg::fwd_impl<float>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
@@ -843,12 +1050,15 @@ int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offset
 int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                        const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
                        const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
-                       void *dw_down, int *err, cudaStream_t st) {
+                       void *dw_down, void *ws, cudaStream_t st) {
   // The weight-gradient GEMMs reduce over tokens, which makes both operands MN-major;
   // tf32 MMAs take K-major operands only, so the fp32 backward is not offered.
   if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (s.prec == MOE_PREC_MXFP8)
+    return gg::mx_bwd_impl(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm, dw_gate,
+                           dw_up, dw_down, ws, st);
   return gg::bwd_impl<bf16>(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
-                            dw_gate, dw_up, dw_down, err, st);
+                            dw_gate, dw_up, dw_down, err_word(ws), st);
 }
 
 }  // namespace moe

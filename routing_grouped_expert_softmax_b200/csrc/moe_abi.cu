@@ -21,7 +21,7 @@ int check_cfg(const moe_config *c) {
   if (c->E > MAX_E || c->k > MAX_K || c->k > c->E) return MOE_ERR_UNSUPPORTED;
   if (c->d % 128 || c->f % 128) return MOE_ERR_UNSUPPORTED;
   if (c->T * (int64_t)c->k >= (int64_t(1) << 31)) return MOE_ERR_UNSUPPORTED;
-  if (c->prec == MOE_PREC_MXFP8) return MOE_ERR_UNSUPPORTED;
+  if (c->prec == MOE_PREC_MXFP8 && c->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -140,7 +140,29 @@ int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, const voi
   }
   RETURN_IF(check_ptrs({dy_perm, x_perm, hu, a, dhu, dx_perm}));
   return launch_grouped_bwd(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
-                            dw_gate, dw_up, dw_down, err_word(ws), S(stream));
+                            dw_gate, dw_up, dw_down, ws, S(stream));
+}
+
+int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int32_t *offsets, int32_t E,
+                         int64_t rows_bound, uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 || (offsets && (cols % 128 || E <= 0 || E > MAX_E)))
+    return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (offsets && rows_bound < rows + 127 * (int64_t)E) return MOE_ERR_INVALID_ARG;
+  RETURN_IF(check_ptrs({src, codes}));
+  RETURN_IF(check_ptrs4({scales}));
+  return cuda_rc(launch_mx_quant_rows(src, rows, cols, offsets, E, offsets ? rows_bound : rows, codes, scales,
+                                      S(stream)));
+}
+
+int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, const int32_t *offsets, int32_t E,
+                         int64_t rows_bound, uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 || (offsets && (E <= 0 || E > MAX_E))) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (offsets && rows_bound < rows + 127 * (int64_t)E) return MOE_ERR_INVALID_ARG;
+  if (!src || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  return cuda_rc(launch_mx_quant_cols(src, rows, cols, offsets, E, offsets ? rows_bound : rows, codes, scales,
+                                      S(stream)));
 }
 
 int moe_unpermute_combine(const moe_config *cfg, const void *y_perm, const int32_t *slot_of_pair,
@@ -260,7 +282,7 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
                                        g->dgate, st)));
   RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, sv->hu, sv->a, sv->offsets, w->w_gate, w->w_up,
-                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, err, st));
+                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st));
   if (!router)
     return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, nullptr, nullptr, nullptr, nullptr,
                                         false, g->dx, st));

@@ -125,6 +125,35 @@ __device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem] with E4M3 operands and E8M0 scales per 32 K-elements
+// read from TMEM (sfa, sfb: column addresses; bits 31:30 select the byte of the 32-bit
+// scale word, i.e. which 32-element K-block of the 128-element stage).
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// Copy a 32-row x 128-bit block of shared memory into TMEM, replicated into all four
+// 32-lane quarters (the scale-factor copy).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Descriptor of a contiguous 512-byte block read as 32 rows of 16 bytes (no swizzle;
+// 8-row core matrices 128 bytes apart).
+__device__ __forceinline__ uint64_t smem_desc_sf(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((128u >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
 // 32 lanes x 32 consecutive fp32 columns of TMEM into 32 registers per thread
 // (thread i of the warp gets lane base+i), waiting for completion in the same asm.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {

@@ -31,6 +31,13 @@ def test_every_declared_symbol_is_exported(lib):
     assert sorted(moe.EXPORTED) == names
 
 
+def test_no_unresolved_library_symbols():
+    # every internal launcher the C ABI calls is defined inside the library
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--undefined-only", moe.LIB_PATH], capture_output=True, text=True).stdout
+    assert "moe" not in out, out
+
+
 def test_workspace_size_is_host_only(lib):
     cfg = moe.config(8192, 2048, 128, 4, 1024)
     ws = moe.moe_workspace_size(cfg)
@@ -50,7 +57,7 @@ def test_invalid_config_rejected(lib, bad):
 
 
 @pytest.mark.parametrize("bad", [dict(E=257), dict(k=9), dict(k=9, E=8), dict(d=192), dict(f=200),
-                                 dict(prec=moe.MOE_PREC_MXFP8)])
+                                 dict(prec=moe.MOE_PREC_MXFP8, dtype=moe.MOE_F32)])
 def test_unsupported_config_rejected(lib, bad):
     base = dict(T=16, d=128, E=8, k=2, f=128, dtype=moe.MOE_BF16, prec=moe.MOE_PREC_NATIVE)
     base.update(bad)

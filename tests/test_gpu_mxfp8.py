@@ -1,0 +1,232 @@
+"""MXFP8 on the GPU: the quantisers bit for bit against the oracle's OCP MX rule, and the
+block-scaled grouped GEMMs (forward and backward) against the oracle run on the same
+quantised operands, within 6e-2 max relative error."""
+import numpy as np
+import pytest
+
+import routing_grouped_expert_softmax_b200 as moe
+from oracle import moe_ref as ref
+from routing_grouped_expert_softmax_b200 import inputs as gen
+from tests.gpu_util import dev, dev_f32, dev_i32, grid, host, offsets_of, random_counts, rel_err
+
+pytestmark = pytest.mark.gpu
+
+TOL_MX = 6e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    import torch
+    assert torch.cuda.is_available()
+    from routing_grouped_expert_softmax_b200 import build
+    build.build()
+
+
+def _special_data(rows, cols, seed):
+    """bf16 values with the quantiser's edge cases planted in some 32-blocks."""
+    rng = np.random.default_rng(seed)
+    v = rng.standard_normal((rows, cols)).astype(np.float32) * np.exp(rng.standard_normal((rows, 1)) * 2)
+    g = ref.e4m3_grid()
+    if rows >= 8 and cols >= 64:
+        v[0, :32] = 0.0                                   # amax = 0 -> scale 2^-127, codes 0
+        v[1, :32] = 1e-30 * rng.standard_normal(32)       # tiny block
+        v[2, :32] = 500.0 * rng.standard_normal(32)       # large values, saturating at 448 X
+        v[3, :32] = -0.0                                  # signed zero
+        mids = (g[:-1] + g[1:]) / 2                       # exact midpoints between codes (X = 1)
+        v[4, :32] = np.concatenate([[256.0], rng.choice(mids[mids < 256], 31)])
+        v[5, 32:64] = -v[4, :32]
+    return gen.bf16_round(v)
+
+
+def _codes_scales_rows(v):
+    codes, scales, _ = ref.mx_quantize(v.astype(np.float64), axis=1)
+    return codes, scales
+
+
+@pytest.mark.parametrize("rows,cols", [(1, 32), (37, 128), (300, 2048), (8, 4096)])
+def test_mx_quantize_rows_identity(rows, cols):
+    import torch
+    v = _special_data(rows, cols, rows)
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(rows, cols // 32, dtype=torch.uint8, device="cuda")
+    moe.moe_mx_quantize_rows(dev(v, "bf16"), rows, cols, None, 0, rows, codes, scales)
+    rc, rs = _codes_scales_rows(v)
+    assert np.array_equal(host(codes), rc)
+    assert np.array_equal(host(scales), rs)
+
+
+@pytest.mark.parametrize("rows,cols", [(32, 32), (96, 256), (4096, 128), (100, 64)])
+def test_mx_quantize_cols_identity(rows, cols):
+    import torch
+    v = _special_data(rows, cols, rows + 1).T.copy().T.copy()
+    nb = (rows + 31) // 32
+    codes = torch.empty(nb * 32, cols, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(nb, cols, dtype=torch.uint8, device="cuda")
+    moe.moe_mx_quantize_cols(dev(v, "bf16"), rows, cols, None, 0, rows, codes, scales)
+    pad = np.zeros((nb * 32, cols))
+    pad[:rows] = v
+    rc, rs, _ = ref.mx_quantize(pad, axis=0)
+    assert np.array_equal(host(codes)[:rows], rc[:rows])
+    assert np.array_equal(host(scales), rs)
+
+
+def _padded(v, offsets):
+    """The expert-padded layout: each expert's rows start at a multiple of 128."""
+    E = len(offsets) - 1
+    counts = np.diff(offsets)
+    pre = np.concatenate([[0], np.cumsum((counts + 127) // 128)])
+    out = np.zeros((int(pre[-1]) * 128, v.shape[1]))
+    for e in range(E):
+        out[pre[e] * 128: pre[e] * 128 + counts[e]] = v[offsets[e]:offsets[e + 1]]
+    return out
+
+
+@pytest.mark.parametrize("E,cols", [(8, 256), (128, 128), (3, 512)])
+def test_mx_quantize_expert_padded(E, cols):
+    import torch
+    rng = np.random.default_rng(E)
+    counts = random_counts(E, 150, rng)
+    offsets = offsets_of(counts)
+    P = int(offsets[-1])
+    v = _special_data(P, cols, E)
+    bound = P + 127 * E
+    d_off = dev_i32(offsets)
+    cr = torch.full((bound, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    sr = torch.full((bound, cols // 32), 0xAB, dtype=torch.uint8, device="cuda")
+    moe.moe_mx_quantize_rows(dev(v, "bf16"), P, cols, d_off, E, bound, cr, sr)
+    pv = _padded(v, offsets)
+    n = pv.shape[0]
+    rc, rs, _ = ref.mx_quantize(pv, axis=1)
+    assert np.array_equal(host(cr)[:n], rc) and np.array_equal(host(sr)[:n], rs)
+    ct = torch.full((bound, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    st = torch.full(((bound + 31) // 32, cols), 0xAB, dtype=torch.uint8, device="cuda")
+    moe.moe_mx_quantize_cols(dev(v, "bf16"), P, cols, d_off, E, bound, ct, st)
+    tc, ts, _ = ref.mx_quantize(pv, axis=0)
+    assert np.array_equal(host(ct)[:n], tc) and np.array_equal(host(st)[:n // 32], ts)
+
+
+# ------------------------------------------------------------------ grouped GEMMs
+
+MX_CASES = [
+    # d, f, E, counts kind
+    (256, 256, 8, "random"),
+    (128, 128, 4, "random"),
+    (384, 256, 3, "one"),
+    (2048, 1024, 8, "random"),
+]
+
+
+def _mx_counts(kind, E, rng):
+    if kind == "one":
+        c = np.zeros(E, np.int64)
+        c[1] = 300
+        return c
+    return random_counts(E, 300, rng)
+
+
+@pytest.mark.parametrize("d,f,E,kind", MX_CASES)
+def test_mx_grouped_swiglu_fwd(d, f, E, kind):
+    import torch
+    rng = np.random.default_rng(d + f + E)
+    offsets = offsets_of(_mx_counts(kind, E, rng))
+    P = int(offsets[-1])
+    x = grid(rng.standard_normal((P, d), dtype=np.float32), "bf16")
+    wg = grid(rng.standard_normal((E, d, f), dtype=np.float32) / np.sqrt(d), "bf16")
+    wu = grid(rng.standard_normal((E, d, f), dtype=np.float32) / np.sqrt(d), "bf16")
+    wd = grid(rng.standard_normal((E, f, d), dtype=np.float32) / np.sqrt(f), "bf16")
+    cfg = moe.config(P, d, E, 1, f, dtype="bf16", prec="mxfp8")
+    ws = moe.alloc_workspace(cfg)
+    hu = torch.empty(P, 2 * f, dtype=torch.bfloat16, device="cuda")
+    a = torch.empty(P, f, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(P, d, dtype=torch.bfloat16, device="cuda")
+    moe.moe_grouped_swiglu_fwd(cfg, dev(x, "bf16"), dev_i32(offsets), dev(wg, "bf16"), dev(wu, "bf16"),
+                               dev(wd, "bf16"), hu, a, y, ws)
+    assert moe.moe_get_error(ws) == 0
+    h, u, ra, ry = ref.grouped_swiglu_mx(x, offsets, wg, wu, wd)
+    g = host(hu)
+    assert rel_err(g[:, :f], h) <= TOL_MX
+    assert rel_err(g[:, f:], u) <= TOL_MX
+    assert rel_err(host(a), ra) <= TOL_MX
+    assert rel_err(host(y), ry) <= TOL_MX
+    # h and u come from exactly quantised operands: far tighter than the MX bar
+    assert rel_err(g[:, :f], h) <= 1e-2
+
+
+@pytest.mark.parametrize("d,f,E,kind", MX_CASES)
+def test_mx_grouped_swiglu_bwd(d, f, E, kind):
+    import torch
+    rng = np.random.default_rng(3 * d + f + E)
+    counts = _mx_counts(kind, E, rng)
+    offsets = offsets_of(counts)
+    P = int(offsets[-1])
+    x = grid(rng.standard_normal((P, d), dtype=np.float32), "bf16")
+    dy = grid(rng.standard_normal((P, d), dtype=np.float32), "bf16")
+    h = grid(rng.standard_normal((P, f), dtype=np.float32), "bf16")
+    u = grid(rng.standard_normal((P, f), dtype=np.float32), "bf16")
+    a = grid(rng.standard_normal((P, f), dtype=np.float32), "bf16")
+    wg = grid(rng.standard_normal((E, d, f), dtype=np.float32) / np.sqrt(d), "bf16")
+    wu = grid(rng.standard_normal((E, d, f), dtype=np.float32) / np.sqrt(d), "bf16")
+    wd = grid(rng.standard_normal((E, f, d), dtype=np.float32) / np.sqrt(f), "bf16")
+    cfg = moe.config(P, d, E, 1, f, dtype="bf16", prec="mxfp8")
+    ws = moe.alloc_workspace(cfg)
+    dhu = torch.empty(P, 2 * f, dtype=torch.bfloat16, device="cuda")
+    dxp = torch.empty(P, d, dtype=torch.bfloat16, device="cuda")
+    dwg = torch.full((E, d, f), 7.0, dtype=torch.bfloat16, device="cuda")
+    dwu = torch.full((E, d, f), 7.0, dtype=torch.bfloat16, device="cuda")
+    dwd = torch.full((E, f, d), 7.0, dtype=torch.bfloat16, device="cuda")
+    moe.moe_grouped_swiglu_bwd(cfg, dev(dy, "bf16"), dev(x, "bf16"), dev(np.concatenate([h, u], 1), "bf16"),
+                               dev(a, "bf16"), dev_i32(offsets), dev(wg, "bf16"), dev(wu, "bf16"), dev(wd, "bf16"),
+                               dhu, dxp, dwg, dwu, dwd, ws)
+    assert moe.moe_get_error(ws) == 0
+    r = ref.grouped_swiglu_bwd_mx(dy, x, h, u, a, offsets, wg, wu, wd)
+    g = host(dhu)
+    assert rel_err(g[:, :f], r["dh"]) <= TOL_MX
+    assert rel_err(g[:, f:], r["du"]) <= TOL_MX
+    assert rel_err(host(dxp), r["dx_perm"]) <= TOL_MX
+    for name, t in (("dw_gate", dwg), ("dw_up", dwu), ("dw_down", dwd)):
+        assert rel_err(host(t), r[name]) <= TOL_MX, name
+    for e in np.nonzero(counts == 0)[0]:
+        assert np.all(host(dwg[e]) == 0) and np.all(host(dwd[e]) == 0)
+
+
+def test_mx_layer_against_oracle_and_bf16_path():
+    import torch
+    T, d, E, k, f = 512, 256, 16, 4, 256
+    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=5)
+    outs = {}
+    for prec in ("native", "mxfp8"):
+        cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
+        ws = moe.alloc_workspace(cfg)
+        saved = moe.alloc_saved(cfg)
+        grads = moe.alloc_grads(cfg)
+        w = [dev(a_, "bf16") for a_ in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down)]
+        wts = moe.layer_weights(w[0], None, w[1], w[2], w[3])
+        x = dev(inp.x, "bf16")
+        y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_layer_fwd(cfg, wts, x, y, saved, ws)
+        moe.moe_layer_bwd(cfg, wts, x, dev(inp.dy, "bf16"), saved, grads, ws)
+        assert moe.moe_get_error(ws) == 0
+        outs[prec] = (host(y), {n: host(grads[n]) for n in ("dx", "dw_gate", "dw_up", "dw_down", "dw_router")},
+                      host(saved["topk_idx"]))
+    # the oracle with every GEMM operand quantised, on the routing both paths share
+    fwd = ref.layer_fwd(inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k)
+    assert np.array_equal(outs["mxfp8"][2], fwd["idx"])
+    h, u, a, y_perm = ref.grouped_swiglu_mx(fwd["x_perm"], fwd["offsets"], inp.w_gate, inp.w_up, inp.w_down)
+    Y = ref.combine(y_perm, fwd["slot_of_pair"], fwd["gate"])
+    dy_perm, dgate = ref.combine_bwd(inp.dy, y_perm, fwd["slot_of_pair"], fwd["gate"])
+    # the layer keeps h, u, a and dy_perm in bf16; the backward GEMMs quantise those tensors
+    b = ref.bf16_rne
+    g = ref.grouped_swiglu_bwd_mx(b(dy_perm), fwd["x_perm"], b(h), b(u), b(a), fwd["offsets"], inp.w_gate,
+                                  inp.w_up, inp.w_down)
+    dx = ref.unpermute_sum(g["dx_perm"], fwd["slot_of_pair"], T, k)
+    dz, dwr, dxr = ref.route_bwd(dgate, fwd["gate"], fwd["idx"], inp.x, inp.w_r)
+    want = dict(dx=dx + dxr, dw_gate=g["dw_gate"], dw_up=g["dw_up"], dw_down=g["dw_down"], dw_router=dwr)
+    ymx, gmx, _ = outs["mxfp8"]
+    assert rel_err(ymx, Y) <= TOL_MX
+    for n, ref_v in want.items():
+        assert rel_err(gmx[n], ref_v) <= TOL_MX, n
+    # and MXFP8 stays close to the bf16 path (quantisation error only)
+    ybf, gbf, _ = outs["native"]
+    assert 0 < rel_err(ymx, ybf) <= 0.1
+    for n in ("dx", "dw_gate", "dw_down"):
+        assert rel_err(gmx[n], gbf[n]) <= 0.15, n
