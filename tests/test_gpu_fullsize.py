@@ -28,7 +28,9 @@ CONFIGS = {
     "e128": dict(T=8192, d=2048, E=128, k=4, f=1024, skew=False, routing="router"),
     "e128_t16k_skew": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=True, routing="router"),
     "e128_t16k_uniform": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=False, routing="uniform"),
+    "e128_t16k_mxfp8": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=False, routing="router", prec="mxfp8"),
 }
+TOL_MX = 6e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -46,37 +48,83 @@ def clear_tokens(z, delta, k):
     return np.all(gaps > 2 * delta[:, None], axis=1)
 
 
-def _token_oracle(inp, t, idx_t, g_t, router):
-    """Oracle y[t] and dx[t] of one token from its routing (experts idx_t, gates g_t)."""
+class _MxWeights:
+    """The oracle's MXFP8 copies of one expert's weights, along each GEMM's own K."""
+
+    def __init__(self, inp):
+        self.inp, self.cache = inp, {}
+
+    def __call__(self, e):
+        if e not in self.cache:
+            q = lambda w, ax: ref.mx_quantize(np.asarray(w, np.float64), axis=ax)[2]
+            i = self.inp
+            self.cache[e] = dict(g=q(i.w_gate[e], 0), u=q(i.w_up[e], 0), d=q(i.w_down[e], 0),
+                                 dT=q(i.w_down[e], 1), gT=q(i.w_gate[e], 1), uT=q(i.w_up[e], 1))
+        return self.cache[e]
+
+
+def _token_oracle(inp, t, idx_t, g_t, router, mx=None):
+    """Oracle y[t] and dx[t] of one token from its routing (experts idx_t, gates g_t).
+    With mx, every GEMM operand is MXFP8-quantised along its own K, as the MXFP8 layer
+    does (row-wise blocks of one token's vectors, and the bf16 tensors it stores)."""
     x = inp.x[t:t + 1].astype(np.float64)
     dY = inp.dy[t].astype(np.float64)
     y = np.zeros(inp.d)
     dx = np.zeros(inp.d)
     dg = np.zeros(len(idx_t))
+    q = lambda v: ref.mx_quantize(v, axis=1)[2]
+    b = ref.bf16_rne
     for j, e in enumerate(idx_t):
-        h, u, a, ye = ref.expert_swiglu(x, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+        if mx is None:
+            h, u, a, ye = ref.expert_swiglu(x, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+            da = (g_t[j] * dY)[None, :] @ inp.w_down[e].astype(np.float64).T
+            dh, du = ref.swiglu_bwd(da, h, u)
+            dx += (dh @ inp.w_gate[e].astype(np.float64).T + du @ inp.w_up[e].astype(np.float64).T)[0]
+        else:
+            w = mx(e)
+            xq = q(x)
+            h, u = xq @ w["g"], xq @ w["u"]
+            a = ref.silu(h) * u
+            ye = q(b(a)) @ w["d"]
+            da = q(b(g_t[j] * dY)[None, :]) @ w["dT"].T
+            dh, du = ref.swiglu_bwd(da, b(h), b(u))
+            dhu = q(b(np.concatenate([dh, du], axis=1)))
+            f = inp.f
+            dx += (dhu[:, :f] @ w["gT"].T + dhu[:, f:] @ w["uT"].T)[0]
         y += g_t[j] * ye[0]
         dg[j] = dY @ ye[0]
-        da = (g_t[j] * dY)[None, :] @ inp.w_down[e].astype(np.float64).T
-        dh, du = ref.swiglu_bwd(da, h, u)
-        dx += (dh @ inp.w_gate[e].astype(np.float64).T + du @ inp.w_up[e].astype(np.float64).T)[0]
     if router:
         dz = ref.gate_logit_grad(dg[None, :], np.asarray(g_t)[None, :], np.asarray(idx_t)[None, :], inp.E)
         dx += (dz @ inp.w_r.astype(np.float64).T)[0]
     return y, dx
 
 
-def _expert_oracle(inp, e, idx, gate):
-    """Oracle weight gradients of expert e from the routing of every token."""
+def _expert_oracle(inp, e, idx, gate, mx=None):
+    """Oracle weight gradients of expert e from the routing of every token (with mx: the
+    MXFP8 layer's operands, the token-axis operands blocked 32 rows at a time from the
+    expert's first row)."""
     pairs = np.nonzero(idx.ravel() == e)[0]           # pair order = the stable slot order
     toks = pairs // inp.k
     g = gate.ravel()[pairs].astype(np.float64)
     X = inp.x[toks].astype(np.float64)
-    h, u, a, _ = ref.expert_swiglu(X, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
-    dy = g[:, None] * inp.dy[toks].astype(np.float64)
-    da = dy @ inp.w_down[e].astype(np.float64).T
-    dh, du = ref.swiglu_bwd(da, h, u)
-    return X.T @ dh, X.T @ du, a.T @ dy
+    if mx is None:
+        h, u, a, _ = ref.expert_swiglu(X, inp.w_gate[e], inp.w_up[e], inp.w_down[e])
+        dy = g[:, None] * inp.dy[toks].astype(np.float64)
+        da = dy @ inp.w_down[e].astype(np.float64).T
+        dh, du = ref.swiglu_bwd(da, h, u)
+        return X.T @ dh, X.T @ du, a.T @ dy
+    w, b, f = mx(e), ref.bf16_rne, inp.f
+    q = lambda v: ref.mx_quantize(v, axis=1)[2]
+    qt = lambda v: ref.mx_quantize_grouped_rows(v, np.array([0, v.shape[0]]))
+    xq = q(X)
+    h, u = xq @ w["g"], xq @ w["u"]
+    a = b(ref.silu(h) * u)
+    dy = b(g[:, None] * inp.dy[toks].astype(np.float64))
+    da = q(dy) @ w["dT"].T
+    dh, du = ref.swiglu_bwd(da, b(h), b(u))
+    dhu = b(np.concatenate([dh, du], axis=1))
+    dwgu = qt(X).T @ qt(dhu)
+    return dwgu[:, :f], dwgu[:, f:], qt(a).T @ qt(dy)
 
 
 @pytest.mark.parametrize("name", list(CONFIGS))
@@ -85,7 +133,10 @@ def test_fullsize(name):
     c = CONFIGS[name]
     T, d, E, k, f = c["T"], c["d"], c["E"], c["k"], c["f"]
     inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=0, skew=c["skew"])
-    cfg = moe.config(T, d, E, k, f, dtype="bf16")
+    prec = c.get("prec", "native")
+    cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
+    mx = _MxWeights(inp) if prec == "mxfp8" else None
+    tol, tol_c = (TOL_MX, TOL_MX) if mx else (TOL, TOL_COMBINE)
     ws = moe.alloc_workspace(cfg)
     saved = moe.alloc_saved(cfg)
     router = c["routing"] == "router"
@@ -145,18 +196,18 @@ def test_fullsize(name):
     gy, gdx = host(y), host(grads["dx"])
     ys, dxs = [], []
     for t in toks:
-        yt, dxt = _token_oracle(inp, t, ridx[t], rgate[t], router)
+        yt, dxt = _token_oracle(inp, t, ridx[t], rgate[t], router, mx)
         ys.append(yt)
         dxs.append(dxt)
-    assert rel_err(gy[toks], np.array(ys)) <= TOL_COMBINE
-    assert rel_err(gdx[toks], np.array(dxs)) <= TOL
+    assert rel_err(gy[toks], np.array(ys)) <= tol_c
+    assert rel_err(gdx[toks], np.array(dxs)) <= tol
 
     # sampled experts' weight gradients (only experts all of whose tokens route clearly)
     touch = (ridx[:, :, None] == np.arange(E)).any(axis=1) | (gi[:, :, None] == np.arange(E)).any(axis=1)
     owners = [e for e in range(E) if clear[touch[:, e]].all()]
     picks = [owners[0], owners[len(owners) // 2], owners[-1]] if E > 8 else owners[:1]
     for e in picks:
-        dwg, dwu, dwd = _expert_oracle(inp, e, ridx, rgate)
-        assert rel_err(host(grads["dw_gate"][e]), dwg) <= TOL, e
-        assert rel_err(host(grads["dw_up"][e]), dwu) <= TOL, e
-        assert rel_err(host(grads["dw_down"][e]), dwd) <= TOL, e
+        dwg, dwu, dwd = _expert_oracle(inp, e, ridx, rgate, mx)
+        assert rel_err(host(grads["dw_gate"][e]), dwg) <= tol, e
+        assert rel_err(host(grads["dw_up"][e]), dwu) <= tol, e
+        assert rel_err(host(grads["dw_down"][e]), dwd) <= tol, e
