@@ -197,6 +197,50 @@ __device__ __forceinline__ void store32(T *dst, const float (&v)[32]) {
 #pragma unroll
   for (int i = 0; i < 32 / N; ++i) d4[i] = Vec<T>::store(&v[i * N]);
 }
+__device__ __forceinline__ uint4 shfl_xor4(uint4 v, int m) {
+  v.x = __shfl_xor_sync(0xffffffffu, v.x, m);
+  v.y = __shfl_xor_sync(0xffffffffu, v.y, m);
+  v.z = __shfl_xor_sync(0xffffffffu, v.z, m);
+  v.w = __shfl_xor_sync(0xffffffffu, v.w, m);
+  return v;
+}
+
+// Store a 32-row x 32-column slab held one row per lane (lane l: slab row l, values v).
+// dst points at column 0 of slab row 0; ld is the row stride in elements; rows >= nvalid
+// are not written.  Every lane of the warp must call it.
+// bf16: a 4x4 transpose of 16-byte pieces inside each group of four lanes, so that each
+// store instruction writes eight whole 64-byte row segments instead of 32 scattered
+// 16-byte pieces.  fp32: each lane writes its own row.
+template <typename T>
+__device__ __forceinline__ void store_slab(T *dst, int64_t ld, int nvalid, const float (&v)[32]) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (sizeof(T) == 2) {
+    uint4 q[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) q[c] = Vec<T>::store(&v[8 * c]);
+    const int j = lane & 3;
+    {  // exchange with lane ^ 1: 1x1 blocks
+      const bool odd = j & 1;
+      uint4 r0 = shfl_xor4(odd ? q[0] : q[1], 1);
+      uint4 r1 = shfl_xor4(odd ? q[2] : q[3], 1);
+      if (odd) { q[0] = r0; q[2] = r1; } else { q[1] = r0; q[3] = r1; }
+    }
+    {  // exchange with lane ^ 2: 2x2 blocks
+      const bool hi = j & 2;
+      uint4 r0 = shfl_xor4(hi ? q[0] : q[2], 2);
+      uint4 r1 = shfl_xor4(hi ? q[1] : q[3], 2);
+      if (hi) { q[0] = r0; q[1] = r1; } else { q[2] = r0; q[3] = r1; }
+    }
+    // lane (4g + j) now holds piece j of slab rows 4g + 0..3
+    const int g4 = lane & ~3;
+#pragma unroll
+    for (int s2 = 0; s2 < 4; ++s2)
+      if (g4 + s2 < nvalid) reinterpret_cast<uint4 *>(dst + (int64_t)(g4 + s2) * ld)[j] = q[s2];
+  } else {
+    if (lane < nvalid) store32(dst + (int64_t)lane * ld, v);
+  }
+}
+
 template <typename T>
 __device__ __forceinline__ void load32(const T *src, float (&v)[32]) {
   const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
@@ -616,7 +660,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else if constexpr (MODE == FWD_GU) {
         // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
         const bool valid = r < tl.rows;
-        const int64_t row = (int64_t)tl.orow0 + r;
+        const int nvalid = min(32, max(0, tl.rows - q * 32));
+        const int64_t srow = (int64_t)tl.orow0 + q * 32;      // output row of slab row 0
         OutT *hu = static_cast<OutT *>(p.out0);
         OutT *aa = static_cast<OutT *>(p.out1);
 #pragma unroll 1
@@ -624,73 +669,73 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           float h[32], u[32];
           ptx::tmem_ld32(taddr + cc, h);
           ptx::tmem_ld32(taddr + BN / 2 + cc, u);
-          if (valid) {
-            const int col = tl.n_blk * (BN / 2) + cc;
-            store32(hu + row * 2 * p.f + col, h);
-            store32(hu + row * 2 * p.f + p.f + col, u);
-            float a[32];
+          const int col = tl.n_blk * (BN / 2) + cc;
+          store_slab(hu + srow * 2 * p.f + col, 2 * p.f, nvalid, h);
+          store_slab(hu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, u);
+          float a[32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) a[i] = h[i] * sigmoidf_(h[i]) * u[i];
-            store32(aa + row * p.f + col, a);
-          }
+          for (int i = 0; i < 32; ++i) a[i] = valid ? h[i] * sigmoidf_(h[i]) * u[i] : 0.f;
+          store_slab(aa + srow * p.f + col, p.f, nvalid, a);
         }
       } else if constexpr (MODE == FWD_DOWN || MODE == DGRAD_GU) {
-        const bool valid = r < tl.rows;
-        const int64_t row = (int64_t)tl.orow0 + r;
+        const int nvalid = min(32, max(0, tl.rows - q * 32));
+        const int64_t srow = (int64_t)tl.orow0 + q * 32;
         OutT *out = static_cast<OutT *>(p.out0);
 #pragma unroll 1
         for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
           ptx::tmem_ld32(taddr + cc, v);
-          if (valid) store32(out + row * p.N + tl.n_blk * BN + cc, v);
+          store_slab(out + srow * p.N + tl.n_blk * BN + cc, p.N, nvalid, v);
         }
       } else if constexpr (MODE == DGRAD_DOWN) {
         // da -> (dh, du) through the SwiGLU derivative, using the saved h and u.  The
         // loads of the next chunk's h, u are issued before this chunk's math.
         const bool valid = r < tl.rows;
+        const int nvalid = min(32, max(0, tl.rows - q * 32));
         const int64_t row = (int64_t)tl.orow0 + r;
+        const int64_t srow = (int64_t)tl.orow0 + q * 32;
         const OutT *hu = static_cast<const OutT *>(p.aux);
         OutT *dhu = static_cast<OutT *>(p.out0);
         constexpr int NV = 32 / Vec<OutT>::N;   // 16-byte vectors per 32 values
+        constexpr int VN = Vec<OutT>::N;
         const int c0 = half * (BN / 2), c1 = (half + 1) * (BN / 2);
         uint4 hv[2][NV], uv[2][NV];
         auto issue = [&](int buf, int cc) {
           const uint4 *hs = reinterpret_cast<const uint4 *>(hu + row * 2 * p.f + tl.n_blk * BN + cc);
           const uint4 *us = reinterpret_cast<const uint4 *>(hu + row * 2 * p.f + p.f + tl.n_blk * BN + cc);
 #pragma unroll
-          for (int i = 0; i < NV; ++i) { hv[buf][i] = __ldg(hs + i); uv[buf][i] = __ldg(us + i); }
+          for (int i = 0; i < NV; ++i) {
+            hv[buf][i] = valid ? __ldg(hs + i) : make_uint4(0, 0, 0, 0);
+            uv[buf][i] = valid ? __ldg(us + i) : make_uint4(0, 0, 0, 0);
+          }
         };
-        if (valid) issue(0, c0);
+        issue(0, c0);
 #pragma unroll
         for (int j = 0; j < (BN / 2) / 32; ++j) {
           const int cc = c0 + j * 32;
           float da[32];
           ptx::tmem_ld32(taddr + cc, da);
-          if (valid) {
-            if (cc + 32 < c1) issue((j + 1) & 1, cc + 32);
-            const int col = tl.n_blk * BN + cc;
-            uint4 *dh_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + col);
-            uint4 *du_dst = reinterpret_cast<uint4 *>(dhu + row * 2 * p.f + p.f + col);
-            constexpr int VN = Vec<OutT>::N;
+          if (cc + 32 < c1) issue((j + 1) & 1, cc + 32);
+          float dh[32], du[32];
 #pragma unroll
-            for (int i = 0; i < NV; ++i) {   // one 16-byte vector of h, u at a time
-              float h[VN], u[VN], dh[VN], du[VN];
-              Vec<OutT>::load(hv[j & 1][i], h);
-              Vec<OutT>::load(uv[j & 1][i], u);
+          for (int i = 0; i < NV; ++i) {   // one 16-byte vector of h, u at a time
+            float h[VN], u[VN];
+            Vec<OutT>::load(hv[j & 1][i], h);
+            Vec<OutT>::load(uv[j & 1][i], u);
 #pragma unroll
-              for (int v = 0; v < VN; ++v) {
-                const float g = da[i * VN + v];
-                const float s = sigmoidf_(h[v]);
-                dh[v] = g * u[v] * s * (1.0f + h[v] * (1.0f - s));
-                du[v] = g * h[v] * s;
-              }
-              dh_dst[i] = Vec<OutT>::store(dh);
-              du_dst[i] = Vec<OutT>::store(du);
+            for (int v = 0; v < VN; ++v) {
+              const float g = da[i * VN + v];
+              const float s = sigmoidf_(h[v]);
+              dh[i * VN + v] = g * u[v] * s * (1.0f + h[v] * (1.0f - s));
+              du[i * VN + v] = g * h[v] * s;
             }
           }
+          const int col = tl.n_blk * BN + cc;
+          store_slab(dhu + srow * 2 * p.f + col, 2 * p.f, nvalid, dh);
+          store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
         }
-      } else {  // weight gradients: row r of the [M x N] block of expert e
-        const int64_t mrow = (int64_t)tl.m_blk * BM + r;
+      } else {  // weight gradients: slab of rows q*32.. of the [M x N] block of expert e
+        const int64_t srow = (int64_t)tl.e * p.M + (int64_t)tl.m_blk * BM + q * 32;
 #pragma unroll 1
         for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
@@ -702,12 +747,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int col = tl.n_blk * BN + cc;
           if constexpr (MODE == WGRAD_DOWN) {
             OutT *out = static_cast<OutT *>(p.out0);
-            store32(out + ((int64_t)tl.e * p.M + mrow) * p.N + col, v);
+            store_slab(out + srow * p.N + col, p.N, 32, v);
           } else {
             // N runs over [dh | du]: columns below f are dW_gate, the rest dW_up
             OutT *out = static_cast<OutT *>(col < p.f ? p.out0 : p.out1);
             const int cf = col < p.f ? col : col - p.f;
-            store32(out + ((int64_t)tl.e * p.M + mrow) * p.f + cf, v);
+            store_slab(out + srow * p.f + cf, p.f, 32, v);
           }
         }
       }
