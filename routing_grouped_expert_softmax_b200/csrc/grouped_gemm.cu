@@ -71,17 +71,21 @@ template <> struct ElemTraits<e4m3> {
   using Out = bf16;
 };
 
-template <typename T, int BN> struct Cfg {
+// BN: the MMA's N.  CG: CTAs per MMA (1, or 2 for a 256-row pair tile in which each CTA
+// holds 128 rows of A and BN/2 columns of B).
+template <typename T, int BN, int CG = 1> struct Cfg {
   static constexpr bool MX = (ElemTraits<T>::ES == 1);
+  static constexpr int BMP = BM * CG;                   // rows of an MMA tile (pair)
+  static constexpr int BNC = BN / CG;                   // columns of B held by one CTA
   static constexpr int ES = ElemTraits<T>::ES;
   static constexpr int KBLK = 128 / ES;                 // K elements per stage (one 128-B swizzle row)
   static constexpr int UMMA_K = 32 / ES;                // K per tcgen05.mma
   static constexpr int BOX_MN = 128 / ES;               // MN elements per TMA box of an MN-major operand
   static constexpr int BOX_BYTES = KBLK * 128;          // bytes of one [KBLK x BOX_MN] box
   static constexpr int A_BYTES = BM * KBLK * ES;
-  static constexpr int B_BYTES = BN * KBLK * ES;
+  static constexpr int B_BYTES = BNC * KBLK * ES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (BN == 256) ? 4 : (BN == 128 ? 6 : 8);
+  static constexpr int STAGES = (STAGE_BYTES >= 48 * 1024) ? 4 : (STAGE_BYTES >= 32 * 1024 ? 6 : 8);
   // two accumulators; MXFP8 adds 8 columns of scale factors (A: 4, B: 4) after them
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
   static constexpr int SF_BYTES = MX ? 1024 : 0;        // per stage: 512-byte scale blocks of A and B
@@ -117,6 +121,7 @@ __device__ __forceinline__ void note_fail(const Params &p, int role, int t, int 
 struct Tile {
   int e, m_blk, n_blk;
   int orow0;      // first output row (row-grouped modes)
+  int mcol0;      // weight-gradient modes: first M index (A column, output row) of this CTA
   int row0;       // first A row (row-grouped) or first K row (weight-gradient)
   int rows;       // valid rows (row-grouped) or valid K rows (weight-gradient)
   int num_kb;
@@ -135,8 +140,9 @@ struct Ctrl {
   int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
 };
 
-template <int MODE, int BN, int KBLK, bool MX>
-__device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl) {
+template <int MODE, int BN, int KBLK, bool MX, int CG = 1>
+__device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl, int rank = 0) {
+  constexpr int BMP = BM * CG;
   if constexpr (MODE == ROUTER) {
     tl.e = 0;
     tl.m_blk = t;
@@ -145,11 +151,12 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.rows = min(BM, p.P - t * BM);
     tl.num_kb = p.K / KBLK;
   } else if constexpr (ModeTraits<MODE>::WGRAD) {
-    const int mt = p.M / BM, nt = p.N / BN;
+    const int mt = p.M / BMP, nt = p.N / BN;
     tl.e = t / (mt * nt);
     int r = t - tl.e * mt * nt;
     tl.m_blk = r / nt;
     tl.n_blk = r - tl.m_blk * nt;
+    tl.mcol0 = tl.m_blk * BMP + rank * BM;
     int lo = p.offsets[tl.e], hi = p.offsets[tl.e + 1];
     tl.rows = hi - lo;
     if constexpr (MX) {
@@ -174,18 +181,19 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.e = lo;
     tl.m_blk = g - c.prefix[lo];
     int off = p.offsets[lo], cnt = p.offsets[lo + 1] - off;
-    tl.orow0 = off + tl.m_blk * BM;
+    tl.orow0 = off + tl.m_blk * BMP + rank * BM;   // this CTA's rows of the (pair) tile
     tl.row0 = MX ? g * BM : tl.orow0;   // quantised A: expert buffers padded to 128 rows
-    tl.rows = min(BM, cnt - tl.m_blk * BM);
+    tl.rows = min(BM, cnt - tl.m_blk * BMP - rank * BM);   // may be <= 0 for the second CTA
+    tl.mcol0 = 0;
     tl.num_kb = p.K / KBLK;
   }
   return true;
 }
 
-template <int MODE, int BN>
+template <int MODE, int BN, int CG = 1>
 __device__ __forceinline__ int total_tiles(const Params &p, const Ctrl &c) {
   if constexpr (MODE == ROUTER) return (p.P + BM - 1) / BM;
-  else if constexpr (ModeTraits<MODE>::WGRAD) return p.E * (p.M / BM) * (p.N / BN);
+  else if constexpr (ModeTraits<MODE>::WGRAD) return p.E * (p.M / (BM * CG)) * (p.N / BN);
   else return c.prefix[p.E] * (p.N / BN);
 }
 
@@ -288,12 +296,14 @@ __device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) 
   return av > bv || (av == bv && ai < bi);
 }
 
-template <typename T, int BN, int MODE>
+template <typename T, int BN, int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1, const Params p) {
-  using C = Cfg<T, BN>;
+  using C = Cfg<T, BN, CG>;
+  static_assert(CG == 1 || (sizeof(T) == 2 && MODE != ROUTER), "CTA pairs: bf16 grouped GEMMs only");
+  constexpr int BMP = C::BMP, BNC = C::BNC;
   using MT = ModeTraits<MODE>;
   // tf32 operands are only ever K-major: the fp32 forward reads pre-transposed weights
   constexpr bool FWD_B_KMAJOR = (sizeof(T) == 4) && (MODE == FWD_GU || MODE == FWD_DOWN);
@@ -306,17 +316,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   volatile int *abort_flag = &c.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // CTA pairs: rank 0 (the leader) issues the MMAs for both CTAs; tiles are dealt per pair
+  const int rank = CG == 2 ? (int)ptx::cluster_ctarank() : 0;
+  const int tile0 = CG == 2 ? (int)ptx::cluster_id_x() : (int)blockIdx.x;
+  const int tstep = CG == 2 ? (int)ptx::ncluster_x() : (int)gridDim.x;
 
   // ------------------------------------------------------------------ prologue
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       // MXFP8: a second arrival once the producer warp has written the stage's scales
+      // pairs: one arrival, the leader's arrive.expect_tx for both CTAs' bytes
       ptx::mbar_init(ptx::smem_u32(&c.full[s]), C::MX ? 2 : 1);
       ptx::mbar_init(ptx::smem_u32(&c.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
-      ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), 32 * EPI_WARPS);
+      ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), EPI_WARPS * CG);   // one arrival per epilogue warp
     }
     ptx::mbar_init(ptx::smem_u32(&c.tail), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
@@ -327,8 +342,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tma_prefetch(&tmB1);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
-    ptx::tmem_relinquish();
+    if constexpr (CG == 2) {
+      ptx::tmem_alloc_pair(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
+      ptx::tmem_relinquish_pair();
+    } else {
+      ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
+      ptx::tmem_relinquish();
+    }
   }
   if (warp == 2 && (!MT::WGRAD || C::MX) && MODE != ROUTER) {
     // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
@@ -337,7 +357,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int i = 0; i < 8; ++i) {
       int e = lane * 8 + i;
       int n = 0;
-      if (e < p.E) n = (p.offsets[e + 1] - p.offsets[e] + BM - 1) / BM;
+      if (e < p.E) n = (p.offsets[e + 1] - p.offsets[e] + BMP - 1) / BMP;
       cnt[i] = n;
       s += n;
     }
@@ -358,9 +378,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
   ptx::tc_fence_before();
   __syncthreads();
+  if constexpr (CG == 2) ptx::cluster_sync();   // the peer's barriers exist before anyone signals them
   ptx::tc_fence_after();
   const uint32_t tmem_base = c.tmem_base;
-  const int ntiles = total_tiles<MODE, BN>(p, c);
+  const int ntiles = total_tiles<MODE, BN, CG>(p, c);
 
   if (warp == 0) {
     // ================================================================ producer
@@ -369,9 +390,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t armed = 0, armed_par = 0;  // per stage: a fill is in flight / its parity
     bool tail_armed = false;
     bool ok = true;
-    for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x) {
+    for (int t = tile0; t < ntiles && ok; t += tstep) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
+      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
       for (int kb = 0; kb < tl.num_kb && ok; ++kb) {
         if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
         ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -381,17 +402,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         int valid = C::KBLK;
         if constexpr (MT::WGRAD && !C::MX) valid = min(C::KBLK, tl.rows - kb * C::KBLK);
         const bool tail = valid < C::KBLK;
-        const uint32_t bar = tail ? ptx::smem_u32(&c.tail) : ptx::smem_u32(&c.full[stage]);
+        const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
+        // pairs: the bytes of both CTAs' loads are counted on the leader's full barrier
+        const uint32_t full_leader = CG == 2 ? ptx::mapa(full_local, 0) : full_local;
+        const uint32_t bar = tail ? ptx::smem_u32(&c.tail) : full_local;
+        const bool pair_load = CG == 2 && !tail;
+        auto ld = [&](uint32_t dst, const CUtensorMap *tm, int x, int y) {
+          if (pair_load) ptx::tma_load_2d_pair(dst, tm, full_leader, x, y);
+          else ptx::tma_load_2d(dst, tm, bar, x, y);
+        };
         if (lane == 0) {
-          ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+          if (tail) ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+          else if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES);
           // ---- A
           if constexpr (MT::A_MN) {
 #pragma unroll
             for (int i = 0; i < BM / C::BOX_MN; ++i)
-              ptx::tma_load_2d(a_dst + i * C::BOX_BYTES, &tmA, bar, tl.m_blk * BM + i * C::BOX_MN,
-                               tl.row0 + kb * C::KBLK);
+              ld(a_dst + i * C::BOX_BYTES, &tmA, tl.mcol0 + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
           } else {
-            ptx::tma_load_2d(a_dst, &tmA, bar, kb * C::KBLK, tl.row0);
+            ld(a_dst, &tmA, kb * C::KBLK, tl.row0);
           }
           // ---- B
           if constexpr (C::MX && MODE == FWD_GU) {
@@ -408,6 +437,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else if constexpr (FWD_B_KMAJOR && MODE == FWD_DOWN) {
             // Wd^T [E*d][f]
             ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+          } else if constexpr (MODE == FWD_GU && CG == 2) {
+            // pair: the leader holds the gate half of B, the peer the up half
+            const int half = BN / 2;
+#pragma unroll
+            for (int i = 0; i < half / C::BOX_MN; ++i)
+              ld(b_dst + i * C::BOX_BYTES, rank == 0 ? &tmB0 : &tmB1, tl.n_blk * half + i * C::BOX_MN,
+                 tl.e * p.K + kb * C::KBLK);
           } else if constexpr (MODE == FWD_GU) {
             const int half = BN / 2;
 #pragma unroll
@@ -424,22 +460,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, i * C::BOX_MN, kb * C::KBLK);
           } else if constexpr (MODE == FWD_DOWN) {
 #pragma unroll
-            for (int i = 0; i < BN / C::BOX_MN; ++i)
-              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * BN + i * C::BOX_MN,
-                               tl.e * p.K + kb * C::KBLK);
+            for (int i = 0; i < BNC / C::BOX_MN; ++i)
+              ld(b_dst + i * C::BOX_BYTES, &tmB0, tl.n_blk * BN + rank * BNC + i * C::BOX_MN,
+                 tl.e * p.K + kb * C::KBLK);
           } else if constexpr (MODE == DGRAD_DOWN) {
-            ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.f + tl.n_blk * BN);
+            ld(b_dst, &tmB0, kb * C::KBLK, tl.e * p.f + tl.n_blk * BN + rank * BNC);
           } else if constexpr (MODE == DGRAD_GU) {
             const int kb_half = p.f / C::KBLK;
             if (kb < kb_half)
-              ptx::tma_load_2d(b_dst, &tmB0, bar, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+              ld(b_dst, &tmB0, kb * C::KBLK, tl.e * p.d + tl.n_blk * BN + rank * BNC);
             else
-              ptx::tma_load_2d(b_dst, &tmB1, bar, (kb - kb_half) * C::KBLK, tl.e * p.d + tl.n_blk * BN);
+              ld(b_dst, &tmB1, (kb - kb_half) * C::KBLK, tl.e * p.d + tl.n_blk * BN + rank * BNC);
           } else {  // weight gradients: B is the MN-major activation gradient
 #pragma unroll
-            for (int i = 0; i < BN / C::BOX_MN; ++i)
-              ptx::tma_load_2d(b_dst + i * C::BOX_BYTES, &tmB0, bar, tl.n_blk * BN + i * C::BOX_MN,
-                               tl.row0 + kb * C::KBLK);
+            for (int i = 0; i < BNC / C::BOX_MN; ++i)
+              ld(b_dst + i * C::BOX_BYTES, &tmB0, tl.n_blk * BN + rank * BNC + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
           }
         }
         if constexpr (C::MX) {
@@ -477,7 +512,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tail_phase ^= 1;
           // In an MN-major box each K row is one 128-byte line: rows [valid, KBLK) are the
           // byte range [valid*128, KBLK*128) of every box.
-          const int nbox_a = BM / C::BOX_MN, nbox_b = BN / C::BOX_MN;
+          const int nbox_a = BM / C::BOX_MN, nbox_b = BNC / C::BOX_MN;
           const int line0 = valid * 8, lines = C::KBLK * 8;  // in 16-byte units
           uint4 z = make_uint4(0, 0, 0, 0);
           for (int b = 0; b < nbox_a + nbox_b; ++b) {
@@ -487,7 +522,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           ptx::fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
+          if (lane == 0) {
+            if constexpr (CG == 2) {
+              // the leader arrives expecting the peer's bytes; the peer posts them once its
+              // zeroed stage is visible (the tensor cores of the pair read it)
+              if (rank == 0) {
+                ptx::mbar_arrive_expect_tx(full_local, C::STAGE_BYTES);
+              } else {
+                ptx::fence_acq_rel_cluster();
+                ptx::mbar_complete_tx_cluster(full_leader, C::STAGE_BYTES);
+              }
+            } else {
+              ptx::mbar_arrive(full_local);
+            }
+          }
         }
         // this stage's full barrier completes (or has completed) the phase of this pass
         armed |= 1u << stage;
@@ -495,10 +543,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
-    // Drain: every TMA fill this warp issued must land before the CTA may exit.
+    // Drain: every TMA fill this warp issued must land before the CTA may exit.  (Pairs:
+    // the leader's full barriers count the peer's bytes too; the peer only has tails.)
     if (lane == 0) {
       for (int s = 0; s < C::STAGES; ++s)
-        if ((armed >> s) & 1u)
+        if (rank == 0 && ((armed >> s) & 1u))
           if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
             note_fail(p, 0, 0, s, 2);
       if (tail_armed && !ptx::mbar_wait(ptx::smem_u32(&c.tail), tail_phase, abort_flag, WAIT_LIMIT_NS))
@@ -506,10 +555,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && rank == 0) {
       constexpr uint32_t idesc = (1u << 4) | (ElemTraits<T>::FMT << 7) | (ElemTraits<T>::FMT << 10) |
                                  ((MT::A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
-                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+                                 ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BMP >> 4) << 24);
       // block-scaled E4M3 x E4M3 (formats 0), UE8M0 scales (bit 23); per-MMA scale-byte ids
       // go in bits 5:4 (B) and 30:29 (A)
       constexpr uint32_t idesc_mx = ((MT::A_MN ? 1u : 0u) << 15) | ((B_MN ? 1u : 0u) << 16) |
@@ -518,9 +567,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < ntiles && ok; t += gridDim.x, ++it) {
+      for (int t = tile0; t < ntiles && ok; t += tstep, ++it) {
         Tile tl;
-        get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
+        get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         ok = ptx::mbar_wait(ptx::smem_u32(&c.tempty[acc]), aph ^ 1, abort_flag, WAIT_LIMIT_NS);
@@ -529,10 +578,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + acc * BN;
         if (tl.num_kb == 0) {
           ptx::mbar_arrive(ptx::smem_u32(&c.tfull[acc]));
+          if constexpr (CG == 2) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&c.tfull[acc]), 1));
           continue;
         }
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          ok = ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
+          // Loaded bytes and commit arrivals are ordered by the barrier itself.  A weight-gradient
+          // tail stage was also zeroed by the peer's ordinary stores: that one wait takes a
+          // cluster-scope acquire, to see them before the pair MMA reads the peer's stage.
+          const bool peer_stores = CG == 2 && MT::WGRAD && kb == tl.num_kb - 1 && (tl.rows % C::KBLK) != 0;
+          ok = peer_stores ? ptx::mbar_wait_cluster(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS)
+                           : ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
           if (!ok) { note_fail(p, 1, t, kb, 1); break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
@@ -561,17 +616,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if constexpr (C::MX)
               ptx::mma_mxf8(d_tmem, adesc, bdesc, idesc_mx | ((uint32_t)kk << 4) | ((uint32_t)kk << 29),
                             sfa_t | ((uint32_t)kk << 30), sfb_t | ((uint32_t)kk << 30), accum);
+            else if constexpr (CG == 2) ptx::mma_f16_pair(d_tmem, adesc, bdesc, idesc, accum);
             else if constexpr (sizeof(T) == 2) ptx::mma_f16(d_tmem, adesc, bdesc, idesc, accum);
             else ptx::mma_tf32(d_tmem, adesc, bdesc, idesc, accum);
           }
-          ptx::tc_commit(ptx::smem_u32(&c.empty[stage]));
+          if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.empty[stage]), 0x3);
+          else ptx::tc_commit(ptx::smem_u32(&c.empty[stage]));
           if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        ptx::tc_commit(ptx::smem_u32(&c.tfull[acc]));
+        if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.tfull[acc]), 0x3);
+        else ptx::tc_commit(ptx::smem_u32(&c.tfull[acc]));
       }
       // Drain: all MMAs issued here complete before TMEM is freed.
-      ptx::tc_commit(ptx::smem_u32(&c.drain));
+      if constexpr (CG == 2) ptx::tc_commit_pair(ptx::smem_u32(&c.drain));
+      else ptx::tc_commit(ptx::smem_u32(&c.drain));
       if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, abort_flag, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
     }
     __syncwarp();
@@ -584,9 +643,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - 2) >> 2;     // 0 or 1
     const int r = q * 32 + lane;          // tile row owned by this thread
     int it = 0;
-    for (int t = blockIdx.x; t < ntiles; t += gridDim.x, ++it) {
+    for (int t = tile0; t < ntiles; t += tstep, ++it) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK, C::MX>(t, p, c, tl);
+      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       bool ok = ptx::mbar_wait(ptx::smem_u32(&c.tfull[acc]), aph, abort_flag, WAIT_LIMIT_NS);
@@ -608,6 +667,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           int ti[MAX_K];
 #pragma unroll
           for (int j = 0; j < MAX_K; ++j) { tv[j] = 0.f; ti[j] = INT_MAX; }
+          float kth_v = 0.f;      // the k-th best so far (an empty slot until k are seen)
+          int kth_i = INT_MAX;
           bool nan_seen = false;
 #pragma unroll 1
           for (int c0 = 0; c0 < p.E; c0 += 32) {
@@ -621,14 +682,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   float z = v[i] + (bias ? __ldg(bias + e) : 0.f);
                   v[i] = z;
                   nan_seen |= (z != z);
-                  float cv = z;
-                  int ci = e;
+                  // one comparison against the current k-th best rejects most logits; the
+                  // insertion network runs only for the few that enter the top k
+                  if (topk_better(z, e, kth_v, kth_i)) {
+                    float cv = z;
+                    int ci = e;
 #pragma unroll
-                  for (int j = 0; j < MAX_K; ++j) {
-                    bool take = j < p.k && topk_better(cv, ci, tv[j], ti[j]);
-                    float sv = tv[j];
-                    int si = ti[j];
-                    if (take) { tv[j] = cv; ti[j] = ci; cv = sv; ci = si; }
+                    for (int j = 0; j < MAX_K; ++j) {
+                      bool take = j < p.k && topk_better(cv, ci, tv[j], ti[j]);
+                      float sv = tv[j];
+                      int si = ti[j];
+                      if (take) { tv[j] = cv; ti[j] = ci; cv = sv; ci = si; }
+                      if (j == p.k - 1) { kth_v = tv[j]; kth_i = ti[j]; }
+                    }
                   }
                 }
               }
@@ -735,7 +801,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
         }
       } else {  // weight gradients: slab of rows q*32.. of the [M x N] block of expert e
-        const int64_t srow = (int64_t)tl.e * p.M + (int64_t)tl.m_blk * BM + q * 32;
+        const int64_t srow = (int64_t)tl.e * p.M + tl.mcol0 + q * 32;
 #pragma unroll 1
         for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
           float v[32];
@@ -756,18 +822,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
+      // release the accumulator: one arrival per warp on the leader's barrier
       ptx::tc_fence_before();
-      ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+      __syncwarp();
+      if (lane == 0) {
+        if (CG == 2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&c.tempty[acc]), 0));
+        else ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+      }
     }
   }
 
   // ------------------------------------------------------------------ teardown
   ptx::tc_fence_before();
   __syncthreads();
+  // pairs: the leader's MMAs read the peer's shared memory and write its TMEM; neither CTA
+  // leaves or frees TMEM before both are done (every wait above is bounded, so both get here)
+  if constexpr (CG == 2) ptx::cluster_sync();
   if (threadIdx.x == 0 && c.abort) set_error(p.err, MOE_ERR_DEVICE_TIMEOUT);
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if constexpr (CG == 2) ptx::tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else ptx::tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
 }
 
@@ -813,21 +888,57 @@ static int sm_count() {
   return n;
 }
 
-template <typename T, int BN, int MODE>
+// Persistent launch: one CTA per SM (CG = 1), or one CTA pair per two SMs in clusters
+// of two (CG = 2); never more CTAs (pairs) than tiles.
+template <typename T, int BN, int MODE, int CG = 1>
 static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p,
                   int64_t max_tiles, cudaStream_t st) {
-  using C = Cfg<T, BN>;
-  auto kern = grouped_gemm_kernel<T, BN, MODE>;
+  using C = Cfg<T, BN, CG>;
+  auto kern = grouped_gemm_kernel<T, BN, MODE, CG>;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
       return MOE_ERR_CUDA;
     attr_set = true;
   }
-  int64_t grid = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
-  kern<<<(unsigned)grid, NUM_THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, p);
+  if constexpr (CG == 1) {
+    const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
+    kern<<<(unsigned)units, NUM_THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(NUM_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CG;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // A persistent grid must be fully resident: pairs of SMs are taken inside one GPC, so
+    // fewer than sm_count/2 pairs may fit at once (a late pair would run after a whole
+    // persistent pair has finished).  Ask the occupancy calculator, once.
+    static int max_pairs = 0;
+    if (!max_pairs) {
+      cfg.gridDim = dim3((unsigned)(sm_count() / CG * CG));
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = sm_count() / CG;
+      max_pairs = std::min(n, sm_count() / CG);
+    }
+    const int64_t units = std::min<int64_t>(max_pairs, std::max<int64_t>(max_tiles, 1));
+    cfg.gridDim = dim3((unsigned)(units * CG));
+    if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p) != cudaSuccess) return MOE_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
+
+// Row-grouped GEMMs use 256-row CTA-pair tiles only when experts hold many rows: the
+// last tile of each expert is on average half empty, which small groups cannot afford.
+#ifndef MOE_PAIR_MIN_ROWS_PER_EXPERT
+#define MOE_PAIR_MIN_ROWS_PER_EXPERT 768
+#endif
+static bool pair_rows(const Shape &s) { return s.P() >= MOE_PAIR_MIN_ROWS_PER_EXPERT * (int64_t)s.E; }
 
 template <typename T>
 static int fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
@@ -865,7 +976,10 @@ static int fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, 
       if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     }
     p.K = s.d; p.N = 2 * s.f; p.out0 = hu; p.out1 = a; p.aux = nullptr;
-    int rc = launch<T, BN, FWD_GU>(tA, tB0, tB1, p, mblocks * (p.N / BN), st);
+    int rc = -1;
+    if constexpr (sizeof(T) == 2)
+      if (pair_rows(s)) rc = launch<T, BN, FWD_GU, 2>(tA, tB0, tB1, p, ((P + 255) / 256 + s.E) * (p.N / BN), st);
+    if (rc < 0) rc = launch<T, BN, FWD_GU>(tA, tB0, tB1, p, mblocks * (p.N / BN), st);
     if (rc) return rc;
   }
   // GEMM 2: y_perm = a [P,f] x Wd [f,d]
@@ -880,7 +994,12 @@ static int fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, 
     else
       ok = make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, BOX_MN, KBLK);
     if (!ok) return MOE_ERR_CUDA;
-    if (bn == 256)
+    rc = -1;
+    if constexpr (sizeof(T) == 2)
+      if (bn == 256 && pair_rows(s))
+        rc = launch<T, 256, FWD_DOWN, 2>(tA, tB0, tB0, p, ((P + 255) / 256 + s.E) * (p.N / 256), st);
+    if (rc >= 0) {
+    } else if (bn == 256)
       rc = launch<T, 256, FWD_DOWN>(tA, tB0, tB0, p, mblocks * (p.N / 256), st);
     else
       rc = launch<T, 128, FWD_DOWN>(tA, tB0, tB0, p, mblocks * (p.N / 128), st);
@@ -906,7 +1025,11 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   {
     if (!make_tmap(&tA, dy_perm, ES, s.d, P, KBLK, BM)) return MOE_ERR_CUDA;
     p.K = s.d; p.N = s.f; p.out0 = dhu; p.aux = hu;
-    if (s.f % 256 == 0) {
+    const int64_t pblocks = (P + 255) / 256 + s.E;
+    if (s.f % 256 == 0 && pair_rows(s)) {
+      if (!make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, KBLK, 128)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, DGRAD_DOWN, 2>(tA, tB0, tB0, p, pblocks * (s.f / 256), st);
+    } else if (s.f % 256 == 0) {
       if (!make_tmap(&tB0, w_down, ES, s.d, (uint64_t)s.E * s.f, KBLK, 256)) return MOE_ERR_CUDA;
       rc = launch<T, 256, DGRAD_DOWN>(tA, tB0, tB0, p, mblocks * (s.f / 256), st);
     } else {
@@ -919,7 +1042,11 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   {
     if (!make_tmap(&tA, a, ES, s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
-    if (s.d % 256 == 0) {
+    if (s.d % 256 == 0 && s.f % 256 == 0) {
+      // weight-gradient tiles are 256 weight rows (no empty rows): always CTA pairs
+      if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, WGRAD_DOWN, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / 256) * (s.d / 256), st);
+    } else if (s.d % 256 == 0) {
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
       rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st);
     } else {
@@ -932,7 +1059,11 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   {
     if (!make_tmap(&tA, dhu, ES, 2 * s.f, P, KBLK, BM)) return MOE_ERR_CUDA;
     p.K = 2 * s.f; p.N = s.d; p.out0 = dx_perm;
-    if (s.d % 256 == 0) {
+    if (s.d % 256 == 0 && pair_rows(s)) {
+      if (!make_tmap(&tB0, w_gate, ES, s.f, (uint64_t)s.E * s.d, KBLK, 128)) return MOE_ERR_CUDA;
+      if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, KBLK, 128)) return MOE_ERR_CUDA;
+      rc = launch<T, 256, DGRAD_GU, 2>(tA, tB0, tB1, p, ((P + 255) / 256 + s.E) * (s.d / 256), st);
+    } else if (s.d % 256 == 0) {
       if (!make_tmap(&tB0, w_gate, ES, s.f, (uint64_t)s.E * s.d, KBLK, 256)) return MOE_ERR_CUDA;
       if (!make_tmap(&tB1, w_up, ES, s.f, (uint64_t)s.E * s.d, KBLK, 256)) return MOE_ERR_CUDA;
       rc = launch<T, 256, DGRAD_GU>(tA, tB0, tB1, p, mblocks * (s.d / 256), st);
@@ -948,7 +1079,9 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
     if (!make_tmap(&tA, x_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     if (!make_tmap(&tB0, dhu, ES, 2 * s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
-    if (s.f % 256 == 0)
+    if (s.f % 256 == 0 && s.d % 256 == 0)
+      rc = launch<T, 256, WGRAD_GU, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / 256) * (2 * s.f / 256), st);
+    else if (s.f % 256 == 0)
       rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st);
     else
       rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st);

@@ -231,10 +231,18 @@ GEMM_CASES = [
     ("bf16", 256, 512, 1, "tiny"),
     ("f32", 128, 256, 8, "random"),
     ("bf16", 2048, 1024, 8, "random"),
+    # large groups: 256-row CTA-pair tiles for the row-grouped GEMMs (P >= 768 E), with an
+    # empty expert and tails that leave the second CTA of a pair without rows
+    ("bf16", 256, 256, 3, "big"),
+    ("bf16", 512, 512, 2, "big2"),
 ]
 
 
 def _counts(kind, E, rng):
+    if kind == "big":
+        return np.array([1000, 0, 1400], np.int64)
+    if kind == "big2":
+        return np.array([1537, 129], np.int64)
     if kind == "random":
         return random_counts(E, 300, rng)
     if kind == "one_expert":
