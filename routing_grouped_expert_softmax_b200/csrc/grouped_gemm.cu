@@ -135,10 +135,19 @@ struct Ctrl {
   uint64_t tempty[2];
   uint64_t tail;
   uint64_t drain;
+  uint64_t xfull[4];      // router: one lane quarter's second-half picks are in xbuf
+  uint64_t xempty[4];     // router: ... and have been merged
   uint32_t tmem_base;
   int abort;
-  int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
+  union {
+    int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
+    float bias[MAX_E];      // router: the logit bias (0 past E)
+  };
 };
+constexpr int CTRL_BYTES = 2048;
+static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
+// Router: shared buffer for the second-half picks, [MAX_K][BM] keys then [MAX_K][BM] experts
+constexpr int ROUTER_XBYTES = 2 * MAX_K * BM * 4;
 
 template <int MODE, int BN, int KBLK, bool MX, int CG = 1>
 __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl, int rank = 0) {
@@ -285,15 +294,21 @@ __device__ __forceinline__ void sf_gather_mnmajor(const uint8_t *sf, int64_t kbl
   *reinterpret_cast<uint4 *>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// Router order: numbers before NaN, larger first, then the lower expert index; an empty
-// slot (index INT_MAX) loses to everything.
-__device__ __forceinline__ bool topk_better(float av, int ai, float bv, int bi) {
-  if (ai == INT_MAX) return false;
-  if (bi == INT_MAX) return true;
-  const bool an = av != av, bn = bv != bv;
-  if (an != bn) return bn;
-  if (an) return ai < bi;
-  return av > bv || (av == bv && ai < bi);
+// Router order key: an unsigned 32-bit number that grows with the logit (-0 counts as +0),
+// 1 for NaN (below every number) and 0 for "no expert".  Among equal keys the lower expert
+// index ranks first.
+__device__ __forceinline__ uint32_t router_key(float z) {
+  if (z != z) return 1u;
+  const uint32_t b = __float_as_uint(z == 0.f ? 0.f : z);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float router_key_value(uint32_t o) {
+  if (o <= 1u) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+// (o, e) ranks above (p, f): the larger key, then the lower expert
+__device__ __forceinline__ bool key_above(uint32_t o, int e, uint32_t po, int pe) {
+  return o > po || (o == po && e < pe);
 }
 
 template <typename T, int BN, int MODE, int CG>
@@ -313,6 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *ring = smem;                                   // STAGES x (A | B)
   uint8_t *sf_ring = smem + C::STAGES * C::STAGE_BYTES;   // MXFP8: STAGES x (SFA | SFB)
   Ctrl &c = *reinterpret_cast<Ctrl *>(smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES));
+  uint32_t *xbuf = reinterpret_cast<uint32_t *>(smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES) + CTRL_BYTES);
   volatile int *abort_flag = &c.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -335,6 +351,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     ptx::mbar_init(ptx::smem_u32(&c.tail), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
+    for (int q = 0; q < 4; ++q) {
+      ptx::mbar_init(ptx::smem_u32(&c.xfull[q]), 32);
+      ptx::mbar_init(ptx::smem_u32(&c.xempty[q]), 32);
+    }
     c.abort = 0;
     ptx::fence_mbar_init();
     ptx::tma_prefetch(&tmA);
@@ -348,6 +368,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     } else {
       ptx::tmem_alloc(ptx::smem_u32(&c.tmem_base), C::TMEM_COLS);
       ptx::tmem_relinquish();
+    }
+  }
+  if constexpr (MODE == ROUTER) {
+    if (warp >= 2) {
+      const float *bias = static_cast<const float *>(p.aux);
+      for (int e = threadIdx.x - 64; e < MAX_E; e += 32 * EPI_WARPS) c.bias[e] = (bias && e < p.E) ? bias[e] : 0.f;
     }
   }
   if (warp == 2 && (!MT::WGRAD || C::MX) && MODE != ROUTER) {
@@ -654,74 +680,174 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + acc * BN;
 
       if constexpr (MODE == ROUTER) {
-        // One token per thread: z = x W_r (+ b) for all E experts, then top-k by an
-        // insertion network over the logits in expert order (a later equal logit never
-        // displaces an earlier one: ties go to the lower index), then the softmax of the
-        // k selected logits.  The first warp of each lane quarter does the work.
-        if (half == 0) {
-          const bool valid = r < tl.rows;
-          const int64_t row = (int64_t)tl.orow0 + r;
-          const float *bias = static_cast<const float *>(p.aux);
-          float *logits = static_cast<float *>(p.out2);
-          float tv[MAX_K];
-          int ti[MAX_K];
+        // One token per tile row.  The two warps of a lane quarter split the experts in
+        // halves and each takes the k best of its half by k max passes over the order keys
+        // (a pass keeps the first of equal keys, so ties go to the lower expert, and drops the
+        // previous pass's pick); the first warp then merges the second warp's picks into its
+        // own through shared memory and writes the gates, the softmax of the k logits.
+        constexpr int HC = BN / 2;
+        const int cb = half * HC;                         // first expert of this half
+        const int ncol = min(HC, max(0, p.E - cb));
+        const bool two = p.E > HC;                        // the second half holds experts
+        const bool valid = r < tl.rows;
+        const int64_t row = (int64_t)tl.orow0 + r;
+        float *logits = static_cast<float *>(p.out2);
+        bool nan_seen = false;
+        uint32_t pk[MAX_K];
+        int pe[MAX_K];
+        if (ncol > 0) {
+          auto load = [&](int cc, float (&v)[32]) {
+            ptx::tmem_ld32(taddr + cb + cc, v);
 #pragma unroll
-          for (int j = 0; j < MAX_K; ++j) { tv[j] = 0.f; ti[j] = INT_MAX; }
-          float kth_v = 0.f;      // the k-th best so far (an empty slot until k are seen)
-          int kth_i = INT_MAX;
-          bool nan_seen = false;
+            for (int i = 0; i < 32; ++i) v[i] += c.bias[cb + cc + i];
+          };
+          auto put_logits = [&](int cc, const float (&v)[32]) {
+            if (!valid || !logits) return;
+            float *dst = logits + row * p.E + cb + cc;
+            if (cb + cc + 32 <= p.E) {
+              store32(dst, v);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i)
+                if (cb + cc + i < p.E) dst[i] = v[i];
+            }
+          };
+          if constexpr (HC <= 64) {
+            // keys of the whole half stay in registers
+            uint32_t o[HC];
+#pragma unroll
+            for (int cc = 0; cc < HC; cc += 32) {
+              if (cc < ncol) {
+                float v[32];
+                load(cc, v);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                  o[cc + i] = cc + i < ncol ? router_key(v[i]) : 0u;
+                  nan_seen |= o[cc + i] == 1u;
+                }
+                put_logits(cc, v);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) o[cc + i] = 0u;
+              }
+            }
+            int prev = -1;
+#pragma unroll
+            for (int j = 0; j < MAX_K; ++j) {
+              pk[j] = 0u;
+              pe[j] = INT_MAX;
+              if (j < p.k) {
+                uint32_t bo[4] = {0u, 0u, 0u, 0u};
+                int bi[4] = {0, 0, 0, 0};
+#pragma unroll
+                for (int i = 0; i < HC; ++i) {
+                  if (i == prev) o[i] = 0u;
+                  if (o[i] > bo[i & 3]) { bo[i & 3] = o[i]; bi[i & 3] = i; }
+                }
+                uint32_t best = bo[0];
+                int bc = bi[0];
+#pragma unroll
+                for (int a = 1; a < 4; ++a)
+                  if (key_above(bo[a], bi[a], best, bc)) { best = bo[a]; bc = bi[a]; }
+                prev = best ? bc : -1;
+                pk[j] = best;
+                pe[j] = best ? cb + bc : INT_MAX;
+              }
+            }
+          } else {
+            // wide halves: every pass reads the accumulator again and keeps the best key
+            // that ranks below the previous pick
 #pragma unroll 1
-          for (int c0 = 0; c0 < p.E; c0 += 32) {
-            float v[32];
-            ptx::tmem_ld32(taddr + c0, v);
-            if (valid) {
+            for (int cc = 0; cc < ncol; cc += 32) {
+              float v[32];
+              load(cc, v);
 #pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const int e = c0 + i;
-                if (e < p.E) {
-                  float z = v[i] + (bias ? __ldg(bias + e) : 0.f);
-                  v[i] = z;
-                  nan_seen |= (z != z);
-                  // one comparison against the current k-th best rejects most logits; the
-                  // insertion network runs only for the few that enter the top k
-                  if (topk_better(z, e, kth_v, kth_i)) {
-                    float cv = z;
-                    int ci = e;
+              for (int i = 0; i < 32; ++i) nan_seen |= (cc + i < ncol) && (v[i] != v[i]);
+              put_logits(cc, v);
+            }
+            uint32_t po = 0xffffffffu;
+            int pc = -1;
 #pragma unroll
-                    for (int j = 0; j < MAX_K; ++j) {
-                      bool take = j < p.k && topk_better(cv, ci, tv[j], ti[j]);
-                      float sv = tv[j];
-                      int si = ti[j];
-                      if (take) { tv[j] = cv; ti[j] = ci; cv = sv; ci = si; }
-                      if (j == p.k - 1) { kth_v = tv[j]; kth_i = ti[j]; }
+            for (int j = 0; j < MAX_K; ++j) {
+              pk[j] = 0u;
+              pe[j] = INT_MAX;
+              if (j < p.k) {
+                uint32_t bo[4] = {0u, 0u, 0u, 0u};
+                int bi[4] = {0, 0, 0, 0};
+#pragma unroll 1
+                for (int cc = 0; cc < ncol; cc += 32) {
+                  float v[32];
+                  load(cc, v);
+#pragma unroll
+                  for (int i = 0; i < 32; ++i) {
+                    const int col = cc + i;
+                    uint32_t o = col < ncol ? router_key(v[i]) : 0u;
+                    if (!(o < po || (o == po && col > pc))) o = 0u;
+                    if (o > bo[i & 3]) { bo[i & 3] = o; bi[i & 3] = col; }
+                  }
+                }
+                uint32_t best = bo[0];
+                int bc = bi[0];
+#pragma unroll
+                for (int a = 1; a < 4; ++a)
+                  if (key_above(bo[a], bi[a], best, bc)) { best = bo[a]; bc = bi[a]; }
+                po = best ? best : 0u;
+                pc = best ? bc : HC;
+                pk[j] = best;
+                pe[j] = best ? cb + bc : INT_MAX;
+              }
+            }
+          }
+        }
+        if (valid && nan_seen) set_error(p.err, MOE_ERR_DEVICE_NAN);
+        if (two) {
+          uint32_t *xk = xbuf;
+          int *xe = reinterpret_cast<int *>(xbuf + MAX_K * BM);
+          if (half == 1) {
+            if (it > 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.xempty[q]), (it - 1) & 1, abort_flag, WAIT_LIMIT_NS);
+            if (ok) {
+#pragma unroll
+              for (int j = 0; j < MAX_K; ++j)
+                if (j < p.k) { xk[j * BM + r] = pk[j]; xe[j * BM + r] = pe[j]; }
+              ptx::mbar_arrive(ptx::smem_u32(&c.xfull[q]));
+            }
+          } else {
+            ok = ptx::mbar_wait(ptx::smem_u32(&c.xfull[q]), it & 1, abort_flag, WAIT_LIMIT_NS);
+            if (ok) {
+#pragma unroll
+              for (int m = 0; m < MAX_K; ++m) {
+                if (m < p.k) {
+                  uint32_t xo = xk[m * BM + r];
+                  int xi = xe[m * BM + r];
+#pragma unroll
+                  for (int j = 0; j < MAX_K; ++j) {
+                    if (j < p.k && key_above(xo, xi, pk[j], pe[j])) {
+                      const uint32_t so = pk[j];
+                      const int si = pe[j];
+                      pk[j] = xo; pe[j] = xi; xo = so; xi = si;
                     }
                   }
                 }
               }
-              if (logits) {
-                if (c0 + 32 <= p.E) {
-                  store32(logits + row * p.E + c0, v);
-                } else {
-#pragma unroll
-                  for (int i = 0; i < 32; ++i)
-                    if (c0 + i < p.E) logits[row * p.E + c0 + i] = v[i];
-                }
-              }
+              ptx::mbar_arrive(ptx::smem_u32(&c.xempty[q]));
             }
           }
-          if (valid) {
-            if (nan_seen) set_error(p.err, MOE_ERR_DEVICE_NAN);
-            int32_t *idx = static_cast<int32_t *>(p.out0);
-            float *gate = static_cast<float *>(p.out1);
-            float ex[MAX_K], sum = 0.f;
+          if (!__all_sync(0xffffffffu, ok)) { if (lane == 0) note_fail(p, 2, t, 0, 3); break; }
+        }
+        if (half == 0 && valid) {
+          int32_t *idx = static_cast<int32_t *>(p.out0);
+          float *gate = static_cast<float *>(p.out1);
+          float ex[MAX_K], sum = 0.f;
+          const float z0 = router_key_value(pk[0]);
 #pragma unroll
-            for (int j = 0; j < MAX_K; ++j)
-              if (j < p.k) { ex[j] = expf(tv[j] - tv[0]); sum += ex[j]; }
-            const float inv = 1.0f / sum;
-#pragma unroll
-            for (int j = 0; j < MAX_K; ++j)
-              if (j < p.k) { idx[row * p.k + j] = ti[j]; gate[row * p.k + j] = ex[j] * inv; }
+          for (int j = 0; j < MAX_K; ++j) {
+            ex[j] = 0.f;
+            if (j < p.k) { ex[j] = expf(router_key_value(pk[j]) - z0); sum += ex[j]; }
           }
+          const float inv = 1.0f / sum;
+#pragma unroll
+          for (int j = 0; j < MAX_K; ++j)
+            if (j < p.k) { idx[row * p.k + j] = pe[j]; gate[row * p.k + j] = ex[j] * inv; }
         }
       } else if constexpr (MODE == FWD_GU) {
         // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
@@ -895,19 +1021,21 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
                   int64_t max_tiles, cudaStream_t st) {
   using C = Cfg<T, BN, CG>;
   auto kern = grouped_gemm_kernel<T, BN, MODE, CG>;
+  constexpr int SMEM = C::SMEM_BYTES + (MODE == ROUTER ? ROUTER_XBYTES : 0);
+  static_assert(SMEM <= 227 * 1024, "shared memory");
   static bool attr_set = false;
   if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
       return MOE_ERR_CUDA;
     attr_set = true;
   }
   if constexpr (CG == 1) {
     const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
-    kern<<<(unsigned)units, NUM_THREADS, C::SMEM_BYTES, st>>>(a, b0, b1, p);
+    kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, p);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(NUM_THREADS);
-    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.dynamicSmemBytes = SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;

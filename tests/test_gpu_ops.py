@@ -98,6 +98,49 @@ def test_route_topk(T, d, E, k, dtype, bias):
     _check_no_device_error(ws)
 
 
+@pytest.mark.parametrize("T,d,E,k,bias,nan_rows", [
+    (1000, 256, 64, 4, True, 0),
+    (333, 384, 128, 4, False, 3),
+    (129, 128, 256, 8, True, 2),
+    (700, 128, 8, 8, False, 0),        # k = E: every expert, in order
+    (515, 256, 16, 8, True, 1),
+    (300, 128, 192, 6, False, 0),      # the second half of a 256-column tile is ragged
+    (2000, 512, 128, 1, False, 0),
+    (300, 128, 36, 4, False, 2),       # the CUDA-core router
+])
+def test_route_topk_selects_exactly_on_its_own_logits(T, d, E, k, bias, nan_rows):
+    """Given the fp32 logits the router wrote, the selection is unique: on every row the
+    experts must be the oracle's top k of those logits (larger first, the lower index on
+    equal logits, NaN below every number) and the gates their renormalised softmax.  Each
+    router column is used by three experts, so exact ties are common."""
+    import torch
+    inp = gen.make_layer_inputs(T, d, E, k, 128, seed=23, skew=bias, with_grad=False)
+    w = np.ascontiguousarray(inp.w_r[:, np.arange(E) // 3])
+    x = inp.x.copy()
+    bad = (np.arange(nan_rows) * 97) % T
+    x[bad, 5] = np.nan
+    cfg = moe.config(T, d, E, k, 128)
+    ws = _ws(cfg)
+    logits = torch.empty(T, E, dtype=torch.float32, device="cuda")
+    idx = torch.empty(T, k, dtype=torch.int32, device="cuda")
+    g = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    b = dev_f32(inp.bias) if bias else None
+    moe.moe_route_topk(cfg, dev(x, "bf16"), dev(w, "bf16"), b, logits, idx, g, ws)
+    zg = host(logits)
+    gi = host(idx)
+    assert np.array_equal(gi, ref.topk_experts(zg, k))
+    if not bias and E >= 3:
+        # exact ties decided the selection on many rows
+        zs = np.take_along_axis(zg, gi.astype(np.int64), axis=1)
+        assert np.mean(np.any(zs[:, :-1] == zs[:, 1:], axis=1) if k > 1 else zs[:, 0] == zg.max(1)) > 0.5
+    fine = ~np.isnan(zg).any(axis=1)
+    assert fine.sum() == T - nan_rows
+    rg = ref.renormalised_gates(ref.softmax(zg[fine]), gi[fine])
+    assert np.max(np.abs(host(g)[fine] - rg)) <= 1e-6
+    code = moe.moe_get_error(ws)
+    assert code == (moe.MOE_ERR_DEVICE_NAN if nan_rows else 0)
+
+
 @pytest.mark.parametrize("T,E,k,kind", [
     (1, 1, 1, "uniform"), (3000, 8, 4, "uniform"), (777, 128, 4, "skewed"), (2048, 256, 8, "skewed"),
     (500, 16, 2, "one_expert"), (4097, 128, 4, "uniform"), (16384, 128, 4, "skewed"),
