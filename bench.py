@@ -34,6 +34,8 @@ WORKLOADS = {
     "e128_t16k_uniform_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "uniform"),
     # a smaller case of the same kernels for profiler captures (still larger than L2)
     "profile_e32_t4k": (4096, 2048, 32, 4, 1024, False, "router"),
+    # 256 rows per expert, as at T=8192, E=128, k=4
+    "profile_e32_t2k": (2048, 2048, 32, 4, 1024, False, "router"),
     # the same shapes with every grouped-GEMM operand in MXFP8 (E4M3 + E8M0 per 32)
     "e128_t16k_mxfp8_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "router", "mxfp8"),
     "e128_mxfp8_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "mxfp8"),

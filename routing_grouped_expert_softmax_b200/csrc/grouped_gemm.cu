@@ -8,7 +8,7 @@
 // стек обучения MoE от Ai2 ...", section "Три числа, три знаменателя" (the gains sit in
 // the feed-forward compute).
 //
-// One persistent kernel, one CTA per SM, 10 warps:
+// One persistent kernel, one CTA per SM, 11 warps:
 //   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) K-blocks in shared
 //               memory (128-byte swizzle), one mbarrier per stage;
 //   warp 1      allocates TMEM; its lane 0 issues tcgen05.mma (128 x BN x 16 per
@@ -17,7 +17,10 @@
 //   warps 2..9  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes
 //               32*(w%4)..+31, i.e. one row per thread; two warps per lane quarter split
 //               the columns), apply the fused elementwise step and store to global
-//               memory, then release the accumulator.
+//               memory (weight gradients: through shared memory and TMA stores), then
+//               release the accumulator;
+//   warp 10     weight gradients: zeroes the K rows of an expert's last stage that lie
+//               past the expert's end, then releases that stage to the MMA issuer.
 // The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered accumulator).
 //
 // Tile schedule.  Row-grouped GEMMs (forward and data-gradient) tile every expert's row
@@ -26,6 +29,7 @@
 // Rows of a block that belong to the next expert are computed and not stored.
 // Weight-gradient GEMMs reduce over one expert's rows; the last K-block of an expert
 // is zero-filled in shared memory past the expert's end before the MMA reads it.
+// CTA pairs (cta_group::2): a 256-row tile whose MMAs the even CTA issues for both.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -39,7 +43,8 @@ enum Mode { FWD_GU = 0, FWD_DOWN = 1, DGRAD_DOWN = 2, DGRAD_GU = 3, WGRAD_DOWN =
 
 constexpr int BM = 128;
 constexpr int EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * EPI_WARPS;  // producer warp, MMA warp, epilogue warps
+constexpr int FIX_WARP = 2 + EPI_WARPS;           // weight gradients: zeroes K rows past an expert
+constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);  // producer, MMA issuer, epilogue warps, tail fixer
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any tile's time
 
 template <int MODE> struct ModeTraits {
@@ -71,9 +76,13 @@ template <> struct ElemTraits<e4m3> {
   using Out = bf16;
 };
 
+constexpr int SMEM_LIMIT = 227 * 1024;
+constexpr int CTRL_BYTES = 2048;
+
 // BN: the MMA's N.  CG: CTAs per MMA (1, or 2 for a 256-row pair tile in which each CTA
-// holds 128 rows of A and BN/2 columns of B).
-template <typename T, int BN, int CG = 1> struct Cfg {
+// holds 128 rows of A and BN/2 columns of B).  EXTRA: bytes of shared memory the mode keeps
+// after the control block; the stage ring gives way to them.
+template <typename T, int BN, int CG = 1, int EXTRA = 0> struct Cfg {
   static constexpr bool MX = (ElemTraits<T>::ES == 1);
   static constexpr int BMP = BM * CG;                   // rows of an MMA tile (pair)
   static constexpr int BNC = BN / CG;                   // columns of B held by one CTA
@@ -85,11 +94,14 @@ template <typename T, int BN, int CG = 1> struct Cfg {
   static constexpr int A_BYTES = BM * KBLK * ES;
   static constexpr int B_BYTES = BNC * KBLK * ES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (STAGE_BYTES >= 48 * 1024) ? 4 : (STAGE_BYTES >= 32 * 1024 ? 6 : 8);
   // two accumulators; MXFP8 adds 8 columns of scale factors (A: 4, B: 4) after them
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
   static constexpr int SF_BYTES = MX ? 1024 : 0;        // per stage: 512-byte scale blocks of A and B
-  static constexpr int SMEM_BYTES = STAGES * (STAGE_BYTES + SF_BYTES) + 1024 /*align slack*/ + 2048 /*bars etc*/;
+  static constexpr int STAGES_WANTED = (STAGE_BYTES >= 48 * 1024) ? 4 : (STAGE_BYTES >= 32 * 1024 ? 6 : 8);
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES - EXTRA) / (STAGE_BYTES + SF_BYTES);
+  static constexpr int STAGES = STAGES_WANTED < STAGES_FIT ? STAGES_WANTED : STAGES_FIT;
+  static_assert(STAGES >= 2, "shared memory");
+  static constexpr int SMEM_BYTES = STAGES * (STAGE_BYTES + SF_BYTES) + 1024 /*align slack*/ + CTRL_BYTES + EXTRA;
 };
 
 struct Params {
@@ -133,7 +145,7 @@ struct Ctrl {
   uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t tail;
+  uint64_t tailbar[8];    // weight gradients: a stage's loads ran past the expert's rows
   uint64_t drain;
   uint64_t xfull[4];      // router: one lane quarter's second-half picks are in xbuf
   uint64_t xempty[4];     // router: ... and have been merged
@@ -144,10 +156,16 @@ struct Ctrl {
     float bias[MAX_E];      // router: the logit bias (0 past E)
   };
 };
-constexpr int CTRL_BYTES = 2048;
 static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
 // Router: shared buffer for the second-half picks, [MAX_K][BM] keys then [MAX_K][BM] experts
 constexpr int ROUTER_XBYTES = 2 * MAX_K * BM * 4;
+// Weight gradients: each epilogue warp stages its output in two boxes of 32 rows x 64 bf16
+// columns (128-byte rows, 128-byte swizzle) that TMA stores write out.
+constexpr int EPI_BOX_BYTES = 32 * 128;
+constexpr int WGRAD_XBYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
+template <int MODE> constexpr int extra_smem() {
+  return MODE == ROUTER ? ROUTER_XBYTES : ModeTraits<MODE>::WGRAD ? WGRAD_XBYTES : 0;
+}
 
 template <int MODE, int BN, int KBLK, bool MX, int CG = 1>
 __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl, int rank = 0) {
@@ -315,8 +333,10 @@ template <typename T, int BN, int MODE, int CG>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                         const __grid_constant__ CUtensorMap tmB0,
-                        const __grid_constant__ CUtensorMap tmB1, const Params p) {
-  using C = Cfg<T, BN, CG>;
+                        const __grid_constant__ CUtensorMap tmB1,
+                        const __grid_constant__ CUtensorMap tmO0,   // weight gradients: outputs
+                        const __grid_constant__ CUtensorMap tmO1, const Params p) {
+  using C = Cfg<T, BN, CG, extra_smem<MODE>()>;
   static_assert(CG == 1 || (sizeof(T) == 2 && MODE != ROUTER), "CTA pairs: bf16 grouped GEMMs only");
   constexpr int BMP = C::BMP, BNC = C::BNC;
   using MT = ModeTraits<MODE>;
@@ -328,7 +348,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint8_t *ring = smem;                                   // STAGES x (A | B)
   uint8_t *sf_ring = smem + C::STAGES * C::STAGE_BYTES;   // MXFP8: STAGES x (SFA | SFB)
   Ctrl &c = *reinterpret_cast<Ctrl *>(smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES));
-  uint32_t *xbuf = reinterpret_cast<uint32_t *>(smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES) + CTRL_BYTES);
+  uint8_t *extra = smem + C::STAGES * (C::STAGE_BYTES + C::SF_BYTES) + CTRL_BYTES;   // 1024-byte aligned
+  uint32_t *xbuf = reinterpret_cast<uint32_t *>(extra);
   volatile int *abort_flag = &c.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -349,7 +370,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
       ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), EPI_WARPS * CG);   // one arrival per epilogue warp
     }
-    ptx::mbar_init(ptx::smem_u32(&c.tail), 1);
+    for (int s = 0; s < C::STAGES; ++s) ptx::mbar_init(ptx::smem_u32(&c.tailbar[s]), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_init(ptx::smem_u32(&c.xfull[q]), 32);
@@ -360,6 +381,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tma_prefetch(&tmA);
     ptx::tma_prefetch(&tmB0);
     ptx::tma_prefetch(&tmB1);
+    if constexpr (MT::WGRAD) {
+      ptx::tma_prefetch(&tmO0);
+      ptx::tma_prefetch(&tmO1);
+    }
   }
   if (warp == 1) {
     if constexpr (CG == 2) {
@@ -371,7 +396,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
   if constexpr (MODE == ROUTER) {
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 2 + EPI_WARPS) {
       const float *bias = static_cast<const float *>(p.aux);
       for (int e = threadIdx.x - 64; e < MAX_E; e += 32 * EPI_WARPS) c.bias[e] = (bias && e < p.E) ? bias[e] : 0.f;
     }
@@ -412,9 +437,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 0) {
     // ================================================================ producer
     int stage = 0;
-    uint32_t phase = 0, tail_phase = 0;
+    uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;  // per stage: a fill is in flight / its parity
-    bool tail_armed = false;
+    uint32_t tarmed = 0, tlast = 0, tnext = 0;  // per stage: a tail fill was issued / the parity
+                                                // of the last one / of the next one
     bool ok = true;
     for (int t = tile0; t < ntiles && ok; t += tstep) {
       Tile tl;
@@ -431,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
         // pairs: the bytes of both CTAs' loads are counted on the leader's full barrier
         const uint32_t full_leader = CG == 2 ? ptx::mapa(full_local, 0) : full_local;
-        const uint32_t bar = tail ? ptx::smem_u32(&c.tail) : full_local;
+        const uint32_t bar = tail ? ptx::smem_u32(&c.tailbar[stage]) : full_local;
         const bool pair_load = CG == 2 && !tail;
         auto ld = [&](uint32_t dst, const CUtensorMap *tm, int x, int y) {
           if (pair_load) ptx::tma_load_2d_pair(dst, tm, full_leader, x, y);
@@ -528,40 +554,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
         }
         if (tail) {
-          // Weight gradients only: K rows past the expert's end belong to another expert
-          // (or lie outside the tensor): zero them before the MMA reads the stage.
-          tail_armed = true;
-          ok = ptx::mbar_wait(ptx::smem_u32(&c.tail), tail_phase, abort_flag, WAIT_LIMIT_NS);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
-          tail_armed = false;
-          tail_phase ^= 1;
-          // In an MN-major box each K row is one 128-byte line: rows [valid, KBLK) are the
-          // byte range [valid*128, KBLK*128) of every box.
-          const int nbox_a = BM / C::BOX_MN, nbox_b = BNC / C::BOX_MN;
-          const int line0 = valid * 8, lines = C::KBLK * 8;  // in 16-byte units
-          uint4 z = make_uint4(0, 0, 0, 0);
-          for (int b = 0; b < nbox_a + nbox_b; ++b) {
-            uint8_t *box = ring + stage * C::STAGE_BYTES + (b < nbox_a ? b * C::BOX_BYTES
-                                                                        : C::A_BYTES + (b - nbox_a) * C::BOX_BYTES);
-            for (int i = line0 + lane; i < lines; i += 32) reinterpret_cast<uint4 *>(box)[i] = z;
-          }
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            if constexpr (CG == 2) {
-              // the leader arrives expecting the peer's bytes; the peer posts them once its
-              // zeroed stage is visible (the tensor cores of the pair read it)
-              if (rank == 0) {
-                ptx::mbar_arrive_expect_tx(full_local, C::STAGE_BYTES);
-              } else {
-                ptx::fence_acq_rel_cluster();
-                ptx::mbar_complete_tx_cluster(full_leader, C::STAGE_BYTES);
-              }
-            } else {
-              ptx::mbar_arrive(full_local);
-            }
-          }
+          // the tail fixer warp zeroes the rows past the expert and releases the stage
+          tarmed |= 1u << stage;
+          tlast = (tlast & ~(1u << stage)) | (tnext & (1u << stage));
+          tnext ^= 1u << stage;
         }
         // this stage's full barrier completes (or has completed) the phase of this pass
         armed |= 1u << stage;
@@ -576,8 +572,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (rank == 0 && ((armed >> s) & 1u))
           if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
             note_fail(p, 0, 0, s, 2);
-      if (tail_armed && !ptx::mbar_wait(ptx::smem_u32(&c.tail), tail_phase, abort_flag, WAIT_LIMIT_NS))
-        note_fail(p, 0, 0, 0, 3);
+      for (int s = 0; s < C::STAGES; ++s)
+        if (((tarmed >> s) & 1u) &&
+            !ptx::mbar_wait(ptx::smem_u32(&c.tailbar[s]), (tlast >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
+          note_fail(p, 0, 0, s, 3);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -660,6 +658,58 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, abort_flag, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
     }
     __syncwarp();
+  } else if (warp == FIX_WARP) {
+    // ================================================================ tail fixer
+    // Weight gradients reduce over an expert's rows: K rows of a stage past the expert's end
+    // belong to another expert (or lie outside the tensor).  This warp follows the producer's
+    // sequence of stages, zeroes those rows once a tail stage's loads have landed and then
+    // releases the stage to the MMA issuer, so that the producer never waits on a load.
+    if constexpr (MT::WGRAD && !C::MX) {
+      int stage = 0;
+      uint32_t tpar = 0;  // per stage: parity of the next tail completion
+      bool ok = true;
+      for (int t = tile0; t < ntiles && ok; t += tstep) {
+        Tile tl;
+        get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
+        for (int kb = 0; kb < tl.num_kb; ++kb) {
+          const int valid = min(C::KBLK, tl.rows - kb * C::KBLK);
+          if (valid < C::KBLK) {
+            ok = ptx::mbar_wait(ptx::smem_u32(&c.tailbar[stage]), (tpar >> stage) & 1u, abort_flag, WAIT_LIMIT_NS);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
+            tpar ^= 1u << stage;
+            // In an MN-major box each K row is one 128-byte line: rows [valid, KBLK) are the
+            // byte range [valid*128, KBLK*128) of every box.
+            const int nbox_a = BM / C::BOX_MN, nbox_b = BNC / C::BOX_MN;
+            const int line0 = valid * 8, lines = C::KBLK * 8;  // in 16-byte units
+            const uint4 z = make_uint4(0, 0, 0, 0);
+            for (int b = 0; b < nbox_a + nbox_b; ++b) {
+              uint8_t *box = ring + stage * C::STAGE_BYTES +
+                             (b < nbox_a ? b * C::BOX_BYTES : C::A_BYTES + (b - nbox_a) * C::BOX_BYTES);
+              for (int i = line0 + lane; i < lines; i += 32) reinterpret_cast<uint4 *>(box)[i] = z;
+            }
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
+              if constexpr (CG == 2) {
+                // the leader arrives expecting the peer's bytes; the peer posts them once its
+                // zeroed stage is visible (the tensor cores of the pair read it)
+                if (rank == 0) {
+                  ptx::mbar_arrive_expect_tx(full_local, C::STAGE_BYTES);
+                } else {
+                  ptx::fence_acq_rel_cluster();
+                  ptx::mbar_complete_tx_cluster(ptx::mapa(full_local, 0), C::STAGE_BYTES);
+                }
+              } else {
+                ptx::mbar_arrive(full_local);
+              }
+            }
+          }
+          if (++stage == C::STAGES) stage = 0;
+        }
+      }
+    }
   } else {
     // ================================================================ epilogue
     using OutT = typename ElemTraits<T>::Out;
@@ -668,6 +718,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;     // 0 or 1
     const int r = q * 32 + lane;          // tile row owned by this thread
+    uint8_t *epi_box = extra + (warp - 2) * 2 * EPI_BOX_BYTES;   // weight gradients
+    int nst = 0;                          // weight gradients: boxes stored by this warp
     int it = 0;
     for (int t = tile0; t < ntiles; t += tstep, ++it) {
       Tile tl;
@@ -926,25 +978,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           store_slab(dhu + srow * 2 * p.f + col, 2 * p.f, nvalid, dh);
           store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
         }
-      } else {  // weight gradients: slab of rows q*32.. of the [M x N] block of expert e
-        const int64_t srow = (int64_t)tl.e * p.M + tl.mcol0 + q * 32;
+      } else {  // weight gradients: rows q*32.. of the [M x N] block of expert e
+        // Each 32 x 64 piece goes through one of the warp's two staging boxes in the layout
+        // of a 128-byte-swizzled TMA box (16-byte chunk j of row r at chunk j ^ (r % 8)); one
+        // lane then stores the box with TMA.  A box is refilled only once the store that
+        // last used it has read it.
+        static_assert(sizeof(OutT) == 2, "weight gradients are stored as bf16");
+        const int orow = tl.e * p.M + tl.mcol0 + q * 32;
 #pragma unroll 1
-        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 32) {
-          float v[32];
-          if (tl.num_kb > 0) ptx::tmem_ld32(taddr + cc, v);
-          else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-          }
-          const int col = tl.n_blk * BN + cc;
-          if constexpr (MODE == WGRAD_DOWN) {
-            OutT *out = static_cast<OutT *>(p.out0);
-            store_slab(out + srow * p.N + col, p.N, 32, v);
+        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 64, ++nst) {
+          float v0[32], v1[32];
+          if (tl.num_kb > 0) {
+            ptx::tmem_ld32(taddr + cc, v0);
+            ptx::tmem_ld32(taddr + cc + 32, v1);
           } else {
-            // N runs over [dh | du]: columns below f are dW_gate, the rest dW_up
-            OutT *out = static_cast<OutT *>(col < p.f ? p.out0 : p.out1);
-            const int cf = col < p.f ? col : col - p.f;
-            store_slab(out + srow * p.f + cf, p.f, 32, v);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) { v0[i] = 0.f; v1[i] = 0.f; }
+          }
+          uint8_t *box = epi_box + (nst & 1) * EPI_BOX_BYTES;
+          if (lane == 0) ptx::bulk_wait_read<1>();
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 w = Vec<OutT>::store(j < 4 ? &v0[8 * j] : &v1[8 * (j - 4)]);
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
+          }
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int col = tl.n_blk * BN + cc;
+            if constexpr (MODE == WGRAD_DOWN) {
+              ptx::tma_store_2d(&tmO0, ptx::smem_u32(box), col, orow);
+            } else {
+              // N runs over [dh | du]: columns below f are dW_gate, the rest dW_up
+              if (col < p.f) ptx::tma_store_2d(&tmO0, ptx::smem_u32(box), col, orow);
+              else ptx::tma_store_2d(&tmO1, ptx::smem_u32(box), col - p.f, orow);
+            }
+            ptx::bulk_commit();
           }
         }
       }
@@ -956,6 +1026,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         else ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
       }
     }
+    // weight gradients: the staging boxes stay in use until their TMA stores complete
+    if constexpr (MT::WGRAD)
+      if (lane == 0) ptx::bulk_wait_all();
   }
 
   // ------------------------------------------------------------------ teardown
@@ -1018,11 +1091,14 @@ static int sm_count() {
 // of two (CG = 2); never more CTAs (pairs) than tiles.
 template <typename T, int BN, int MODE, int CG = 1>
 static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p,
-                  int64_t max_tiles, cudaStream_t st) {
-  using C = Cfg<T, BN, CG>;
+                  int64_t max_tiles, cudaStream_t st, const CUtensorMap *o0 = nullptr,
+                  const CUtensorMap *o1 = nullptr) {
+  using C = Cfg<T, BN, CG, extra_smem<MODE>()>;
   auto kern = grouped_gemm_kernel<T, BN, MODE, CG>;
-  constexpr int SMEM = C::SMEM_BYTES + (MODE == ROUTER ? ROUTER_XBYTES : 0);
-  static_assert(SMEM <= 227 * 1024, "shared memory");
+  constexpr int SMEM = C::SMEM_BYTES;
+  static_assert(SMEM <= SMEM_LIMIT, "shared memory");
+  if (ModeTraits<MODE>::WGRAD && (!o0 || !o1)) return MOE_ERR_INVALID_ARG;
+  const CUtensorMap &out0 = o0 ? *o0 : a, &out1 = o1 ? *o1 : a;
   static bool attr_set = false;
   if (!attr_set) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
@@ -1031,7 +1107,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   }
   if constexpr (CG == 1) {
     const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
-    kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, p);
+    kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, out0, out1, p);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(NUM_THREADS);
@@ -1056,7 +1132,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
     }
     const int64_t units = std::min<int64_t>(max_pairs, std::max<int64_t>(max_tiles, 1));
     cfg.gridDim = dim3((unsigned)(units * CG));
-    if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, p) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, out0, out1, p) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -1168,18 +1244,20 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   }
   // (2) dWd[e] = a^T [f, rows_e] x dy_perm [rows_e, d]
   {
+    CUtensorMap tO;
+    if (!make_tmap(&tO, dw_down, ES, s.d, (uint64_t)s.E * s.f, 64, 32)) return MOE_ERR_CUDA;
     if (!make_tmap(&tA, a, ES, s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
     if (s.d % 256 == 0 && s.f % 256 == 0) {
       // weight-gradient tiles are 256 weight rows (no empty rows): always CTA pairs
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 256, WGRAD_DOWN, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / 256) * (s.d / 256), st);
+      rc = launch<T, 256, WGRAD_DOWN, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / 256) * (s.d / 256), st, &tO, &tO);
     } else if (s.d % 256 == 0) {
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st);
+      rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st, &tO, &tO);
     } else {
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 128, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st);
+      rc = launch<T, 128, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st, &tO, &tO);
     }
     if (rc) return rc;
   }
@@ -1206,13 +1284,17 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   {
     if (!make_tmap(&tA, x_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     if (!make_tmap(&tB0, dhu, ES, 2 * s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
+    CUtensorMap tO0, tO1;
+    if (!make_tmap(&tO0, dw_gate, ES, s.f, (uint64_t)s.E * s.d, 64, 32) ||
+        !make_tmap(&tO1, dw_up, ES, s.f, (uint64_t)s.E * s.d, 64, 32))
+      return MOE_ERR_CUDA;
     p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
     if (s.f % 256 == 0 && s.d % 256 == 0)
-      rc = launch<T, 256, WGRAD_GU, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / 256) * (2 * s.f / 256), st);
+      rc = launch<T, 256, WGRAD_GU, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / 256) * (2 * s.f / 256), st, &tO0, &tO1);
     else if (s.f % 256 == 0)
-      rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st);
+      rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st, &tO0, &tO1);
     else
-      rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st);
+      rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st, &tO0, &tO1);
     if (rc) return rc;
   }
   return MOE_OK;
@@ -1311,9 +1393,11 @@ static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, 
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, aqt.codes, 1, s.f, R, 128, 128) || !make_tmap(&tB, dyqt.codes, 1, s.d, R, 128, 128))
     return MOE_ERR_CUDA;
+  CUtensorMap tO0, tO1;
+  if (!make_tmap(&tO0, dw_down, 2, s.d, ef, 64, 32)) return MOE_ERR_CUDA;
   p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
   p.sfa = aqt.scales; p.sfa_ld = s.f; p.sfb = dyqt.scales; p.sfb_ld = s.d;
-  rc = launch<e4m3, 128, WGRAD_DOWN>(tA, tB, tB, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st);
+  rc = launch<e4m3, 128, WGRAD_DOWN>(tA, tB, tB, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st, &tO0, &tO0);
   if (rc) return rc;
   // (3) dx_perm = [dh | du] [Wg | Wu]^T
   if (launch_mx_quant_rows(dhu, P, 2 * s.f, offsets, s.E, R, dhuq.codes, dhuq.scales, st) ||
@@ -1331,9 +1415,11 @@ static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, 
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, xqt.codes, 1, s.d, R, 128, 128) || !make_tmap(&tB, dhuqt.codes, 1, 2 * s.f, R, 128, 128))
     return MOE_ERR_CUDA;
+  if (!make_tmap(&tO0, dw_gate, 2, s.f, ed, 64, 32) || !make_tmap(&tO1, dw_up, 2, s.f, ed, 64, 32))
+    return MOE_ERR_CUDA;
   p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
   p.sfa = xqt.scales; p.sfa_ld = s.d; p.sfb = dhuqt.scales; p.sfb_ld = 2 * s.f;
-  return launch<e4m3, 128, WGRAD_GU>(tA, tB, tB, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st);
+  return launch<e4m3, 128, WGRAD_GU>(tA, tB, tB, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st, &tO0, &tO1);
 }
 
 }  // namespace gg
