@@ -33,7 +33,11 @@ arithmetic out.  Where they are silent this oracle takes the plainest reading:
   * rows inside one expert's buffer keep the order of the routed pairs
     (pair i = t*k + j), i.e. a stable counting sort by expert;
   * MXFP8: OCP Microscaling v1.0 with E4M3 elements and an E8M0 scale per
-    32-element block along each GEMM's reduction axis.
+    32-element block along each GEMM's reduction axis;
+  * shared expert ([bigchange], section "Что инженер может попробовать на
+    практике": the production rows use top-four routing and one shared expert):
+    a SwiGLU of the routed experts' shape that every token passes through, its
+    output added to the routed experts' gate-weighted sum with weight 1.
 
 Parity pins for every function live in tests/test_oracle_*.py.  Nothing here
 is "parity unpinned".
@@ -193,20 +197,31 @@ def combine(y_perm, slot_of_pair, gate):
     return Y
 
 
-def layer_fwd(x, w_r, w_gate, w_up, w_down, k, bias=None):
-    """Whole forward step.  Returns a dict with every intermediate."""
+def shared_expert_fwd(x, shared):
+    """The shared expert on every token: shared = (W_gate [d,f], W_up [d,f], W_down [f,d])."""
+    h, u, a, y = expert_swiglu(x, *shared)
+    return dict(shared_h=h, shared_u=u, shared_a=a, shared_y=y)
+
+
+def layer_fwd(x, w_r, w_gate, w_up, w_down, k, bias=None, shared=None):
+    """Whole forward step.  Returns a dict with every intermediate.  shared: None or the
+    shared expert's (W_gate, W_up, W_down)."""
     E = w_gate.shape[0]
     z, p, idx, gate = route(x, w_r, k, bias)
     counts, offsets, slot_of_pair, pair_of_slot = routing_metadata(idx, E)
     x_perm = permute(x, pair_of_slot, k)
     h, u, a, y_perm = grouped_swiglu(x_perm, offsets, w_gate, w_up, w_down)
     Y = combine(y_perm, slot_of_pair, gate)
-    return dict(z=z, p=p, idx=idx, gate=gate, counts=counts, offsets=offsets,
-                slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot, x_perm=x_perm,
-                h=h, u=u, a=a, y_perm=y_perm, y=Y)
+    out = dict(z=z, p=p, idx=idx, gate=gate, counts=counts, offsets=offsets,
+               slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot, x_perm=x_perm,
+               h=h, u=u, a=a, y_perm=y_perm, y=Y)
+    if shared is not None:
+        out.update(shared_expert_fwd(x, shared))
+        out["y"] = Y + out["shared_y"]
+    return out
 
 
-def layer_fwd_routed(x, idx, gate, w_gate, w_up, w_down):
+def layer_fwd_routed(x, idx, gate, w_gate, w_up, w_down, shared=None):
     """Forward step from given routing (uniform random routing enters here)."""
     E = w_gate.shape[0]
     k = idx.shape[1]
@@ -214,9 +229,13 @@ def layer_fwd_routed(x, idx, gate, w_gate, w_up, w_down):
     x_perm = permute(x, pair_of_slot, k)
     h, u, a, y_perm = grouped_swiglu(x_perm, offsets, w_gate, w_up, w_down)
     Y = combine(y_perm, slot_of_pair, gate)
-    return dict(idx=np.asarray(idx), gate=np.asarray(gate, F64), counts=counts,
-                offsets=offsets, slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot,
-                x_perm=x_perm, h=h, u=u, a=a, y_perm=y_perm, y=Y)
+    out = dict(idx=np.asarray(idx), gate=np.asarray(gate, F64), counts=counts,
+               offsets=offsets, slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot,
+               x_perm=x_perm, h=h, u=u, a=a, y_perm=y_perm, y=Y)
+    if shared is not None:
+        out.update(shared_expert_fwd(x, shared))
+        out["y"] = Y + out["shared_y"]
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -310,7 +329,20 @@ def route_bwd(dgate, gate, idx, x, w_r):
     return dz, dw_r, dx
 
 
-def layer_bwd(fwd, dY, x, w_r, w_gate, w_up, w_down):
+def shared_expert_bwd(dY, x, fwd, shared):
+    """The shared expert's backward: its output gradient is dY itself (weight 1).  The
+    SwiGLU backward of one expert holding every token, in the same steps as the routed
+    experts'.  Returns dx and the three weight gradients."""
+    T = np.asarray(x).shape[0]
+    one = [np.asarray(w, F64)[None] for w in shared]     # one expert [1, ...]
+    g = grouped_swiglu_bwd(dY, x, fwd["shared_h"], fwd["shared_u"], fwd["shared_a"],
+                           np.array([0, T]), *one)
+    return dict(shared_dx=g["dx_perm"], dw_shared_gate=g["dw_gate"][0],
+                dw_shared_up=g["dw_up"][0], dw_shared_down=g["dw_down"][0],
+                shared_dh=g["dh"], shared_du=g["du"])
+
+
+def layer_bwd(fwd, dY, x, w_r, w_gate, w_up, w_down, shared=None):
     """Whole backward step, given the forward dict from layer_fwd."""
     T, k = fwd["gate"].shape
     dy_perm, dgate = combine_bwd(dY, fwd["y_perm"], fwd["slot_of_pair"], fwd["gate"])
@@ -320,17 +352,25 @@ def layer_bwd(fwd, dY, x, w_r, w_gate, w_up, w_down):
     dz, dw_r, dx_r = route_bwd(dgate, fwd["gate"], fwd["idx"], x, w_r)
     out = dict(dy_perm=dy_perm, dgate=dgate, dz=dz, dw_r=dw_r, dx=dx + dx_r,
                dx_experts=dx, **g)
+    if shared is not None:
+        out.update(shared_expert_bwd(dY, x, fwd, shared))
+        out["dx"] = out["dx"] + out["shared_dx"]
     return out
 
 
-def layer_bwd_routed(fwd, dY, w_gate, w_up, w_down):
-    """Backward with routing held fixed (no router gradient): uniform-random routing."""
+def layer_bwd_routed(fwd, dY, w_gate, w_up, w_down, x=None, shared=None):
+    """Backward with routing held fixed (no router gradient): uniform-random routing.
+    With a shared expert, x (the layer input) is needed too."""
     T, k = fwd["gate"].shape
     dy_perm, dgate = combine_bwd(dY, fwd["y_perm"], fwd["slot_of_pair"], fwd["gate"])
     g = grouped_swiglu_bwd(dy_perm, fwd["x_perm"], fwd["h"], fwd["u"], fwd["a"],
                            fwd["offsets"], w_gate, w_up, w_down)
     dx = unpermute_sum(g["dx_perm"], fwd["slot_of_pair"], T, k)
-    return dict(dy_perm=dy_perm, dgate=dgate, dx=dx, **g)
+    out = dict(dy_perm=dy_perm, dgate=dgate, dx=dx, **g)
+    if shared is not None:
+        out.update(shared_expert_bwd(dY, x, fwd, shared))
+        out["dx"] = out["dx"] + out["shared_dx"]
+    return out
 
 
 # ---------------------------------------------------------------------------
