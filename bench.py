@@ -39,6 +39,10 @@ WORKLOADS = {
     # the same shapes with every grouped-GEMM operand in MXFP8 (E4M3 + E8M0 per 32)
     "e128_t16k_mxfp8_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "router", "mxfp8"),
     "e128_mxfp8_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "mxfp8"),
+    # the C3 shapes plus one shared expert (every token, weight 1) of the routed experts' shape
+    "e128_shared_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "native", {"shared": True}),
+    # the C3 shapes keeping no [h | u] between forward and backward (recomputed there)
+    "e128_recompute_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "native", {"recompute": True}),
 }
 DEFAULT = "e128_fwd_bwd"
 
@@ -146,24 +150,30 @@ def run_ours(args):
     name = args.workload
     T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
     prec = WORKLOADS[name][7] if len(WORKLOADS[name]) > 7 else "native"
+    opts = WORKLOADS[name][8] if len(WORKLOADS[name]) > 8 else {}
+    shared, recompute = bool(opts.get("shared")), bool(opts.get("recompute"))
     inp = make_inputs(name, seed=0)
     cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
     st = torch.cuda.current_stream()
     ws = moe.alloc_workspace(cfg)
-    saved = moe.alloc_saved(cfg, logits=False)
-    grads = moe.alloc_grads(cfg, router=(routing == "router"))
+    saved = moe.alloc_saved(cfg, logits=False, shared=shared, recompute=recompute)
+    grads = moe.alloc_grads(cfg, router=(routing == "router"), shared=shared)
     x = to_dev_bf16(inp.x, torch)
     dy = to_dev_bf16(inp.dy, torch)
     wr, wg, wu, wd = (to_dev_bf16(a, torch) for a in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down))
     bias = torch.from_numpy(inp.bias).cuda() if inp.bias is not None else None
-    w = moe.layer_weights(wr, bias, wg, wu, wd)
+    sh = None
+    if shared:
+        from routing_grouped_expert_softmax_b200 import inputs as gen
+        sh = tuple(to_dev_bf16(a, torch) for a in gen.make_shared_expert(d, f, seed=1))
+    w = moe.layer_weights(wr, bias, wg, wu, wd, shared=sh)
     y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
     fwd_fn = moe.moe_layer_fwd
     if routing == "uniform":
         saved["topk_idx"].copy_(torch.from_numpy(inp.extra["idx"]))
         saved["topk_gate"].copy_(torch.from_numpy(inp.extra["gate"]))
         fwd_fn = moe.moe_layer_fwd_routed
-    launches_per_step = count_launches(routing, prec)
+    launches_per_step = count_launches(routing, prec, shared, recompute)
 
     def step():
         fwd_fn(cfg, w, x, y, saved, ws, st)
@@ -202,13 +212,14 @@ def run_ours(args):
 
     # ---- the grouped GEMMs alone (6 tcgen05 launches per step), same stream and inputs
     g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    hu_buf = saved["hu"] if saved["hu"] is not None else grads["dhu"]   # recompute keeps no h | u
     fwd_ms = bwd_ms = 0.0
     for _ in range(args.steps):
         g0.record(st)
-        moe.moe_grouped_swiglu_fwd(cfg, saved["x_perm"], saved["offsets"], wg, wu, wd, saved["hu"],
+        moe.moe_grouped_swiglu_fwd(cfg, saved["x_perm"], saved["offsets"], wg, wu, wd, hu_buf,
                                    saved["a"], saved["y_perm"], ws, st)
         g1.record(st)
-        moe.moe_grouped_swiglu_bwd(cfg, grads["dy_perm"], saved["x_perm"], saved["hu"], saved["a"],
+        moe.moe_grouped_swiglu_bwd(cfg, grads["dy_perm"], saved["x_perm"], hu_buf, saved["a"],
                                    saved["offsets"], wg, wu, wd, grads["dhu"], grads["dx_perm"],
                                    grads["dw_gate"], grads["dw_up"], grads["dw_down"], ws, st)
         g2.record(st)
@@ -267,6 +278,7 @@ def run_ours(args):
         "config": {"workload": name, "T": T, "d_model": d, "experts": E, "top_k": k, "ffn": f,
                    "routing": "skewed (Zipf bias)" if skew else routing, "gemm_precision": prec,
                    "parallelism": f"replicas x{ws_n}" if ws_n > 1 else "single GPU",
+                   "shared_expert": shared, "recompute_hu": recompute,
                    "l2": "no flush: 1.6 GB of expert weights per step exceed the 126 MB L2"},
         "roofline": {"kernel": "grouped SwiGLU GEMMs (6 tcgen05 launches: fwd gate/up, fwd down, "
                                "dgrad down, wgrad down, dgrad gate/up, wgrad gate/up)",
@@ -296,13 +308,22 @@ def gen_bits(a):
     return gen.bf16_bits(a).view(np.int16).reshape(-1)
 
 
-def count_launches(routing, prec="native"):
+def count_launches(routing, prec="native", shared=False, recompute=False):
     """Kernels one step launches: forward (router 1, metadata 3, permute 1, grouped GEMMs 2,
     combine 1) and backward (combine-bwd 1, grouped GEMMs 4, router transpose 1, router
-    weight-gradient 3, unpermute-sum 1); MXFP8 adds 4 quantisers forward, 8 backward."""
+    weight-gradient 3, unpermute-sum 1); MXFP8 adds 4 quantisers forward, 8 backward.  A
+    shared expert adds its group offsets and 2 GEMMs forward, offsets and 4 GEMMs backward
+    (MXFP8: 4 + 8 more quantisers); recompute adds one GEMM per expert set backward (MXFP8:
+    with its 2 quantisers)."""
     fwd = (1 if routing == "router" else 0) + 3 + 1 + 2 + 1
     bwd = 1 + 4 + (5 if routing == "router" else 1)
-    return fwd + bwd + (12 if prec == "mxfp8" else 0)
+    n = fwd + bwd + (12 if prec == "mxfp8" else 0)
+    sets = 2 if shared else 1
+    if shared:
+        n += 1 + 2 + 1 + 4 + (12 if prec == "mxfp8" else 0)
+    if recompute:
+        n += sets * (1 + (2 if prec == "mxfp8" else 0))
+    return n
 
 
 def cpu_baseline(inp, k, n_tokens):

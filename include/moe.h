@@ -233,6 +233,14 @@ typedef struct moe_layer_weights {
   const void *w_gate;   /* [E,d,f] */
   const void *w_up;     /* [E,d,f] */
   const void *w_down;   /* [E,f,d] */
+  /* Optional shared expert (bigchange.ai, "Olmo-core 3 открывает стек обучения MoE от
+   * Ai2 ...", section "Что инженер может попробовать на практике": the published production
+   * rows route each token to four experts and also use one shared expert).  A SwiGLU of
+   * the routed experts' shape that every token passes through; its output is added to the
+   * gate-weighted sum of the routed experts with weight 1.  All three NULL: none. */
+  const void *w_shared_gate; /* [d,f] */
+  const void *w_shared_up;   /* [d,f] */
+  const void *w_shared_down; /* [f,d] */
 } moe_layer_weights;
 
 /* Buffers the forward fills and the backward reads (caller-owned). */
@@ -245,9 +253,11 @@ typedef struct moe_layer_saved {
   int32_t *slot_of_pair;  /* [P] */
   int32_t *pair_of_slot;  /* [P] */
   void *x_perm;           /* [P,d] */
-  void *hu;               /* [P,2f] */
+  void *hu;               /* [P,2f] (h | u), or NULL: the backward recomputes them */
   void *a;                /* [P,f] */
   void *y_perm;           /* [P,d] */
+  void *shared_hu;        /* [T,2f] with a shared expert, or NULL: recomputed */
+  void *shared_a;         /* [T,f] with a shared expert */
 } moe_layer_saved;
 
 /* Outputs of the backward, plus its intermediates (caller-owned). */
@@ -259,13 +269,24 @@ typedef struct moe_layer_grads {
   void *dw_down;     /* [E,f,d] */
   void *dy_perm;     /* [P,d] intermediate */
   float *dgate;      /* [T,k] intermediate */
-  void *dhu;         /* [P,2f] intermediate */
+  void *dhu;         /* [P,2f] intermediate (also holds recomputed h | u) */
   void *dx_perm;     /* [P,d] intermediate */
+  void *dw_shared_gate; /* [d,f] with a shared expert */
+  void *dw_shared_up;   /* [d,f] */
+  void *dw_shared_down; /* [f,d] */
+  void *shared_dhu;     /* [T,2f] intermediate with a shared expert */
 } moe_layer_grads;
 
 /* Whole forward: route_topk -> build_offsets -> permute -> grouped SwiGLU ->
  * unpermute_combine, all enqueued on `stream` with no host synchronisation.
- *   x [T,d]; y [T,d] out. */
+ *   x [T,d]; y [T,d] out.
+ * With a shared expert, its SwiGLU runs through the grouped GEMM as one group of all T
+ * tokens (x itself is that group's buffer), writes y, and the combine adds the routed
+ * experts' gate-weighted rows to it.
+ * Recompute (bigchange.ai, section "Три числа, три знаменателя": the largest published
+ * row recomputes activations in every layer): saved->hu == NULL keeps only a; the
+ * backward then recomputes h | u from x_perm (one extra grouped GEMM) into g->dhu and
+ * runs the SwiGLU backward in place there.  The same holds for saved->shared_hu. */
 MOE_API int moe_layer_fwd(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
                   const moe_layer_saved *saved, void *ws, moe_stream_t stream);
 

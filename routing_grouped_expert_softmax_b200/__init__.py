@@ -50,14 +50,16 @@ class MoeConfig(ctypes.Structure):
         return self.T * self.k
 
 
-class LayerWeights(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("w_router", "bias", "w_gate", "w_up", "w_down")]
-
-
+WEIGHT_FIELDS = ("w_router", "bias", "w_gate", "w_up", "w_down", "w_shared_gate", "w_shared_up",
+                 "w_shared_down")
 SAVED_FIELDS = ("logits", "topk_idx", "topk_gate", "counts", "offsets", "slot_of_pair",
-                "pair_of_slot", "x_perm", "hu", "a", "y_perm")
+                "pair_of_slot", "x_perm", "hu", "a", "y_perm", "shared_hu", "shared_a")
 GRAD_FIELDS = ("dx", "dw_router", "dw_gate", "dw_up", "dw_down", "dy_perm", "dgate", "dhu",
-               "dx_perm")
+               "dx_perm", "dw_shared_gate", "dw_shared_up", "dw_shared_down", "shared_dhu")
+
+
+class LayerWeights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in WEIGHT_FIELDS]
 
 
 class LayerSaved(ctypes.Structure):
@@ -235,8 +237,11 @@ def _struct(cls, fields, d):
     return cls(*[ptr(d.get(n)) for n in fields])
 
 
-def layer_weights(w_router, bias, w_gate, w_up, w_down) -> LayerWeights:
-    return LayerWeights(ptr(w_router), ptr(bias), ptr(w_gate), ptr(w_up), ptr(w_down))
+def layer_weights(w_router, bias, w_gate, w_up, w_down, shared=None) -> LayerWeights:
+    """shared: None, or (w_shared_gate [d,f], w_shared_up [d,f], w_shared_down [f,d])."""
+    sg, su, sd = shared if shared is not None else (None, None, None)
+    return LayerWeights(ptr(w_router), ptr(bias), ptr(w_gate), ptr(w_up), ptr(w_down), ptr(sg), ptr(su),
+                        ptr(sd))
 
 
 def moe_layer_fwd(cfg, weights: LayerWeights, x, y, saved: dict, ws, stream=None):
@@ -271,11 +276,14 @@ def alloc_workspace(cfg, device="cuda"):
     return torch.zeros(max(moe_workspace_size(cfg), 256), dtype=torch.uint8, device=device)
 
 
-def alloc_saved(cfg, device="cuda", logits=True) -> dict:
+def alloc_saved(cfg, device="cuda", logits=True, shared=False, recompute=False) -> dict:
+    """Forward buffers.  shared: room for a shared expert's activations; recompute: keep no
+    [h | u] (the backward recomputes them), which leaves hu (and shared_hu) None."""
     import torch
     dt = torch_dtype(cfg)
     T, d, E, k, f, P = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.T * cfg.k
     i32 = dict(dtype=torch.int32, device=device)
+    keep_hu = not recompute
     return dict(
         logits=torch.empty(T, E, dtype=torch.float32, device=device) if logits else None,
         topk_idx=torch.empty(T, k, **i32),
@@ -283,13 +291,15 @@ def alloc_saved(cfg, device="cuda", logits=True) -> dict:
         counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
         slot_of_pair=torch.empty(P, **i32), pair_of_slot=torch.empty(P, **i32),
         x_perm=torch.empty(P, d, dtype=dt, device=device),
-        hu=torch.empty(P, 2 * f, dtype=dt, device=device),
+        hu=torch.empty(P, 2 * f, dtype=dt, device=device) if keep_hu else None,
         a=torch.empty(P, f, dtype=dt, device=device),
         y_perm=torch.empty(P, d, dtype=dt, device=device),
+        shared_hu=torch.empty(T, 2 * f, dtype=dt, device=device) if shared and keep_hu else None,
+        shared_a=torch.empty(T, f, dtype=dt, device=device) if shared else None,
     )
 
 
-def alloc_grads(cfg, device="cuda", router=True) -> dict:
+def alloc_grads(cfg, device="cuda", router=True, shared=False) -> dict:
     import torch
     dt = torch_dtype(cfg)
     T, d, E, k, f, P = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.T * cfg.k
@@ -303,4 +313,8 @@ def alloc_grads(cfg, device="cuda", router=True) -> dict:
         dgate=torch.empty(T, k, dtype=torch.float32, device=device),
         dhu=torch.empty(P, 2 * f, dtype=dt, device=device),
         dx_perm=torch.empty(P, d, dtype=dt, device=device),
+        dw_shared_gate=torch.empty(d, f, dtype=dt, device=device) if shared else None,
+        dw_shared_up=torch.empty(d, f, dtype=dt, device=device) if shared else None,
+        dw_shared_down=torch.empty(f, d, dtype=dt, device=device) if shared else None,
+        shared_dhu=torch.empty(T, 2 * f, dtype=dt, device=device) if shared else None,
     )

@@ -43,7 +43,7 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Workspace carve-up shared by the host launchers.
 struct WsLayout {
   size_t block_counts;   // int32 [nblocks][E]
-  size_t w_rt;           // fp32 [E][d]   (transposed router weight)
+  size_t w_rt;           // [E][d] in the storage type (transposed router weight)
   size_t dwr_partial;    // fp32 [RB_SPLIT][E][d]
   size_t wt;             // fp32 storage only: Wg^T, Wu^T [E][f][d] and Wd^T [E][d][f]
   size_t dz_slot;        // fp32 [P]: router logit gradient of the pair in each slot
@@ -52,6 +52,9 @@ struct WsLayout {
   //   *_r: blocks along the row (K-major use), *_t: blocks down the rows (token axis)
   size_t xq_r, aq_r, dyq_r, dhuq_r, xq_t, aq_t, dyq_t, dhuq_t;  // activations, Ppad rows
   size_t wgu_c, wd_c, wd_r, wgu_r;                              // weights
+  // int32 {0, T}: the shared expert's single group.  Last, so that a layout for the shared
+  // expert's shape (E = 1, k = 1: every region no larger) never reaches it.
+  size_t group_offsets;
   size_t total;
 };
 // bytes of an MXFP8 operand [rows][cols] with scales along the row / down the rows
@@ -88,6 +91,7 @@ inline WsLayout ws_layout(const Shape &s) {
     L.wd_r = off;   off += mx_bytes_r(ef, s.d);
     L.wgu_r = off;  off += mx_bytes_r(ed, 2 * s.f);
   }
+  L.group_offsets = off; off += 256;   // {0, T}: the shared expert's single group
   L.total = off;
   return L;
 }
@@ -146,16 +150,18 @@ cudaError_t launch_build_offsets(const Shape &s, const int32_t *idx, int32_t *co
                                  int32_t *block_counts, int *err, cudaStream_t st);
 cudaError_t launch_permute(const Shape &s, const void *x, const int32_t *slot_of_pair,
                            void *x_perm, cudaStream_t st);
+// accumulate: add to the values y already holds (the shared expert's output)
 cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const int32_t *sop,
-                                     const float *gate, void *y, cudaStream_t st);
+                                     const float *gate, void *y, cudaStream_t st, bool accumulate = false);
+cudaError_t launch_group_offsets(int32_t *o, int64_t T, cudaStream_t st);
 cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm,
                                const int32_t *sop, const float *gate, void *dy_perm,
                                float *dgate, cudaStream_t st);
 // dx[t] = sum_j dx_perm[slot(t,j)] (+ sum_j dz_j W_r^T[e_j] when w_rt != nullptr)
 cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int32_t *sop,
                                  const float *dgate, const float *gate, const int32_t *idx,
-                                 const float *w_rt, bool accumulate, void *dx, cudaStream_t st);
-cudaError_t launch_router_transpose(const Shape &s, const void *w_r, float *w_rt, cudaStream_t st);
+                                 const void *w_rt, bool accumulate, void *dx, cudaStream_t st);
+cudaError_t launch_router_transpose(const Shape &s, const void *w_r, void *w_rt, cudaStream_t st);
 // dW_r from the expert-contiguous rows x_perm and the slot maps (layer backward)
 cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, const int32_t *pos,
                                         const int32_t *offsets, const float *dgate, const float *gate,

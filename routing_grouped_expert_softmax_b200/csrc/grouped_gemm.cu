@@ -902,7 +902,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (j < p.k) { idx[row * p.k + j] = pe[j]; gate[row * p.k + j] = ex[j] * inv; }
         }
       } else if constexpr (MODE == FWD_GU) {
-        // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range
+        // columns [0, BN/2) hold h = x Wg, [BN/2, BN) hold u = x Wu for the same f-range;
+        // either output may be absent (h, u not kept when the backward recomputes them; a not
+        // needed when the backward recomputes h, u)
         const bool valid = r < tl.rows;
         const int nvalid = min(32, max(0, tl.rows - q * 32));
         const int64_t srow = (int64_t)tl.orow0 + q * 32;      // output row of slab row 0
@@ -914,12 +916,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tmem_ld32(taddr + cc, h);
           ptx::tmem_ld32(taddr + BN / 2 + cc, u);
           const int col = tl.n_blk * (BN / 2) + cc;
-          store_slab(hu + srow * 2 * p.f + col, 2 * p.f, nvalid, h);
-          store_slab(hu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, u);
-          float a[32];
+          if (hu) {
+            store_slab(hu + srow * 2 * p.f + col, 2 * p.f, nvalid, h);
+            store_slab(hu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, u);
+          }
+          if (aa) {
+            float a[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) a[i] = valid ? h[i] * sigmoidf_(h[i]) * u[i] : 0.f;
-          store_slab(aa + srow * p.f + col, p.f, nvalid, a);
+            for (int i = 0; i < 32; ++i) a[i] = valid ? h[i] * sigmoidf_(h[i]) * u[i] : 0.f;
+            store_slab(aa + srow * p.f + col, p.f, nvalid, a);
+          }
         }
       } else if constexpr (MODE == FWD_DOWN || MODE == DGRAD_GU) {
         const int nvalid = min(32, max(0, tl.rows - q * 32));
@@ -1186,6 +1192,7 @@ static int fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, 
     if (rc < 0) rc = launch<T, BN, FWD_GU>(tA, tB0, tB1, p, mblocks * (p.N / BN), st);
     if (rc) return rc;
   }
+  if (!y_perm) return MOE_OK;   // [h | u] only (the backward's recompute)
   // GEMM 2: y_perm = a [P,f] x Wd [f,d]
   {
     if (!make_tmap(&tA, a, ES, s.f, P, KBLK, BM)) return MOE_ERR_CUDA;
@@ -1338,7 +1345,7 @@ static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offset
   const MxOp wgu = mx_r(ws, L.wgu_c, ed, 2 * s.f), wd = mx_r(ws, L.wd_c, ef, s.d);
   if (launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st) ||
       launch_mx_quant_cols_gu(w_gate, w_up, ed, s.f, wgu.codes, wgu.scales, st) ||
-      launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st))
+      (y_perm && launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st)))
     return MOE_ERR_CUDA;
   int *err = err_word(ws);
   Params p{};
@@ -1351,7 +1358,7 @@ static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offset
   p.K = s.d; p.N = 2 * s.f; p.out0 = hu; p.out1 = a;
   p.sfa = xq.scales; p.sfa_ld = s.d / 32; p.sfb = wgu.scales; p.sfb_ld = 2 * s.f;
   int rc = launch<e4m3, 128, FWD_GU>(tA, tB, tB, p, mblocks * (p.N / 128), st);
-  if (rc) return rc;
+  if (rc || !y_perm) return rc;   // no y_perm: [h | u] only (the backward's recompute)
   // GEMM 2: y_perm = a Wd
   if (launch_mx_quant_rows(a, P, s.f, offsets, s.E, R, aq.codes, aq.scales, st)) return MOE_ERR_CUDA;
   if (!make_tmap(&tA, aq.codes, 1, s.f, R, 128, BM) || !make_tmap(&tB, wd.codes, 1, s.d, ef, 128, 128))

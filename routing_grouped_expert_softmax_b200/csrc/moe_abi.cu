@@ -31,6 +31,12 @@ int check_ptrs(std::initializer_list<const void *> ps) {
     if (!p || !aligned16(p)) return MOE_ERR_INVALID_ARG;
   return MOE_OK;
 }
+// As check_ptrs, but NULL is allowed (an optional buffer).
+int check_ptrs_or_null(std::initializer_list<const void *> ps) {
+  for (const void *p : ps)
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
 // Pointers that only need to be non-null and 4-byte aligned (index and fp32 arrays).
 int check_ptrs4(std::initializer_list<const void *> ps) {
   for (const void *p : ps)
@@ -207,12 +213,26 @@ int moe_route_bwd(const moe_config *cfg, const float *dgate, const float *topk_g
   }
   WsLayout L = ws_layout(s);
   char *w = static_cast<char *>(ws);
-  float *w_rt = reinterpret_cast<float *>(w + L.w_rt);
+  void *w_rt = w + L.w_rt;
   float *part = reinterpret_cast<float *>(w + L.dwr_partial);
   RETURN_IF(cuda_rc(launch_router_transpose(s, w_router, w_rt, S(stream))));
   RETURN_IF(cuda_rc(launch_router_wgrad(s, dgate, topk_gate, topk_idx, x, part, dw_router, S(stream))));
   return cuda_rc(launch_unpermute_sum(s, nullptr, nullptr, dgate, topk_gate, topk_idx, w_rt, true, dx,
                                       S(stream)));
+}
+
+// The shared expert as a problem of its own: one group (E = 1) of all T tokens (k = 1).
+static Shape shared_shape(const Shape &s) {
+  Shape t = s;
+  t.E = 1;
+  t.k = 1;
+  return t;
+}
+
+// 0: no shared expert; 1: a complete one; -1: some of its pointers missing.
+static int shared_expert(const moe_layer_weights *w) {
+  const int n = (w->w_shared_gate != nullptr) + (w->w_shared_up != nullptr) + (w->w_shared_down != nullptr);
+  return n == 0 ? 0 : n == 3 ? 1 : -1;
 }
 
 static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
@@ -221,12 +241,20 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   if (!w || !sv) return MOE_ERR_INVALID_ARG;
   if (!ws) return MOE_ERR_WORKSPACE;
   Shape s = shape_of(cfg);
+  const int shared = shared_expert(w);
+  if (shared < 0) return MOE_ERR_INVALID_ARG;
   RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down}));
   RETURN_IF(check_ptrs4({sv->counts, sv->offsets}));
   if (route) RETURN_IF(check_ptrs4({w->w_router}));
+  if (shared) RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down}));
   if (cfg->T > 0) {
-    RETURN_IF(check_ptrs({x, y, sv->x_perm, sv->hu, sv->a, sv->y_perm}));
+    RETURN_IF(check_ptrs({x, y, sv->x_perm, sv->a, sv->y_perm}));
+    RETURN_IF(check_ptrs_or_null({sv->hu}));
     RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, sv->pair_of_slot}));
+    if (shared) {
+      RETURN_IF(check_ptrs({sv->shared_a}));
+      RETURN_IF(check_ptrs_or_null({sv->shared_hu}));
+    }
   }
   cudaStream_t st = S(stream);
   int *err = err_word(ws);
@@ -241,7 +269,14 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   RETURN_IF(cuda_rc(launch_permute(s, x, sv->slot_of_pair, sv->x_perm, st)));
   RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, sv->hu, sv->a,
                                sv->y_perm, ws, st));
-  return cuda_rc(launch_unpermute_combine(s, sv->y_perm, sv->slot_of_pair, sv->topk_gate, y, st));
+  if (shared) {
+    // the shared expert's output goes straight into y; the combine then adds to it
+    int32_t *go = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.group_offsets);
+    RETURN_IF(cuda_rc(launch_group_offsets(go, s.T, st)));
+    RETURN_IF(launch_grouped_fwd(shared_shape(s), x, go, w->w_shared_gate, w->w_shared_up, w->w_shared_down,
+                                 sv->shared_hu, sv->shared_a, y, ws, st));
+  }
+  return cuda_rc(launch_unpermute_combine(s, sv->y_perm, sv->slot_of_pair, sv->topk_gate, y, st, shared));
 }
 
 int moe_layer_fwd(const moe_config *cfg, const moe_layer_weights *w, const void *x, void *y,
@@ -263,13 +298,23 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   cudaStream_t st = S(stream);
   int *err = err_word(ws);
   const bool router = g->dw_router != nullptr;
+  const int shared = shared_expert(w);
+  if (shared < 0) return MOE_ERR_INVALID_ARG;
   RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down, g->dw_gate, g->dw_up, g->dw_down}));
   RETURN_IF(check_ptrs4({sv->offsets}));
   if (router) RETURN_IF(check_ptrs4({w->w_router, g->dw_router}));
   if (router && cfg->T > 0) RETURN_IF(check_ptrs4({sv->pair_of_slot}));
+  if (shared)
+    RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down, g->dw_shared_gate,
+                          g->dw_shared_up, g->dw_shared_down}));
   if (cfg->T > 0) {
-    RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->hu, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
+    RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
+    RETURN_IF(check_ptrs_or_null({sv->hu}));
     RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, g->dgate}));
+    if (shared) {
+      RETURN_IF(check_ptrs({sv->shared_a, g->shared_dhu}));
+      RETURN_IF(check_ptrs_or_null({sv->shared_hu}));
+    }
   }
   if (cfg->T == 0) {
     size_t wb = (size_t)s.E * s.d * s.f * s.es();
@@ -277,18 +322,46 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
     if (e == cudaSuccess) e = cudaMemsetAsync(g->dw_up, 0, wb, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(g->dw_down, 0, wb, st);
     if (e == cudaSuccess && router) e = cudaMemsetAsync(g->dw_router, 0, (size_t)s.d * s.E * 4, st);
+    const size_t sb = (size_t)s.d * s.f * s.es();
+    if (e == cudaSuccess && shared) e = cudaMemsetAsync(g->dw_shared_gate, 0, sb, st);
+    if (e == cudaSuccess && shared) e = cudaMemsetAsync(g->dw_shared_up, 0, sb, st);
+    if (e == cudaSuccess && shared) e = cudaMemsetAsync(g->dw_shared_down, 0, sb, st);
     return cuda_rc(e);
   }
   RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
                                        g->dgate, st)));
-  RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, sv->hu, sv->a, sv->offsets, w->w_gate, w->w_up,
+  // recompute: [h | u] = x_perm [Wg | Wu] into dhu, where the SwiGLU backward then runs in place
+  const void *hu = sv->hu;
+  if (!hu) {
+    RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, g->dhu, nullptr,
+                                 nullptr, ws, st));
+    hu = g->dhu;
+  }
+  RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, hu, sv->a, sv->offsets, w->w_gate, w->w_up,
                                w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st));
+  if (shared) {
+    // one group of all tokens: its dy is dY itself (weight 1) and its dx, in token order,
+    // is written to dx, to which the routed experts' rows are then added
+    const Shape s1 = shared_shape(s);
+    WsLayout L = ws_layout(s);
+    int32_t *go = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.group_offsets);
+    RETURN_IF(cuda_rc(launch_group_offsets(go, s.T, st)));
+    const void *shu = sv->shared_hu;
+    if (!shu) {
+      RETURN_IF(launch_grouped_fwd(s1, x, go, w->w_shared_gate, w->w_shared_up, w->w_shared_down, g->shared_dhu,
+                                   nullptr, nullptr, ws, st));
+      shu = g->shared_dhu;
+    }
+    RETURN_IF(launch_grouped_bwd(s1, dy, x, shu, sv->shared_a, go, w->w_shared_gate, w->w_shared_up,
+                                 w->w_shared_down, g->shared_dhu, g->dx, g->dw_shared_gate, g->dw_shared_up,
+                                 g->dw_shared_down, ws, st));
+  }
   if (!router)
     return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, nullptr, nullptr, nullptr, nullptr,
-                                        false, g->dx, st));
+                                        shared, g->dx, st));
   WsLayout L = ws_layout(s);
   char *wsc = static_cast<char *>(ws);
-  float *w_rt = reinterpret_cast<float *>(wsc + L.w_rt);
+  void *w_rt = wsc + L.w_rt;
   RETURN_IF(cuda_rc(launch_router_transpose(s, w->w_router, w_rt, st)));
   RETURN_IF(cuda_rc(launch_router_wgrad_grouped(s, sv->x_perm, sv->pair_of_slot, sv->offsets, g->dgate,
                                                 sv->topk_gate, reinterpret_cast<float *>(wsc + L.dz_slot),
@@ -296,7 +369,7 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
                                                 st)));
   // dx = sum_j dx_perm[slot(t,j)] + dz W_r^T in one pass
   return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, g->dgate, sv->topk_gate, sv->topk_idx,
-                                      w_rt, false, g->dx, st));
+                                      w_rt, shared, g->dx, st));
 }
 
 }  // extern "C"

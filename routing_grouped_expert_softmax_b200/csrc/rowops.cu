@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__res
                                                               const int32_t *__restrict__ sop,
                                                               const float *__restrict__ gate,
                                                               uint4 *__restrict__ y, int64_t Tn,
-                                                              int k, int nv) {
+                                                              int k, int nv, bool accumulate) {
   constexpr int N = Vec<T>::N;
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
@@ -72,9 +72,15 @@ __global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__res
   for (int v0 = 0; v0 < nv; v0 += 64) {
     float acc[2][N];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (accumulate && v < nv) {
+        Vec<T>::load(y[t * nv + v], acc[u]);   // y already holds the shared expert's output
+      } else {
 #pragma unroll
-      for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
+        for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
+      }
+    }
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
       if (j < k) {
@@ -121,20 +127,37 @@ __global__ void __launch_bounds__(ROW_THREADS) combine_bwd_kernel(
     g[j] = __shfl_sync(0xffffffffu, my_g, j);
     dot[j] = 0.f;
   }
-  for (int v = lane; v < nv; v += 32) {
-    float fd[N];
-    Vec<T>::load(__ldg(dy + t * nv + v), fd);
+  // two 16-byte vectors per lane per pass, so that more loads are in flight
+  for (int v0 = 0; v0 < nv; v0 += 64) {
+    float fd[2][N];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < nv) Vec<T>::load(__ldg(dy + t * nv + v), fd[u]);
+    }
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
       if (j < k) {
-        float fy[N], o[N];
-        Vec<T>::load(__ldg(y_perm + slot[j] * nv + v), fy);
+        uint4 ry[2];
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-          dot[j] = fmaf(fd[i], fy[i], dot[j]);
-          o[i] = g[j] * fd[i];
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < nv) ry[u] = __ldg(y_perm + slot[j] * nv + v);
         }
-        dy_perm[slot[j] * nv + v] = Vec<T>::store(o);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < nv) {
+            float fy[N], o[N];
+            Vec<T>::load(ry[u], fy);
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+              dot[j] = fmaf(fd[u][i], fy[i], dot[j]);
+              o[i] = g[j] * fd[u][i];
+            }
+            dy_perm[slot[j] * nv + v] = Vec<T>::store(o);
+          }
+        }
       }
     }
   }
@@ -162,13 +185,14 @@ __device__ __forceinline__ void token_dz(const float *dgate, const float *gate, 
 }
 
 // dx[t] = [dx[t]] + sum_j dx_perm[slot(t,j)] + sum_j dz_j W_r^T[e_j]
-// (dx_perm / w_rt may each be null; accumulate reads the old dx)
+// (dx_perm / w_rt may each be null; accumulate reads the old dx).  w_rt is the transposed
+// router weight [E][d] in the storage type T (an exact copy of W_r's values).
 template <typename T>
 __global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
     const uint4 *__restrict__ dx_perm, const int32_t *__restrict__ sop,
     const float *__restrict__ dgate, const float *__restrict__ gate, const int32_t *__restrict__ idx,
-    const float *__restrict__ w_rt, bool accumulate, uint4 *__restrict__ dx, int64_t Tn, int k,
-    int nv, int d) {
+    const uint4 *__restrict__ w_rt, bool accumulate, uint4 *__restrict__ dx, int64_t Tn, int k,
+    int nv) {
   constexpr int N = Vec<T>::N;
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
@@ -186,43 +210,61 @@ __global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) e[j] = (j < k) ? idx[t * k + j] : 0;
   }
-  for (int v = lane; v < nv; v += 32) {
-    float acc[N];
-    if (accumulate) {
-      Vec<T>::load(dx[t * nv + v], acc);
-    } else {
+  // two 16-byte vectors per lane per pass, so that more loads are in flight
+  for (int v0 = 0; v0 < nv; v0 += 64) {
+    float acc[2][N];
 #pragma unroll
-      for (int i = 0; i < N; ++i) acc[i] = 0.f;
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (accumulate && v < nv) {
+        Vec<T>::load(dx[t * nv + v], acc[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
+      }
     }
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
       if (j < k) {
-        if (dx_perm) {
-          float f[N];
-          Vec<T>::load(__ldg(dx_perm + slot[j] * nv + v), f);
+        uint4 rp[2], rw[2];
 #pragma unroll
-          for (int i = 0; i < N; ++i) acc[i] += f[i];
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < nv) {
+            if (dx_perm) rp[u] = __ldg(dx_perm + slot[j] * nv + v);
+            if (w_rt) rw[u] = __ldg(w_rt + (int64_t)e[j] * nv + v);
+          }
         }
-        if (w_rt) {
-          const float4 *wr = reinterpret_cast<const float4 *>(w_rt + (int64_t)e[j] * d + (int64_t)v * N);
 #pragma unroll
-          for (int i = 0; i < N / 4; ++i) {
-            float4 q = __ldg(wr + i);
-            acc[4 * i] = fmaf(dz[j], q.x, acc[4 * i]);
-            acc[4 * i + 1] = fmaf(dz[j], q.y, acc[4 * i + 1]);
-            acc[4 * i + 2] = fmaf(dz[j], q.z, acc[4 * i + 2]);
-            acc[4 * i + 3] = fmaf(dz[j], q.w, acc[4 * i + 3]);
+        for (int u = 0; u < 2; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < nv) {
+            float f[N];
+            if (dx_perm) {
+              Vec<T>::load(rp[u], f);
+#pragma unroll
+              for (int i = 0; i < N; ++i) acc[u][i] += f[i];
+            }
+            if (w_rt) {
+              Vec<T>::load(rw[u], f);
+#pragma unroll
+              for (int i = 0; i < N; ++i) acc[u][i] = fmaf(dz[j], f[i], acc[u][i]);
+            }
           }
         }
       }
     }
-    dx[t * nv + v] = Vec<T>::store(acc);
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int v = v0 + u * 32 + lane;
+      if (v < nv) dx[t * nv + v] = Vec<T>::store(acc[u]);
+    }
   }
 }
 
-// w_rt[e][i] = W_r[i][e] (fp32), 32x32 tiles through shared memory.
+// w_rt[e][i] = W_r[i][e] (same storage type), 32x32 tiles through shared memory.
 template <typename T>
-__global__ void router_transpose_kernel(const T *__restrict__ w_r, float *__restrict__ w_rt, int d,
+__global__ void router_transpose_kernel(const T *__restrict__ w_r, T *__restrict__ w_rt, int d,
                                         int E) {
   __shared__ float tile[32][33];
   int i0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
@@ -233,7 +275,7 @@ __global__ void router_transpose_kernel(const T *__restrict__ w_r, float *__rest
   __syncthreads();
   for (int r = threadIdx.y; r < 32; r += blockDim.y) {
     int e = e0 + r, i = i0 + threadIdx.x;
-    if (e < E && i < d) w_rt[(int64_t)e * d + i] = tile[threadIdx.x][r];
+    if (e < E && i < d) w_rt[(int64_t)e * d + i] = from_f<T>(tile[threadIdx.x][r]);   // exact
   }
 }
 
@@ -443,15 +485,28 @@ cudaError_t launch_permute(const Shape &s, const void *x, const int32_t *sop, vo
 }
 
 cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const int32_t *sop,
-                                     const float *gate, void *y, cudaStream_t st) {
+                                     const float *gate, void *y, cudaStream_t st, bool accumulate) {
   if (s.T == 0) return cudaSuccess;
   int nv = s.d * s.es() / 16;
   auto yp = static_cast<const uint4 *>(y_perm);
   auto yo = static_cast<uint4 *>(y);
   if (s.dtype == MOE_BF16)
-    combine_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv);
+    combine_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
   else
-    combine_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv);
+    combine_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+  return cudaGetLastError();
+}
+
+// offsets of one group holding every token: {0, T}
+__global__ void group_offsets_kernel(int32_t *o, int32_t T) {
+  if (threadIdx.x == 0) {
+    o[0] = 0;
+    o[1] = T;
+  }
+}
+
+cudaError_t launch_group_offsets(int32_t *o, int64_t T, cudaStream_t st) {
+  group_offsets_kernel<<<1, 32, 0, st>>>(o, (int32_t)T);
   return cudaGetLastError();
 }
 
@@ -471,26 +526,29 @@ cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_per
 
 cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int32_t *sop,
                                  const float *dgate, const float *gate, const int32_t *idx,
-                                 const float *w_rt, bool accumulate, void *dx, cudaStream_t st) {
+                                 const void *w_rt, bool accumulate, void *dx, cudaStream_t st) {
   if (s.T == 0) return cudaSuccess;
   int nv = s.d * s.es() / 16;
   auto a = static_cast<const uint4 *>(dx_perm);
+  auto w = static_cast<const uint4 *>(w_rt);
   auto o = static_cast<uint4 *>(dx);
   if (s.dtype == MOE_BF16)
-    unpermute_sum_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w_rt,
-                                                                      accumulate, o, s.T, s.k, nv, s.d);
+    unpermute_sum_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w,
+                                                                      accumulate, o, s.T, s.k, nv);
   else
-    unpermute_sum_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w_rt,
-                                                                       accumulate, o, s.T, s.k, nv, s.d);
+    unpermute_sum_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w,
+                                                                       accumulate, o, s.T, s.k, nv);
   return cudaGetLastError();
 }
 
-cudaError_t launch_router_transpose(const Shape &s, const void *w_r, float *w_rt, cudaStream_t st) {
+cudaError_t launch_router_transpose(const Shape &s, const void *w_r, void *w_rt, cudaStream_t st) {
   dim3 grid((s.d + 31) / 32, (s.E + 31) / 32), block(32, 8);
   if (s.dtype == MOE_BF16)
-    router_transpose_kernel<bf16><<<grid, block, 0, st>>>(static_cast<const bf16 *>(w_r), w_rt, s.d, s.E);
+    router_transpose_kernel<bf16><<<grid, block, 0, st>>>(static_cast<const bf16 *>(w_r), static_cast<bf16 *>(w_rt),
+                                                          s.d, s.E);
   else
-    router_transpose_kernel<float><<<grid, block, 0, st>>>(static_cast<const float *>(w_r), w_rt, s.d, s.E);
+    router_transpose_kernel<float><<<grid, block, 0, st>>>(static_cast<const float *>(w_r),
+                                                           static_cast<float *>(w_rt), s.d, s.E);
   return cudaGetLastError();
 }
 

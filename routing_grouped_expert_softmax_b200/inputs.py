@@ -92,6 +92,18 @@ def make_layer_inputs(T: int, d: int, E: int, k: int, f: int, dtype: str = "bf16
     return LayerInputs(T, d, E, k, f, dtype, x, w_r, w_gate, w_up, w_down, dy, bias)
 
 
+def make_shared_expert(d: int, f: int, dtype: str = "bf16", seed: int = 0,
+                       weight_std: float = 0.02):
+    """Shared-expert weights W_gate [d,f], W_up [d,f], W_down [f,d], drawn in that order from
+    N(0, weight_std^2) with their own seed; rounded to bf16 for bf16 workloads."""
+    rng = np.random.default_rng(seed)
+    ws = [(weight_std * rng.standard_normal(shape, dtype=np.float32)).astype(np.float32)
+          for shape in ((d, f), (d, f), (f, d))]
+    if dtype == "bf16":
+        ws = [bf16_round(a) for a in ws]
+    return tuple(ws)
+
+
 def uniform_random_routing(T: int, E: int, k: int, seed: int = 0):
     """Per token, k distinct experts drawn uniformly without replacement; gates 1/k.
 

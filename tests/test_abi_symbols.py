@@ -79,3 +79,15 @@ def test_empty_batch_launches_nothing(lib):
     cfg = moe.config(0, 128, 8, 2, 128)
     assert lib.moe_permute(ctypes.byref(cfg), None, None, None, None) == moe.MOE_OK
     assert lib.moe_unpermute_combine(ctypes.byref(cfg), None, None, None, None, None) == moe.MOE_OK
+
+
+def test_partial_shared_expert_rejected_on_host(lib):
+    # shared gate and up given, down missing: rejected before anything is launched
+    cfg = moe.config(16, 128, 8, 2, 128)
+    w = moe.LayerWeights(16, None, 16, 16, 16, 16, 16, None)
+    sv = moe.LayerSaved(*([16] * len(moe.SAVED_FIELDS)))
+    gr = moe.LayerGrads(*([16] * len(moe.GRAD_FIELDS)))
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_layer_bwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), ctypes.byref(gr),
+                             16, None) == moe.MOE_ERR_INVALID_ARG
