@@ -210,55 +210,31 @@ __global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) e[j] = (j < k) ? idx[t * k + j] : 0;
   }
-  // two 16-byte vectors per lane per pass, so that more loads are in flight
-  for (int v0 = 0; v0 < nv; v0 += 64) {
-    float acc[2][N];
+  for (int v = lane; v < nv; v += 32) {
+    float acc[N];
+    if (accumulate) {
+      Vec<T>::load(dx[t * nv + v], acc);
+    } else {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * 32 + lane;
-      if (accumulate && v < nv) {
-        Vec<T>::load(dx[t * nv + v], acc[u]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
-      }
+      for (int i = 0; i < N; ++i) acc[i] = 0.f;
     }
 #pragma unroll
     for (int j = 0; j < MAX_K; ++j) {
       if (j < k) {
-        uint4 rp[2], rw[2];
+        float f[N];
+        if (dx_perm) {
+          Vec<T>::load(__ldg(dx_perm + slot[j] * nv + v), f);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < nv) {
-            if (dx_perm) rp[u] = __ldg(dx_perm + slot[j] * nv + v);
-            if (w_rt) rw[u] = __ldg(w_rt + (int64_t)e[j] * nv + v);
-          }
+          for (int i = 0; i < N; ++i) acc[i] += f[i];
         }
+        if (w_rt) {
+          Vec<T>::load(__ldg(w_rt + (int64_t)e[j] * nv + v), f);
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int v = v0 + u * 32 + lane;
-          if (v < nv) {
-            float f[N];
-            if (dx_perm) {
-              Vec<T>::load(rp[u], f);
-#pragma unroll
-              for (int i = 0; i < N; ++i) acc[u][i] += f[i];
-            }
-            if (w_rt) {
-              Vec<T>::load(rw[u], f);
-#pragma unroll
-              for (int i = 0; i < N; ++i) acc[u][i] = fmaf(dz[j], f[i], acc[u][i]);
-            }
-          }
+          for (int i = 0; i < N; ++i) acc[i] = fmaf(dz[j], f[i], acc[i]);
         }
       }
     }
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int v = v0 + u * 32 + lane;
-      if (v < nv) dx[t * nv + v] = Vec<T>::store(acc[u]);
-    }
+    dx[t * nv + v] = Vec<T>::store(acc);
   }
 }
 
