@@ -625,8 +625,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tmem_cp_32x128b_x4(sfa_t, ptx::smem_desc_sf(sf_s));
             ptx::tmem_cp_32x128b_x4(sfb_t, ptx::smem_desc_sf(sf_s + 512));
           }
+          // a weight-gradient tail stage: only the UMMA_K-row slices that hold expert rows
+          int nk = C::KBLK / C::UMMA_K;
+          if constexpr (MT::WGRAD && !C::MX)
+            nk = min(nk, (tl.rows - kb * C::KBLK + C::UMMA_K - 1) / C::UMMA_K);
 #pragma unroll
           for (int kk = 0; kk < C::KBLK / C::UMMA_K; ++kk) {
+            if (kk >= nk) break;
             uint64_t adesc, bdesc;
             if constexpr (MT::A_MN)
               adesc = ptx::smem_desc_sw128(a_addr + kk * C::UMMA_K * 128, C::BOX_BYTES, 1024);
@@ -678,10 +683,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
             tpar ^= 1u << stage;
-            // In an MN-major box each K row is one 128-byte line: rows [valid, KBLK) are the
-            // byte range [valid*128, KBLK*128) of every box.
+            // In an MN-major box each K row is one 128-byte line.  The MMA issuer reads only
+            // the UMMA_K-row slices that hold expert rows, so rows [valid, round_up(valid,
+            // UMMA_K)), the byte range [valid*128, that*128) of every box, are zeroed.
             const int nbox_a = BM / C::BOX_MN, nbox_b = BNC / C::BOX_MN;
-            const int line0 = valid * 8, lines = C::KBLK * 8;  // in 16-byte units
+            const int line0 = valid * 8;                                           // 16-byte units
+            const int lines = ((valid + C::UMMA_K - 1) / C::UMMA_K) * C::UMMA_K * 8;
             const uint4 z = make_uint4(0, 0, 0, 0);
             for (int b = 0; b < nbox_a + nbox_b; ++b) {
               uint8_t *box = ring + stage * C::STAGE_BYTES +
