@@ -122,6 +122,23 @@ def dist_env():
     return ws, rank, local
 
 
+def max_over_ranks(x: float, device: str) -> float:
+    """The largest x over all ranks of the process group (x itself on one process): a
+    multi-GPU time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms: float) -> float:
+    """Whole-job throughput: the tokens all ranks processed over the slowest rank's time."""
+    return tokens_per_rank * world / (ms * 1e-3)
+
+
 def make_inputs(name, seed):
     from routing_grouped_expert_softmax_b200 import inputs as gen
     T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
@@ -203,12 +220,7 @@ def run_ours(args):
     barrier()
     clk.window(t_start, time.time())
     clk.__exit__()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms_max = ms
-    if ws_n > 1:
-        t = torch.tensor([ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_max = float(t.item())
+    ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
 
     # ---- the grouped GEMMs alone (6 tcgen05 launches per step), same stream and inputs
     g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
@@ -276,11 +288,7 @@ def run_ours(args):
     st.wait_stream(s_out)
     e1.record(st)
     barrier()
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if ws_n > 1:
-        t = torch.tensor([e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
     assert moe.moe_get_error(ws) == 0
 
     P = T * k
@@ -304,7 +312,7 @@ def run_ours(args):
     traffic = tr["bytes"] if tr and tr["sources_sha1"] == gemm_sources_sha1() else None
     out = {
         "metric": "MoE-layer tokens/s (E=128,k=4,bf16 fwd+bwd) 1xB200; grouped-GEMM % TC peak",
-        "value": T * ws_n / (ms_max * 1e-3),
+        "value": job_tokens_per_s(T, ws_n, ms_max),
         "unit": "tokens/s",
         "n_gpus": ws_n,
         "steps": args.steps,
@@ -338,7 +346,7 @@ def run_ours(args):
                      "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                      "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
                      "bwd_tflops": flops_bwd / (bwd_ms * 1e-3) / 1e12},
-        "e2e": {"value": T * ws_n / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": job_tokens_per_s(T, ws_n, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": 2 * T * d * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
@@ -438,14 +446,19 @@ def run_reference(args):
     T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
     inp = make_inputs(name, seed=0)
     from oracle import moe_ref as ref
-    # size each step's token sample so that the K timed steps take about two minutes
+    # size each step's token sample so that the W warm-up and K timed steps take about two
+    # minutes together
     probe = 16
     t0 = time.perf_counter()
     fwd = ref.layer_fwd(inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
     ref.layer_bwd(fwd, inp.dy[:probe], inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
     t_probe = time.perf_counter() - t0
-    n = int(max(4, min(args.cpu_tokens, probe * (120.0 / max(args.steps, 1)) / max(t_probe, 1e-3))))
+    n_steps = max(args.steps + args.warmup, 1)
+    n = int(max(4, min(args.cpu_tokens, probe * (120.0 / n_steps) / max(t_probe, 1e-3))))
     xs, dys = inp.x[:n], inp.dy[:n]
+    for _ in range(args.warmup):
+        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+        ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
     times = []
     for _ in range(args.steps):
         t0 = time.perf_counter()
