@@ -190,7 +190,8 @@ MOE_API int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, c
  *   written into buffers padded to 128 rows per expert; padded row 128*pre[e] + i holds
  *   src row offsets[e] + i for i < count_e and zeros after, pre[e] = sum_{e'<e}
  *   ceil(count_e'/128); the buffers must hold rows_bound >= rows + 127*E rows.
- * cols must be a multiple of 32 (of 128 for the rows variant with offsets). */
+ * cols must be a multiple of 32 (of 128 for the rows variant with offsets).  src and codes
+ * 16-byte aligned, scales 4-byte aligned (else MOE_ERR_INVALID_ARG). */
 MOE_API int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int32_t *offsets,
                                  int32_t E, int64_t rows_bound, uint8_t *codes, uint8_t *scales,
                                  moe_stream_t stream);

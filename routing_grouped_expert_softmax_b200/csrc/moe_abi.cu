@@ -166,7 +166,8 @@ int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, const int3
   if (rows < 0 || cols <= 0 || cols % 32 || (offsets && (E <= 0 || E > MAX_E))) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
   if (offsets && rows_bound < rows + 127 * (int64_t)E) return MOE_ERR_INVALID_ARG;
-  if (!src || !codes || !scales) return MOE_ERR_INVALID_ARG;
+  RETURN_IF(check_ptrs({src, codes}));
+  RETURN_IF(check_ptrs4({scales}));
   return cuda_rc(launch_mx_quant_cols(src, rows, cols, offsets, E, offsets ? rows_bound : rows, codes, scales,
                                       S(stream)));
 }

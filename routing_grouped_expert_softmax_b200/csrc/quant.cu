@@ -125,7 +125,43 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16 *__restri
   }
 }
 
-// ---- cols: one thread per (column, 32-row block).
+// Four adjacent columns of a 32-row block: reads 8 bytes of every row (one warp reads 256
+// contiguous bytes per row) once for the block maxima and again (from cache) to quantise,
+// and stores 4 code bytes per row and the 4 scale bytes.
+__device__ __forceinline__ uint2 mx_row8(const bf16 *src, int64_t ld_src, int i, int nvalid) {
+  return i < nvalid ? __ldg(reinterpret_cast<const uint2 *>(src + i * ld_src)) : make_uint2(0u, 0u);
+}
+__device__ __forceinline__ void mx_cols4(const bf16 *src, int64_t ld_src, int nvalid, uint8_t *codes,
+                                         int64_t ld_codes, uint8_t *scales) {
+  float amax[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint2 r = mx_row8(src, ld_src, i, nvalid);
+    amax[0] = fmaxf(amax[0], fabsf(__uint_as_float(r.x << 16)));
+    amax[1] = fmaxf(amax[1], fabsf(__uint_as_float(r.x & 0xFFFF0000u)));
+    amax[2] = fmaxf(amax[2], fabsf(__uint_as_float(r.y << 16)));
+    amax[3] = fmaxf(amax[3], fabsf(__uint_as_float(r.y & 0xFFFF0000u)));
+  }
+  int sc[4];
+  float inv[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    sc[j] = mx_scale_exp(amax[j]);
+    inv[j] = exp2_neg(sc[j]);
+  }
+#pragma unroll 8
+  for (int i = 0; i < 32; ++i) {
+    const uint2 r = mx_row8(src, ld_src, i, nvalid);
+    const uint32_t w =
+        (uint32_t)e4m3x2(__uint_as_float(r.x << 16) * inv[0], __uint_as_float(r.x & 0xFFFF0000u) * inv[1]) |
+        ((uint32_t)e4m3x2(__uint_as_float(r.y << 16) * inv[2], __uint_as_float(r.y & 0xFFFF0000u) * inv[3]) << 16);
+    *reinterpret_cast<uint32_t *>(codes + i * ld_codes) = w;
+  }
+  *reinterpret_cast<uint32_t *>(scales) = (uint32_t)(sc[0] + 127) | ((uint32_t)(sc[1] + 127) << 8) |
+                                          ((uint32_t)(sc[2] + 127) << 16) | ((uint32_t)(sc[3] + 127) << 24);
+}
+
+// ---- cols: one thread per (4 adjacent columns, 32-row block).  C % 4 == 0.
 __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restrict__ src, int64_t R, int C,
                                                             const int32_t *__restrict__ offsets, int E,
                                                             uint8_t *__restrict__ codes,
@@ -135,7 +171,7 @@ __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restri
     if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
     __syncthreads();
   }
-  const int c = blockIdx.x * 256 + threadIdx.x;
+  const int c = 4 * (blockIdx.x * 256 + threadIdx.x);
   const int64_t rb = blockIdx.y;                       // 32-row block
   const int64_t rows_out = offsets ? (int64_t)pre[E] * 128 : R;
   if (rb * 32 >= rows_out || c >= C) return;
@@ -154,53 +190,26 @@ __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restri
       nvalid = (int)(left < 32 ? left : 32);
     }
   }
-  float v[32];
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    v[i] = (i < nvalid) ? __bfloat162float(src[(sr0 + i) * C + c]) : 0.f;
-    amax = fmaxf(amax, fabsf(v[i]));
-  }
-  const int s = mx_scale_exp(amax);
-  const float inv = exp2_neg(s);
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    uint16_t q = e4m3x2(v[i] * inv, v[i + 1] * inv);
-    codes[(rb * 32 + i) * C + c] = (uint8_t)(q & 0xFF);
-    codes[(rb * 32 + i + 1) * C + c] = (uint8_t)(q >> 8);
-  }
-  scales[rb * C + c] = (uint8_t)(s + 127);
+  if (sr0 < 0) sr0 = 0;   // nothing is read from it then
+  mx_cols4(src + sr0 * C + c, C, nvalid, codes + rb * 32 * C + c, C, scales + rb * C + c);
 }
 
 // ---- weights of the gate/up GEMM, blocked down the rows, with gate and up columns
 // interleaved in 64-column chunks: output column 128*j + i is gate column 64*j + i for
-// i < 64 and up column 64*j + (i - 64) otherwise.  src: W_gate, W_up [R][f].
+// i < 64 and up column 64*j + (i - 64) otherwise.  src: W_gate, W_up [R][f].  One thread per
+// 4 adjacent output columns (never split across a 64-column chunk) and 32-row block.
 __global__ void __launch_bounds__(256) mx_quant_cols_gu_kernel(const bf16 *__restrict__ wg,
                                                                const bf16 *__restrict__ wu, int64_t R, int f,
                                                                uint8_t *__restrict__ codes,
                                                                uint8_t *__restrict__ scales) {
-  const int oc = blockIdx.x * 256 + threadIdx.x;      // output column in [0, 2f)
+  const int oc = 4 * (blockIdx.x * 256 + threadIdx.x);   // output column in [0, 2f)
   const int64_t rb = blockIdx.y;
   if (oc >= 2 * f || rb * 32 >= R) return;
   const int j = oc >> 7, i = oc & 127;
   const bf16 *src = i < 64 ? wg : wu;
   const int c = 64 * j + (i & 63);
-  float v[32];
-  float amax = 0.f;
-#pragma unroll
-  for (int r = 0; r < 32; ++r) {
-    v[r] = __bfloat162float(src[(rb * 32 + r) * f + c]);
-    amax = fmaxf(amax, fabsf(v[r]));
-  }
-  const int s = mx_scale_exp(amax);
-  const float inv = exp2_neg(s);
-#pragma unroll
-  for (int r = 0; r < 32; r += 2) {
-    uint16_t q = e4m3x2(v[r] * inv, v[r + 1] * inv);
-    codes[(rb * 32 + r) * (2 * f) + oc] = (uint8_t)(q & 0xFF);
-    codes[(rb * 32 + r + 1) * (2 * f) + oc] = (uint8_t)(q >> 8);
-  }
-  scales[rb * (2 * f) + oc] = (uint8_t)(s + 127);
+  const int nvalid = (int)(R - rb * 32 < 32 ? R - rb * 32 : 32);
+  mx_cols4(src + rb * 32 * f + c, f, nvalid, codes + rb * 32 * (2 * f) + oc, 2 * f, scales + rb * (2 * f) + oc);
 }
 
 // ---- weights of the gate/up data-gradient GEMM, blocked along the rows of [W_gate | W_up]
@@ -249,14 +258,14 @@ cudaError_t launch_mx_quant_rows(const void *src, int64_t R, int K, const int32_
 cudaError_t launch_mx_quant_cols(const void *src, int64_t R, int C, const int32_t *offsets, int E, int64_t rows_bound,
                                  uint8_t *codes, uint8_t *scales, cudaStream_t st) {
   if (rows_bound <= 0) return cudaSuccess;
-  dim3 grid((unsigned)((C + 255) / 256), (unsigned)((rows_bound + 31) / 32));
+  dim3 grid((unsigned)((C / 4 + 255) / 256), (unsigned)((rows_bound + 31) / 32));
   mx_quant_cols_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(src), R, C, offsets, E, codes, scales);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_cols_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
                                     uint8_t *scales, cudaStream_t st) {
-  dim3 grid((unsigned)((2 * f + 255) / 256), (unsigned)((R + 31) / 32));
+  dim3 grid((unsigned)((2 * f / 4 + 255) / 256), (unsigned)((R + 31) / 32));
   mx_quant_cols_gu_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(wg), static_cast<const bf16 *>(wu), R, f,
                                                 codes, scales);
   return cudaGetLastError();
