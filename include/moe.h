@@ -192,6 +192,19 @@ MOE_API int moe_grouped_swiglu_bwd(const moe_config *cfg, const void *dy_perm, c
  *   ceil(count_e'/128); the buffers must hold rows_bound >= rows + 127*E rows.
  * cols must be a multiple of 32 (of 128 for the rows variant with offsets).  src and codes
  * 16-byte aligned, scales 4-byte aligned (else MOE_ERR_INVALID_ARG). */
+/* FP8 dispatch (unite.ai, "Ai2 κυκλοφορεί το Olmo-Core 3 ...", section "Παραλληλισμός,
+ * Ακρίβεια και Τεχνικές Μνήμης": MXFP8 also for the data moved between experts): the
+ * permute of moe_permute (x_perm [P,d] bf16, a bit copy of each routed row) and, in the same
+ * pass, each routed row in MXFP8 with blocks of 32 along d, written as moe_mx_quantize_rows
+ * with offsets writes it: codes [rows_bound][d] and scales [rows_bound][d/32], padded row
+ * 128*pre[e] + (slot - offsets[e]).  Rows of the padding past an expert's count are left
+ * as they were.  bf16 only (else MOE_ERR_UNSUPPORTED); rows_bound >= T*k + 127*E; x, x_perm,
+ * codes 16-byte aligned, slot_of_pair, offsets, scales 4-byte aligned.  offsets from
+ * moe_build_offsets. */
+MOE_API int moe_permute_mxfp8(const moe_config *cfg, const void *x, const int32_t *slot_of_pair,
+                              const int32_t *offsets, void *x_perm, int64_t rows_bound,
+                              uint8_t *codes, uint8_t *scales, moe_stream_t stream);
+
 MOE_API int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int32_t *offsets,
                                  int32_t E, int64_t rows_bound, uint8_t *codes, uint8_t *scales,
                                  moe_stream_t stream);

@@ -36,7 +36,7 @@ EXPORTED = [
     "moe_build_offsets", "moe_build_offsets_noalloc", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
     "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd", "moe_mx_quantize_rows",
-    "moe_mx_quantize_cols",
+    "moe_mx_quantize_cols", "moe_permute_mxfp8",
 ]
 
 
@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
                                                     ctypes.c_int64, _P, _P, _P]),
             "moe_mx_quantize_cols": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, ctypes.c_int32,
                                                     ctypes.c_int64, _P, _P, _P]),
+            "moe_permute_mxfp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_int64, _P, _P, _P]),
             "moe_layer_fwd": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
                                              ctypes.POINTER(LayerSaved), _P, _P]),
             "moe_layer_fwd_routed": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
@@ -226,6 +227,11 @@ def moe_route_bwd(cfg, dgate, topk_gate, topk_idx, x, w_router, dx, dw_router, w
 def moe_mx_quantize_rows(src, rows, cols, offsets, E, rows_bound, codes, scales, stream=None):
     _call("moe_mx_quantize_rows", ptr(src), rows, cols, ptr(offsets), E, rows_bound, ptr(codes),
           ptr(scales), stream_handle(stream))
+
+
+def moe_permute_mxfp8(cfg, x, slot_of_pair, offsets, x_perm, rows_bound, codes, scales, stream=None):
+    _call("moe_permute_mxfp8", ctypes.byref(cfg), ptr(x), ptr(slot_of_pair), ptr(offsets), ptr(x_perm),
+          rows_bound, ptr(codes), ptr(scales), stream_handle(stream))
 
 
 def moe_mx_quantize_cols(src, rows, cols, offsets, E, rows_bound, codes, scales, stream=None):

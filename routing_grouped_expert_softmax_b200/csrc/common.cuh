@@ -154,6 +154,10 @@ cudaError_t launch_permute(const Shape &s, const void *x, const int32_t *slot_of
 cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const int32_t *sop,
                                      const float *gate, void *y, cudaStream_t st, bool accumulate = false);
 cudaError_t launch_group_offsets(int32_t *o, int64_t T, cudaStream_t st);
+// FP8 dispatch: the permute that also writes each routed row in MXFP8 (blocks of 32 along d)
+// into the expert buffers padded to 128 rows (bf16 storage, d % 32 == 0)
+cudaError_t launch_mx_permute(const void *x, const int32_t *sop, const int32_t *offsets, int E, int64_t T, int k,
+                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st);
 cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm,
                                const int32_t *sop, const float *gate, void *dy_perm,
                                float *dgate, cudaStream_t st);
@@ -169,9 +173,11 @@ cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, cons
 cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
                                 const int32_t *idx, const void *x, float *partial,
                                 float *dw_r, cudaStream_t st);
+// x_quantized (MXFP8 only): the workspace already holds x_perm's MXFP8 rows, written by
+// launch_mx_permute into the layout ws_layout(s) gives them.
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets,
                        const void *w_gate, const void *w_up, const void *w_down, void *hu,
-                       void *a, void *y_perm, void *ws, cudaStream_t st);
+                       void *a, void *y_perm, void *ws, cudaStream_t st, bool x_quantized = false);
 // dst[b][c][r] = src[b][r][c] (fp32)
 cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st);
 // MXFP8 quantisers (quant.cu).  offsets != nullptr: source rows are expert groups written

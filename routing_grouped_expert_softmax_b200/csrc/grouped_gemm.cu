@@ -1345,12 +1345,13 @@ static MxOp mx_r(void *ws, size_t off, int64_t rows, int64_t cols) {
 // Forward with both operands of both GEMMs quantised to MXFP8 (blocks along K).
 static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
-                       cudaStream_t st) {
+                       cudaStream_t st, bool x_quantized) {
   const WsLayout L = ws_layout(s);
   const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
   const MxOp xq = mx_r(ws, L.xq_r, R, s.d), aq = mx_r(ws, L.aq_r, R, s.f);
   const MxOp wgu = mx_r(ws, L.wgu_c, ed, 2 * s.f), wd = mx_r(ws, L.wd_c, ef, s.d);
-  if (launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st) ||
+  // x_quantized: the FP8 dispatch (launch_mx_permute) already wrote xq's rows
+  if ((!x_quantized && launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st)) ||
       launch_mx_quant_cols_gu(w_gate, w_up, ed, s.f, wgu.codes, wgu.scales, st) ||
       (y_perm && launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st)))
     return MOE_ERR_CUDA;
@@ -1445,9 +1446,9 @@ int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float
 
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
-                       cudaStream_t st) {
+                       cudaStream_t st, bool x_quantized) {
   if (s.prec == MOE_PREC_MXFP8)
-    return gg::mx_fwd_impl(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
+    return gg::mx_fwd_impl(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st, x_quantized);
   if (s.dtype == MOE_BF16)
     return gg::fwd_impl<bf16>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
   return gg::fwd_impl<float>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);

@@ -161,6 +161,18 @@ int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int3
                                       S(stream)));
 }
 
+int moe_permute_mxfp8(const moe_config *cfg, const void *x, const int32_t *slot_of_pair, const int32_t *offsets,
+                      void *x_perm, int64_t rows_bound, uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  const Shape s = shape_of(cfg);
+  if (rows_bound < s.Ppad()) return MOE_ERR_INVALID_ARG;
+  RETURN_IF(check_ptrs({x, x_perm, codes}));
+  RETURN_IF(check_ptrs4({slot_of_pair, offsets, scales}));
+  return cuda_rc(launch_mx_permute(x, slot_of_pair, offsets, s.E, s.T, s.k, s.d, x_perm, codes, scales, S(stream)));
+}
+
 int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, const int32_t *offsets, int32_t E,
                          int64_t rows_bound, uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
   if (rows < 0 || cols <= 0 || cols % 32 || (offsets && (E <= 0 || E > MAX_E))) return MOE_ERR_INVALID_ARG;
@@ -267,9 +279,17 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   RETURN_IF(cuda_rc(launch_build_offsets(s, sv->topk_idx, sv->counts, sv->offsets, sv->slot_of_pair,
                                          sv->pair_of_slot, bc, err, st)));
   if (cfg->T == 0) return MOE_OK;
-  RETURN_IF(cuda_rc(launch_permute(s, x, sv->slot_of_pair, sv->x_perm, st)));
+  const bool mx = s.prec == MOE_PREC_MXFP8;
+  if (mx) {
+    // FP8 dispatch: the permute also writes x_perm's MXFP8 rows where the forward GEMM reads them
+    uint8_t *xq = static_cast<uint8_t *>(ws) + L.xq_r;
+    RETURN_IF(cuda_rc(launch_mx_permute(x, sv->slot_of_pair, sv->offsets, s.E, s.T, s.k, s.d, sv->x_perm, xq,
+                                        xq + s.Ppad() * s.d, st)));
+  } else {
+    RETURN_IF(cuda_rc(launch_permute(s, x, sv->slot_of_pair, sv->x_perm, st)));
+  }
   RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, sv->hu, sv->a,
-                               sv->y_perm, ws, st));
+                               sv->y_perm, ws, st, mx));
   if (shared) {
     // the shared expert's output goes straight into y; the combine then adds to it
     int32_t *go = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.group_offsets);

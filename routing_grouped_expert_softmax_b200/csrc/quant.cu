@@ -247,6 +247,80 @@ __global__ void __launch_bounds__(256) mx_quant_rows_gu_kernel(const bf16 *__res
   }
 }
 
+// ---- FP8 dispatch: x_perm[slot(t,j)] = x[t] (a bit copy) and, in the same pass, the row in
+// MXFP8 (blocks of 32 along d) at padded row 128*pre[e] + (slot - offsets[e]) of the expert
+// buffers, e the expert holding the slot.  One warp per token; lane l quantises the 32-column
+// blocks l, l+32, ... once and writes them to all k destinations.  Padded rows past an
+// expert's count are not written (the gate/up GEMM computes and drops them).
+__global__ void __launch_bounds__(256) mx_permute_kernel(const bf16 *__restrict__ x, const int32_t *__restrict__ sop,
+                                                         const int32_t *__restrict__ offsets, int E, int64_t T,
+                                                         int k, int d, bf16 *__restrict__ x_perm,
+                                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales) {
+  __shared__ int pre[MAX_E + 1];
+  if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (t >= T) return;
+  int64_t my_slot = 0, my_prow = 0;
+  if (lane < k) {
+    my_slot = sop[t * k + lane];
+    int lo = 0, hi = E;   // the expert whose range holds the slot: offsets[lo] <= slot < offsets[lo + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (offsets[mid] <= my_slot) lo = mid; else hi = mid;
+    }
+    my_prow = (int64_t)pre[lo] * 128 + (my_slot - offsets[lo]);
+  }
+  int64_t slot[MAX_K], prow[MAX_K];
+#pragma unroll
+  for (int j = 0; j < MAX_K; ++j) {
+    slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    prow[j] = __shfl_sync(0xffffffffu, my_prow, j);
+  }
+  for (int c0 = 0; c0 < d; c0 += 1024) {
+    const int col = c0 + lane * 32;
+    if (col >= d) break;
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(x + t * d + col);
+    uint4 raw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) raw[i] = __ldg(s4 + i);
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) Vec<bf16>::load(raw[i], &v[8 * i]);
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    const int sc = mx_scale_exp(amax);
+    const float inv = exp2_neg(sc);
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      w[i] = (uint32_t)e4m3x2(v[4 * i] * inv, v[4 * i + 1] * inv) |
+             ((uint32_t)e4m3x2(v[4 * i + 2] * inv, v[4 * i + 3] * inv) << 16);
+#pragma unroll
+    for (int j = 0; j < MAX_K; ++j) {
+      if (j < k) {
+        uint4 *xp = reinterpret_cast<uint4 *>(x_perm + slot[j] * d + col);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xp[i] = raw[i];
+        uint4 *d4 = reinterpret_cast<uint4 *>(codes + prow[j] * d + col);
+        d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        scales[prow[j] * (d / 32) + col / 32] = (uint8_t)(sc + 127);
+      }
+    }
+  }
+}
+
+cudaError_t launch_mx_permute(const void *x, const int32_t *sop, const int32_t *offsets, int E, int64_t T, int k,
+                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  mx_permute_kernel<<<(unsigned)((T + 7) / 8), 256, 0, st>>>(static_cast<const bf16 *>(x), sop, offsets, E, T, k, d,
+                                                             static_cast<bf16 *>(x_perm), codes, scales);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mx_quant_rows(const void *src, int64_t R, int K, const int32_t *offsets, int E, int64_t rows_bound,
                                  uint8_t *codes, uint8_t *scales, cudaStream_t st) {
   if (rows_bound <= 0) return cudaSuccess;

@@ -105,6 +105,37 @@ def test_mx_quantize_expert_padded(E, cols):
     assert np.array_equal(host(ct)[:n], tc) and np.array_equal(host(st)[:n // 32], ts)
 
 
+@pytest.mark.parametrize("T,d,E,k", [(300, 256, 8, 2), (1000, 2048, 128, 4), (77, 128, 5, 3),
+                                     (513, 1024, 16, 8)])
+def test_permute_mxfp8_is_the_permute_and_the_row_quantiser(T, d, E, k):
+    """FP8 dispatch: x_perm bit for bit as the oracle's permute, and every routed row's
+    codes and scales bit for bit as the oracle's OCP MX rule on the expert-padded layout;
+    the padding rows past each expert's count are left untouched."""
+    import torch
+    idx, _ = gen.uniform_random_routing(T, E, k, seed=T)
+    counts, offsets, sop, pos = ref.routing_metadata(idx, E)
+    x = _special_data(T, d, T)
+    cfg = moe.config(T, d, E, k, 128)
+    bound = T * k + 127 * E
+    xp = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    codes = torch.full((bound, d), 0xAB, dtype=torch.uint8, device="cuda")
+    scales = torch.full((bound, d // 32), 0xAB, dtype=torch.uint8, device="cuda")
+    moe.moe_permute_mxfp8(cfg, dev(x, "bf16"), dev_i32(sop), dev_i32(offsets), xp, bound, codes, scales)
+    xpr = ref.permute(x, pos, k)
+    assert np.array_equal(host(xp), xpr)
+    pv = _padded(xpr, offsets)
+    rc, rs, _ = ref.mx_quantize(pv, axis=1)
+    pre = np.concatenate([[0], np.cumsum((np.diff(offsets) + 127) // 128)])
+    valid = np.zeros(bound, bool)
+    for e in range(E):
+        valid[pre[e] * 128: pre[e] * 128 + int(offsets[e + 1] - offsets[e])] = True
+    hc, hs = host(codes), host(scales)
+    n = pv.shape[0]
+    assert np.array_equal(hc[:n][valid[:n]], rc[valid[:n]])
+    assert np.array_equal(hs[:n][valid[:n]], rs[valid[:n]])
+    assert np.all(hc[~valid] == 0xAB) and np.all(hs[~valid] == 0xAB)
+
+
 # ------------------------------------------------------------------ grouped GEMMs
 
 MX_CASES = [
