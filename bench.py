@@ -298,7 +298,7 @@ def run_ours(args):
     gemm_ms = fwd_ms + bwd_ms
     tflops = (flops_fwd + flops_bwd) / (gemm_ms * 1e-3) / 1e12
     # The GEMMs are timed back to back for `steps` iterations (a long, power-capped loop), so
-    # the tensor roof is the sustained bf16 figure.  An MXFP8 contraction is judged against
+    # the tensor roof is the sustained bf16 figure.  An MXFP8 contraction is measured against
     # the fp8 peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25).
     bf16_peak = pk["bf16_sus"] or pk["bf16"]
     peak_tc = bf16_peak * (2.0 if prec == "mxfp8" else 1.0)

@@ -23,7 +23,7 @@ pytestmark = pytest.mark.gpu
 TOL = 2e-2
 TOL_COMBINE = 1e-2
 
-CONFIGS = {
+FULL_SIZE_CASES = {
     "e8": dict(T=8192, d=2048, E=8, k=4, f=1024, skew=False, routing="router"),
     "e128": dict(T=8192, d=2048, E=128, k=4, f=1024, skew=False, routing="router"),
     "e128_t16k_skew": dict(T=16384, d=2048, E=128, k=4, f=1024, skew=True, routing="router"),
@@ -127,10 +127,10 @@ def _expert_oracle(inp, e, idx, gate, mx=None):
     return dwgu[:, :f], dwgu[:, f:], qt(a).T @ qt(dy)
 
 
-@pytest.mark.parametrize("name", list(CONFIGS))
+@pytest.mark.parametrize("name", list(FULL_SIZE_CASES))
 def test_fullsize(name):
     import torch
-    c = CONFIGS[name]
+    c = FULL_SIZE_CASES[name]
     T, d, E, k, f = c["T"], c["d"], c["E"], c["k"], c["f"]
     inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=0, skew=c["skew"])
     prec = c.get("prec", "native")
