@@ -91,3 +91,46 @@ def test_partial_shared_expert_rejected_on_host(lib):
         == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_layer_bwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), ctypes.byref(gr),
                              16, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_permute_mxfp8_host_validation(lib):
+    cfg = moe.config(16, 128, 8, 2, 128)
+    bound = 16 * 2 + 127 * 8
+    ok = (ctypes.byref(cfg), 16, 16, 16, 16, bound, 16, 16, None)
+    # fp32 storage has no MXFP8 path
+    c32 = moe.config(16, 128, 8, 2, 128, dtype="f32")
+    assert lib.moe_permute_mxfp8(ctypes.byref(c32), *ok[1:]) == moe.MOE_ERR_UNSUPPORTED
+    # the padded buffers must hold T*k + 127*E rows
+    assert lib.moe_permute_mxfp8(ctypes.byref(cfg), 16, 16, 16, 16, bound - 1, 16, 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    # x, x_perm and codes move as 16-byte vectors
+    assert lib.moe_permute_mxfp8(ctypes.byref(cfg), 24, 16, 16, 16, bound, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_mxfp8(ctypes.byref(cfg), 16, 16, 16, 16, bound, 8, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_permute_mxfp8(ctypes.byref(cfg), 16, 16, None, 16, bound, 16, 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    # an empty batch launches nothing
+    c0 = moe.config(0, 128, 8, 2, 128)
+    assert lib.moe_permute_mxfp8(ctypes.byref(c0), None, None, None, None, 0, None, None, None) == moe.MOE_OK
+
+
+def test_mx_quantize_cols_alignment(lib):
+    assert lib.moe_mx_quantize_cols(24, 64, 64, None, 0, 64, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_mx_quantize_cols(16, 64, 64, None, 0, 64, 16, 6, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_mx_quantize_cols(16, 64, 48, None, 0, 64, 16, 16, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_shared_expert_and_recompute_host_validation(lib):
+    cfg = moe.config(16, 128, 8, 2, 128)
+    w = moe.LayerWeights(16, None, 16, 16, 16, 16, 16, 16)      # a complete shared expert
+    fields = {n: 16 for n in moe.SAVED_FIELDS}
+    fields["shared_a"] = None                                     # ... but no room for its a
+    sv = moe.LayerSaved(*[fields[n] for n in moe.SAVED_FIELDS])
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    # recompute: hu may be NULL but, when given, must be 16-byte aligned
+    fields = {n: 16 for n in moe.SAVED_FIELDS}
+    fields["hu"] = 24
+    sv = moe.LayerSaved(*[fields[n] for n in moe.SAVED_FIELDS])
+    w0 = moe.LayerWeights(16, None, 16, 16, 16, None, None, None)
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(w0), 16, 16, ctypes.byref(sv), 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
