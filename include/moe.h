@@ -89,19 +89,22 @@ typedef struct moe_config {
   int32_t prec;  /* enum moe_prec */
 } moe_config;
 
-/* Bytes of device workspace every call taking `ws` needs for this config.
+/* (the pages have no counterpart: calling-convention plumbing)
+ * Bytes of device workspace every call taking `ws` needs for this config.
  * The workspace holds the error word and small scratch (per-block histograms,
  * a transposed router weight, router-gradient partial sums).  Zero it once
  * (cudaMemset) before its first use; the library keeps it consistent after. */
 MOE_API size_t moe_workspace_size(const moe_config *cfg);
 
-/* Synchronise `stream`, then report and clear the device error word in `ws`.
+/* (the pages have no counterpart: error reporting)
+ * Synchronise `stream`, then report and clear the device error word in `ws`.
  * *code receives 0 or an OR of MOE_ERR_DEVICE_* bits. */
 MOE_API int moe_get_error(void *ws, moe_stream_t stream, int32_t *code);
 
 /* ---------------------------------------------------------------- routing */
 
-/* Router forward.  logits z = x W_r (+ bias) in fp32; top-k on z, listed by
+/* Router forward (source: qidao123.com, section "新闻原文", 4 of E experts per token; unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης").
+ * logits z = x W_r (+ bias) in fp32; top-k on z, listed by
  * descending logit with equal logits to the lower index; gates
  * g_j = exp(z_j) / sum_j' exp(z_j') over the k selected logits (equal to the
  * full softmax renormalised over the selection).
@@ -112,12 +115,15 @@ MOE_API int moe_route_topk(const moe_config *cfg, const void *x, const void *w_r
                    const float *bias, float *logits, int32_t *topk_idx,
                    float *topk_gate, void *ws, moe_stream_t stream);
 
-/* The router's second half alone: top-k and renormalised gates from given
+/* (source: as moe_route_topk)
+ * The router's second half alone: top-k and renormalised gates from given
  * fp32 logits [T,E].  Same selection and gate rule as moe_route_topk. */
 MOE_API int moe_topk_gating(const moe_config *cfg, const float *logits, int32_t *topk_idx,
                     float *topk_gate, void *ws, moe_stream_t stream);
 
-/* GPU-resident routing metadata (stable counting sort of the P pairs by expert):
+/* (source: unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης" and ettayeb.fr, section "Trois parallélismes, trois optimisations de routage": the routing metadata stays on the GPU so the CPU
+ * never waits for a copy back)
+ * GPU-resident routing metadata (stable counting sort of the P pairs by expert):
  *   counts[e] = pairs routed to e; offsets[0..E] = exclusive scan of counts
  *   (offsets[E] = P); slot_of_pair[i] = offsets[e] + number of pairs i' < i
  *   with the same expert; pair_of_slot = its inverse.
@@ -145,14 +151,19 @@ MOE_API int moe_build_offsets_noalloc(const moe_config *cfg, const int32_t *topk
                                       int32_t *counts, int32_t *offsets, int32_t *slot_of_pair,
                                       int32_t *pair_of_slot, moe_stream_t stream);
 
-/* Rowwise dispatch: x_perm[slot_of_pair[t*k+j]] = x[t] (a bit copy).
+/* (source: unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης", and ettayeb.fr,
+ * section "Trois parallélismes, trois optimisations de routage": routed rows are written
+ * straight into the experts' input buffers, "rowwise" placement)
+ * Rowwise dispatch: x_perm[slot_of_pair[t*k+j]] = x[t] (a bit copy).
  *   x [T,d] dtype; slot_of_pair [P]; x_perm [P,d] dtype. */
 MOE_API int moe_permute(const moe_config *cfg, const void *x, const int32_t *slot_of_pair,
                 void *x_perm, moe_stream_t stream);
 
 /* ------------------------------------------------------ grouped expert FFN */
 
-/* Grouped SwiGLU forward over the expert-contiguous rows of x_perm.  For each
+/* (source: unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης": one grouped GEMM runs the experts' small matmuls, scheduled from
+ * the device)
+ * Grouped SwiGLU forward over the expert-contiguous rows of x_perm.  For each
  * expert e and its rows R_e = [offsets[e], offsets[e+1]):
  *   h = x_perm[R_e] Wg[e], u = x_perm[R_e] Wu[e], a = silu(h) * u,
  *   y_perm[R_e] = a Wd[e].
@@ -165,7 +176,8 @@ MOE_API int moe_grouped_swiglu_fwd(const moe_config *cfg, const void *x_perm, co
                            const void *w_gate, const void *w_up, const void *w_down,
                            void *hu, void *a, void *y_perm, void *ws, moe_stream_t stream);
 
-/* Grouped SwiGLU backward.  Per expert e (rows R_e):
+/* (source: as moe_grouped_swiglu_fwd; the backward is its chain rule)
+ * Grouped SwiGLU backward.  Per expert e (rows R_e):
  *   da = dy_perm Wd^T; dh = da * u * silu'(h); du = da * silu(h);
  *   dhu = [dh | du] ([P,2f], written); dx_perm = dh Wg^T + du Wu^T;
  *   dWd[e] = a^T dy_perm; dWg[e] = x_perm^T dh; dWu[e] = x_perm^T du.
@@ -214,25 +226,29 @@ MOE_API int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, co
 
 /* ---------------------------------------------------------------- combine */
 
-/* Gate-weighted unpermute: y[t] = sum_j topk_gate[t,j] * y_perm[slot_of_pair[t*k+j]],
+/* (source: unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης": the inverse of the rowwise placement, weighted by the gates)
+ * Gate-weighted unpermute: y[t] = sum_j topk_gate[t,j] * y_perm[slot_of_pair[t*k+j]],
  * accumulated in fp32.  y_perm [P,d]; y [T,d] dtype. */
 MOE_API int moe_unpermute_combine(const moe_config *cfg, const void *y_perm,
                           const int32_t *slot_of_pair, const float *topk_gate, void *y,
                           moe_stream_t stream);
 
-/* Backward of the combine: dy_perm[slot(t,j)] = g[t,j] * dy[t];
+/* (source: as moe_unpermute_combine; its chain rule)
+ * Backward of the combine: dy_perm[slot(t,j)] = g[t,j] * dy[t];
  * dgate[t,j] = <dy[t], y_perm[slot(t,j)]> (fp32).
  *   dy [T,d]; y_perm [P,d]; dy_perm [P,d] out; dgate [T,k] fp32 out. */
 MOE_API int moe_combine_bwd(const moe_config *cfg, const void *dy, const void *y_perm,
                     const int32_t *slot_of_pair, const float *topk_gate, void *dy_perm,
                     float *dgate, moe_stream_t stream);
 
-/* Backward of the permute: dx[t] = sum_j dx_perm[slot(t,j)] (fp32 sum).
+/* (source: as moe_permute; its chain rule)
+ * Backward of the permute: dx[t] = sum_j dx_perm[slot(t,j)] (fp32 sum).
  *   dx_perm [P,d]; dx [T,d] out. */
 MOE_API int moe_unpermute_sum(const moe_config *cfg, const void *dx_perm,
                       const int32_t *slot_of_pair, void *dx, moe_stream_t stream);
 
-/* Router backward.  dz[t,S_j] = g_j (dgate_j - sum_j' g_j' dgate_j'), zero on
+/* (source: as moe_route_topk; its chain rule)
+ * Router backward.  dz[t,S_j] = g_j (dgate_j - sum_j' g_j' dgate_j'), zero on
  * unselected experts; dw_router = x^T dz ([d,E] fp32, overwritten);
  * dx[t] += dz[t] W_r^T (dx [T,d] dtype, read and written). */
 MOE_API int moe_route_bwd(const moe_config *cfg, const float *dgate, const float *topk_gate,
