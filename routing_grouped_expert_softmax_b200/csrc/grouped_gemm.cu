@@ -33,6 +33,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -1059,15 +1061,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ------------------------------------------------------------------ host side
+// A process may drive several GPUs, from several host threads: facts about a device are
+// cached per device ordinal (0 = not known yet), and the driver entry point once.
+constexpr int MAX_DEVICES = 64;
+
+static int device_ordinal() {
+  int dev = -1;
+  return cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < MAX_DEVICES ? dev : -1;
+}
+
 static PFN_cuTensorMapEncodeTiled_v12000 get_encode() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void *ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -1090,13 +1101,16 @@ static bool make_tmap(CUtensorMap *m, const void *ptr, int es, uint64_t cols, ui
 }
 
 static int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static std::atomic<int> cache[MAX_DEVICES];
+  const int dev = device_ordinal();
+  if (dev >= 0) {
+    const int n = cache[dev].load(std::memory_order_relaxed);
+    if (n > 0) return n;
   }
+  int n = 0;
+  if (dev < 0 || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+    n = 148;
+  if (dev >= 0) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
@@ -1112,11 +1126,14 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   static_assert(SMEM <= SMEM_LIMIT, "shared memory");
   if (ModeTraits<MODE>::WGRAD && (!o0 || !o1)) return MOE_ERR_INVALID_ARG;
   const CUtensorMap &out0 = o0 ? *o0 : a, &out1 = o1 ? *o1 : a;
-  static bool attr_set = false;
-  if (!attr_set) {
+  // the shared-memory opt-in is a per-device property of the kernel: set once per device
+  // (two threads racing here both set it, which is harmless)
+  static std::atomic<bool> attr_set[MAX_DEVICES];
+  const int dev = device_ordinal();
+  if (dev < 0 || !attr_set[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
       return MOE_ERR_CUDA;
-    attr_set = true;
+    if (dev >= 0) attr_set[dev].store(true, std::memory_order_release);
   }
   if constexpr (CG == 1) {
     const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
@@ -1135,13 +1152,15 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
     cfg.numAttrs = 1;
     // A persistent grid must be fully resident: pairs of SMs are taken inside one GPC, so
     // fewer than sm_count/2 pairs may fit at once (a late pair would run after a whole
-    // persistent pair has finished).  Ask the occupancy calculator, once.
-    static int max_pairs = 0;
-    if (!max_pairs) {
+    // persistent pair has finished).  Ask the occupancy calculator, once per device.
+    static std::atomic<int> pairs_cache[MAX_DEVICES];
+    int max_pairs = dev >= 0 ? pairs_cache[dev].load(std::memory_order_relaxed) : 0;
+    if (max_pairs <= 0) {
       cfg.gridDim = dim3((unsigned)(sm_count() / CG * CG));
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) n = sm_count() / CG;
       max_pairs = std::min(n, sm_count() / CG);
+      if (dev >= 0) pairs_cache[dev].store(max_pairs, std::memory_order_relaxed);
     }
     const int64_t units = std::min<int64_t>(max_pairs, std::max<int64_t>(max_tiles, 1));
     cfg.gridDim = dim3((unsigned)(units * CG));
