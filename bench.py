@@ -222,6 +222,18 @@ def run_ours(args):
     clk.__exit__()
     ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
 
+    # ---- step-time spread: up to 50 more steps, each between its own pair of events
+    n_spread = min(args.steps, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_spread)]
+    for a_ev, b_ev in evs:
+        a_ev.record(st)
+        step()
+        b_ev.record(st)
+    torch.cuda.synchronize()
+    per_step = sorted(a_ev.elapsed_time(b_ev) for a_ev, b_ev in evs)
+    p50 = max_over_ranks(float(np.percentile(per_step, 50)), "cuda") if per_step else None
+    p90 = max_over_ranks(float(np.percentile(per_step, 90)), "cuda") if per_step else None
+
     # ---- the grouped GEMMs alone (6 tcgen05 launches per step), same stream and inputs
     g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
     hu_buf = saved["hu"] if saved["hu"] is not None else grads["dhu"]   # recompute keeps no h | u
@@ -318,6 +330,7 @@ def run_ours(args):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms_max,
+        "ms_per_step_p50": p50, "ms_per_step_p90": p90,
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
