@@ -55,3 +55,26 @@ def test_ctypes_structures_match_the_header():
         for f in fields:
             desc = getattr(cls, f)
             assert (desc.offset, desc.size) == c[(cname, f)], (cname, f)
+
+
+def _prototypes():
+    """name -> number of parameters, from the MOE_API declarations in moe.h."""
+    import re
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(([^)]*)\)\s*;", src):
+        params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_the_prototypes():
+    lib = moe.lib() if os.path.exists(moe.LIB_PATH) else None
+    if lib is None:
+        pytest.skip("library not built")
+    protos = _prototypes()
+    assert sorted(protos) == sorted(moe.EXPORTED)
+    for name, n in protos.items():
+        fn = getattr(lib, name)
+        assert fn.argtypes is not None and len(fn.argtypes) == n, (name, n, fn.argtypes)
