@@ -4,7 +4,8 @@ TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
 benchmark's CPU-baseline leg may import this module.  The library never calls
 it, and it shares no code with the CUDA path.
 
-Every function is written for a reader to check by eye: NumPy in float64, an
+Every function is written for a reader to check by eye: NumPy in float64 (the
+routed layer can also run in float32, only to time it as the CPU baseline), an
 explicit loop over experts, a library matmul or sort as a single step, no
 blocking or fusion.
 
@@ -44,9 +45,36 @@ is "parity unpinned".
 """
 from __future__ import annotations
 
+import contextlib
+
 import numpy as np
 
 F64 = np.float64
+
+# Working precision of the routed layer's arithmetic (routing, FFN, combine and their
+# backward): float64 for parity, the default; float32 only to time the same code as the CPU
+# baseline (working_precision).  The MXFP8 quantisers below always work in float64.
+_PRECISION = [F64]
+
+
+def _wdt():
+    return _PRECISION[0]
+
+
+def _work(a):
+    """a as an array in the working precision."""
+    return np.asarray(a, _PRECISION[0])
+
+
+@contextlib.contextmanager
+def working_precision(dtype):
+    """Run the routed layer's functions in another floating type (np.float32 for timing)."""
+    old = _PRECISION[0]
+    _PRECISION[0] = np.dtype(dtype).type
+    try:
+        yield
+    finally:
+        _PRECISION[0] = old
 
 
 # ---------------------------------------------------------------------------
@@ -56,15 +84,15 @@ F64 = np.float64
 
 def router_logits(x, w_r, bias=None):
     """z = x W_r (+ b): one logit per (token, expert).  x [T,d], w_r [d,E], bias [E]."""
-    z = np.asarray(x, F64) @ np.asarray(w_r, F64)
+    z = _work(x) @ _work(w_r)
     if bias is not None:
-        z = z + np.asarray(bias, F64)[None, :]
+        z = z + _work(bias)[None, :]
     return z
 
 
 def softmax(z):
     """Row-wise softmax over the last axis."""
-    z = np.asarray(z, F64)
+    z = _work(z)
     m = z.max(axis=-1, keepdims=True)
     e = np.exp(z - m)
     return e / e.sum(axis=-1, keepdims=True)
@@ -78,7 +106,7 @@ def topk_experts(z, k):
     the same as selecting on softmax probabilities (softmax is monotone) but
     does not invent ties through rounding of exp.  Returns int32 [T,k].
     """
-    z = np.asarray(z, F64)
+    z = _work(z)
     T, E = z.shape
     index = np.broadcast_to(np.arange(E), (T, E))
     # np.lexsort sorts by the last key first: primary key -z, then expert index.
@@ -88,7 +116,7 @@ def topk_experts(z, k):
 
 def renormalised_gates(p, idx):
     """g_j = p_{S_j} / sum_{j'} p_{S_j'}: softmax probabilities renormalised over the selection."""
-    sel = np.take_along_axis(np.asarray(p, F64), np.asarray(idx, np.int64), axis=1)
+    sel = np.take_along_axis(_work(p), np.asarray(idx, np.int64), axis=1)
     return sel / sel.sum(axis=1, keepdims=True)
 
 
@@ -141,7 +169,7 @@ def routing_metadata(idx, E):
 
 def permute(x, pair_of_slot, k):
     """Rowwise dispatch: x_perm[s] = x[token of the pair in slot s]."""
-    return np.asarray(x, F64)[np.asarray(pair_of_slot) // k]
+    return _work(x)[np.asarray(pair_of_slot) // k]
 
 
 # ---------------------------------------------------------------------------
@@ -159,24 +187,24 @@ def sigmoid(h):
 
 def expert_swiglu(xr, w_gate_e, w_up_e, w_down_e):
     """One expert on its rows: h = x Wg, u = x Wu, a = silu(h) * u, y = a Wd."""
-    xr = np.asarray(xr, F64)
-    h = xr @ np.asarray(w_gate_e, F64)
-    u = xr @ np.asarray(w_up_e, F64)
+    xr = _work(xr)
+    h = xr @ _work(w_gate_e)
+    u = xr @ _work(w_up_e)
     a = silu(h) * u
-    y = a @ np.asarray(w_down_e, F64)
+    y = a @ _work(w_down_e)
     return h, u, a, y
 
 
 def grouped_swiglu(x_perm, offsets, w_gate, w_up, w_down):
     """Every expert's SwiGLU on its contiguous row range [offsets[e], offsets[e+1])."""
-    x_perm = np.asarray(x_perm, F64)
+    x_perm = _work(x_perm)
     P = x_perm.shape[0]
     f = w_gate.shape[2]
     d = w_down.shape[2]
-    h = np.zeros((P, f))
-    u = np.zeros((P, f))
-    a = np.zeros((P, f))
-    y = np.zeros((P, d))
+    h = np.zeros((P, f), _wdt())
+    u = np.zeros((P, f), _wdt())
+    a = np.zeros((P, f), _wdt())
+    y = np.zeros((P, d), _wdt())
     for e in range(w_gate.shape[0]):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi > lo:
@@ -187,11 +215,11 @@ def grouped_swiglu(x_perm, offsets, w_gate, w_up, w_down):
 
 def combine(y_perm, slot_of_pair, gate):
     """Gate-weighted unpermute: Y[t] = sum_j g[t,j] * y_perm[slot(t,j)]."""
-    gate = np.asarray(gate, F64)
+    gate = _work(gate)
     T, k = gate.shape
     slots = np.asarray(slot_of_pair).reshape(T, k)
-    y_perm = np.asarray(y_perm, F64)
-    Y = np.zeros((T, y_perm.shape[1]))
+    y_perm = _work(y_perm)
+    Y = np.zeros((T, y_perm.shape[1]), _wdt())
     for j in range(k):
         Y += gate[:, j:j + 1] * y_perm[slots[:, j]]
     return Y
@@ -229,7 +257,7 @@ def layer_fwd_routed(x, idx, gate, w_gate, w_up, w_down, shared=None):
     x_perm = permute(x, pair_of_slot, k)
     h, u, a, y_perm = grouped_swiglu(x_perm, offsets, w_gate, w_up, w_down)
     Y = combine(y_perm, slot_of_pair, gate)
-    out = dict(idx=np.asarray(idx), gate=np.asarray(gate, F64), counts=counts,
+    out = dict(idx=np.asarray(idx), gate=_work(gate), counts=counts,
                offsets=offsets, slot_of_pair=slot_of_pair, pair_of_slot=pair_of_slot,
                x_perm=x_perm, h=h, u=u, a=a, y_perm=y_perm, y=Y)
     if shared is not None:
@@ -244,13 +272,13 @@ def layer_fwd_routed(x, idx, gate, w_gate, w_up, w_down, shared=None):
 
 def combine_bwd(dY, y_perm, slot_of_pair, gate):
     """dy_perm[slot(t,j)] = g[t,j] dY[t];  dgate[t,j] = <dY[t], y_perm[slot(t,j)]>."""
-    dY = np.asarray(dY, F64)
-    gate = np.asarray(gate, F64)
+    dY = _work(dY)
+    gate = _work(gate)
     T, k = gate.shape
     slots = np.asarray(slot_of_pair).reshape(T, k)
-    y_perm = np.asarray(y_perm, F64)
+    y_perm = _work(y_perm)
     dy_perm = np.zeros_like(y_perm)
-    dgate = np.zeros((T, k))
+    dgate = np.zeros((T, k), _wdt())
     for j in range(k):
         dy_perm[slots[:, j]] = gate[:, j:j + 1] * dY
         dgate[:, j] = np.sum(dY * y_perm[slots[:, j]], axis=1)
@@ -271,20 +299,20 @@ def swiglu_bwd(da, h, u):
 def grouped_swiglu_bwd(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_down):
     """Per expert: da = dy Wd^T; (dh, du) = SwiGLU'; dx = dh Wg^T + du Wu^T;
     dWd = a^T dy; dWg = x^T dh; dWu = x^T du."""
-    dy_perm = np.asarray(dy_perm, F64)
-    x_perm = np.asarray(x_perm, F64)
+    dy_perm = _work(dy_perm)
+    x_perm = _work(x_perm)
     E = w_gate.shape[0]
     dh = np.zeros_like(h)
     du = np.zeros_like(u)
     dx_perm = np.zeros_like(x_perm)
-    dw_gate = np.zeros(w_gate.shape)
-    dw_up = np.zeros(w_up.shape)
-    dw_down = np.zeros(w_down.shape)
+    dw_gate = np.zeros(w_gate.shape, _wdt())
+    dw_up = np.zeros(w_up.shape, _wdt())
+    dw_down = np.zeros(w_down.shape, _wdt())
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi == lo:
             continue
-        wg, wu, wd = (np.asarray(w[e], F64) for w in (w_gate, w_up, w_down))
+        wg, wu, wd = (_work(w[e]) for w in (w_gate, w_up, w_down))
         da = dy_perm[lo:hi] @ wd.T
         dh[lo:hi], du[lo:hi] = swiglu_bwd(da, h[lo:hi], u[lo:hi])
         dw_down[e] = a[lo:hi].T @ dy_perm[lo:hi]
@@ -297,8 +325,8 @@ def grouped_swiglu_bwd(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_down):
 def unpermute_sum(dx_perm, slot_of_pair, T, k):
     """dx[t] = sum_j dx_perm[slot(t,j)] (the gate was already applied in combine_bwd)."""
     slots = np.asarray(slot_of_pair).reshape(T, k)
-    dx_perm = np.asarray(dx_perm, F64)
-    dx = np.zeros((T, dx_perm.shape[1]))
+    dx_perm = _work(dx_perm)
+    dx = np.zeros((T, dx_perm.shape[1]), _wdt())
     for j in range(k):
         dx += dx_perm[slots[:, j]]
     return dx
@@ -310,12 +338,12 @@ def gate_logit_grad(dgate, gate, idx, E):
     dz[t, S_j] = g_j (dg_j - sum_j' g_j' dg_j'); zero for experts not selected
     (the selection is piecewise constant in z).
     """
-    dgate = np.asarray(dgate, F64)
-    gate = np.asarray(gate, F64)
+    dgate = _work(dgate)
+    gate = _work(gate)
     T, k = gate.shape
     inner = np.sum(gate * dgate, axis=1, keepdims=True)
     dz_sel = gate * (dgate - inner)
-    dz = np.zeros((T, E))
+    dz = np.zeros((T, E), _wdt())
     np.put_along_axis(dz, np.asarray(idx, np.int64), dz_sel, axis=1)
     return dz
 
@@ -324,8 +352,8 @@ def route_bwd(dgate, gate, idx, x, w_r):
     """Router backward: dz as above, dW_r = x^T dz, dx_router = dz W_r^T."""
     E = w_r.shape[1]
     dz = gate_logit_grad(dgate, gate, idx, E)
-    dw_r = np.asarray(x, F64).T @ dz
-    dx = dz @ np.asarray(w_r, F64).T
+    dw_r = _work(x).T @ dz
+    dx = dz @ _work(w_r).T
     return dz, dw_r, dx
 
 
@@ -334,7 +362,7 @@ def shared_expert_bwd(dY, x, fwd, shared):
     SwiGLU backward of one expert holding every token, in the same steps as the routed
     experts'.  Returns dx and the three weight gradients."""
     T = np.asarray(x).shape[0]
-    one = [np.asarray(w, F64)[None] for w in shared]     # one expert [1, ...]
+    one = [_work(w)[None] for w in shared]     # one expert [1, ...]
     g = grouped_swiglu_bwd(dY, x, fwd["shared_h"], fwd["shared_u"], fwd["shared_a"],
                            np.array([0, T]), *one)
     return dict(shared_dx=g["dx_perm"], dw_shared_gate=g["dw_gate"][0],
@@ -371,7 +399,6 @@ def layer_bwd_routed(fwd, dY, w_gate, w_up, w_down, x=None, shared=None):
         out.update(shared_expert_bwd(dY, x, fwd, shared))
         out["dx"] = out["dx"] + out["shared_dx"]
     return out
-
 
 # ---------------------------------------------------------------------------
 # MXFP8: [unite.ai] / [ettayeb] / [kitmori] ("MXFP8 for selected operations,
@@ -503,15 +530,14 @@ def mx_quantize_grouped_rows(v, offsets):
 def grouped_swiglu_mx(x_perm, offsets, w_gate, w_up, w_down):
     """Forward expert FFN with every GEMM operand MXFP8-quantised along its own K.
 
-    GEMM 1: x_perm (K = d, along rows' columns) with W_gate/W_up (K = d, along
+    GEMM 1: x_perm (K = d, along rows' columns) with W_gate/W_up (K = d, down
     their rows).  GEMM 2: a (K = f) with W_down (K = f).  Products and sums in
     float64 on the dequantised values.  The MXFP8 GEMMs output bf16, so GEMM 2
-    quantises a as stored: bf16(a).  Returns h, u, a unrounded.
+    quantises a as stored: bf16(a).  Returns h, u, a unrounded.  Each expert's
+    weights are quantised inside the loop (blocks never cross experts), so only
+    experts holding rows are quantised.
     """
     xq = mx_quantize(x_perm, axis=1)[2]
-    wgq = mx_quantize(w_gate, axis=1)[2]
-    wuq = mx_quantize(w_up, axis=1)[2]
-    wdq = mx_quantize(w_down, axis=1)[2]
     P = xq.shape[0]
     f = w_gate.shape[2]
     d = w_down.shape[2]
@@ -523,14 +549,14 @@ def grouped_swiglu_mx(x_perm, offsets, w_gate, w_up, w_down):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi == lo:
             continue
-        h[lo:hi] = xq[lo:hi] @ wgq[e]
-        u[lo:hi] = xq[lo:hi] @ wuq[e]
+        h[lo:hi] = xq[lo:hi] @ mx_quantize(w_gate[e], axis=0)[2]
+        u[lo:hi] = xq[lo:hi] @ mx_quantize(w_up[e], axis=0)[2]
         a[lo:hi] = silu(h[lo:hi]) * u[lo:hi]
     aq = mx_quantize(bf16_rne(a), axis=1)[2]
     for e in range(w_gate.shape[0]):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi > lo:
-            y[lo:hi] = aq[lo:hi] @ wdq[e]
+            y[lo:hi] = aq[lo:hi] @ mx_quantize(w_down[e], axis=0)[2]
     return h, u, a, y
 
 
@@ -541,26 +567,25 @@ def grouped_swiglu_bwd_mx(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_dow
     K = 2f with [W_gate|W_up]^T); weight-gradient GEMMs reduce over the tokens
     of one expert (blocks of 32 rows inside each expert, zero-padded).  [dh|du]
     is the bf16 output of the first GEMM's epilogue, so both GEMMs that read it
-    quantise bf16([dh|du]).  Returns dh, du unrounded.
+    quantise bf16([dh|du]).  Returns dh, du unrounded.  Weights are quantised per
+    expert, as in grouped_swiglu_mx.
     """
     dy_perm = np.asarray(dy_perm, F64)
     x_perm = np.asarray(x_perm, F64)
     E = w_gate.shape[0]
     f = w_gate.shape[2]
     dyq_k = mx_quantize(dy_perm, axis=1)[2]
-    wdq_t = mx_quantize(w_down, axis=2)[2]          # W_down^T has K = d along W_down's columns
     dh = np.zeros_like(h)
     du = np.zeros_like(u)
     for e in range(E):
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi == lo:
             continue
-        da = dyq_k[lo:hi] @ wdq_t[e].T
+        wdq_t = mx_quantize(w_down[e], axis=1)[2]     # W_down^T has K = d along W_down's columns
+        da = dyq_k[lo:hi] @ wdq_t.T
         dh[lo:hi], du[lo:hi] = swiglu_bwd(da, h[lo:hi], u[lo:hi])
     dhu = bf16_rne(np.concatenate([dh, du], axis=1))
     dhuq_k = mx_quantize(dhu, axis=1)[2]
-    wgu = np.concatenate([np.asarray(w_gate, F64), np.asarray(w_up, F64)], axis=2)  # [E, d, 2f]
-    wguq_t = mx_quantize(wgu, axis=2)[2]
     # weight-gradient operands: reduction over tokens inside each expert
     aq_t = mx_quantize_grouped_rows(a, offsets)
     dyq_t = mx_quantize_grouped_rows(dy_perm, offsets)
@@ -574,9 +599,90 @@ def grouped_swiglu_bwd_mx(dy_perm, x_perm, h, u, a, offsets, w_gate, w_up, w_dow
         lo, hi = int(offsets[e]), int(offsets[e + 1])
         if hi == lo:
             continue
-        dx_perm[lo:hi] = dhuq_k[lo:hi] @ wguq_t[e].T
+        wgu = np.concatenate([np.asarray(w_gate[e], F64), np.asarray(w_up[e], F64)], axis=1)  # [d, 2f]
+        wguq_t = mx_quantize(wgu, axis=1)[2]
+        dx_perm[lo:hi] = dhuq_k[lo:hi] @ wguq_t.T
         dw_down[e] = aq_t[lo:hi].T @ dyq_t[lo:hi]
         dwgu = xq_t[lo:hi].T @ dhuq_t[lo:hi]
         dw_gate[e] = dwgu[:, :f]
         dw_up[e] = dwgu[:, f:]
     return dict(dh=dh, du=du, dx_perm=dx_perm, dw_gate=dw_gate, dw_up=dw_up, dw_down=dw_down)
+
+
+# ---------------------------------------------------------------------------
+# The MXFP8 layer step: the steps of layer_fwd / layer_bwd in the same order, with the
+# grouped GEMMs above in place of the bf16 ones.  The MXFP8 GEMMs write bf16, and the layer
+# keeps five tensors in that storage between its GEMMs; each later step reads the stored
+# bf16 value, so the oracle rounds exactly these (and nothing else) to bf16:
+#   h, u     GEMM 1's outputs, read by the SwiGLU backward;
+#   a        silu(h) * u from GEMM 1's unrounded outputs, quantised by GEMM 2 and by
+#            the down projection's weight-gradient GEMM (rounded inside the GEMM steps);
+#   dy_perm  g * dY, quantised by both GEMMs that read it;
+#   [dh|du]  the SwiGLU backward's output, quantised by both GEMMs that read it
+#            (rounded inside grouped_swiglu_bwd_mx).
+# y_perm, dgate, dx_perm and the weight gradients stay unrounded, as in the bf16 oracle.
+# ---------------------------------------------------------------------------
+
+def shared_expert_fwd_mx(x, shared):
+    """The shared expert with MXFP8 GEMMs: one group holding every token."""
+    T = np.asarray(x).shape[0]
+    one = [np.asarray(w, F64)[None] for w in shared]
+    h, u, a, y = grouped_swiglu_mx(x, np.array([0, T]), *one)
+    return dict(shared_h=h, shared_u=u, shared_a=a, shared_y=y)
+
+
+def shared_expert_bwd_mx(dY, x, fwd, shared):
+    """Its backward: output gradient dY (weight 1), the stored bf16 h, u, a as for the
+    routed experts."""
+    T = np.asarray(x).shape[0]
+    one = [np.asarray(w, F64)[None] for w in shared]
+    b = bf16_rne
+    g = grouped_swiglu_bwd_mx(dY, x, b(fwd["shared_h"]), b(fwd["shared_u"]), b(fwd["shared_a"]),
+                              np.array([0, T]), *one)
+    return dict(shared_dx=g["dx_perm"], dw_shared_gate=g["dw_gate"][0], dw_shared_up=g["dw_up"][0],
+                dw_shared_down=g["dw_down"][0], shared_dh=g["dh"], shared_du=g["du"])
+
+
+def layer_fwd_mx(x, w_r, w_gate, w_up, w_down, k, bias=None, routing=None, shared=None):
+    """Whole forward step with MXFP8 grouped GEMMs.  routing: None (the router runs), or
+    (idx, gate) given (uniform random routing; then no router logits).  shared: None or
+    the shared expert's (W_gate, W_up, W_down)."""
+    E = w_gate.shape[0]
+    out = {}
+    if routing is None:
+        z, p, idx, gate = route(x, w_r, k, bias)
+        out.update(z=z, p=p)
+    else:
+        idx, gate = np.asarray(routing[0]), np.asarray(routing[1], F64)
+        k = idx.shape[1]
+    counts, offsets, slot_of_pair, pair_of_slot = routing_metadata(idx, E)
+    x_perm = permute(x, pair_of_slot, k)
+    h, u, a, y_perm = grouped_swiglu_mx(x_perm, offsets, w_gate, w_up, w_down)
+    Y = combine(y_perm, slot_of_pair, gate)
+    out.update(idx=idx, gate=gate, counts=counts, offsets=offsets, slot_of_pair=slot_of_pair,
+               pair_of_slot=pair_of_slot, x_perm=x_perm, h=h, u=u, a=a, y_perm=y_perm, y=Y)
+    if shared is not None:
+        out.update(shared_expert_fwd_mx(x, shared))
+        out["y"] = Y + out["shared_y"]
+    return out
+
+
+def layer_bwd_mx(fwd, dY, x, w_r, w_gate, w_up, w_down, router=True, shared=None):
+    """Whole backward step with MXFP8 grouped GEMMs, given the forward dict from
+    layer_fwd_mx.  router=False: routing held fixed (no router gradient)."""
+    T, k = fwd["gate"].shape
+    dy_perm, dgate = combine_bwd(dY, fwd["y_perm"], fwd["slot_of_pair"], fwd["gate"])
+    b = bf16_rne
+    g = grouped_swiglu_bwd_mx(b(dy_perm), fwd["x_perm"], b(fwd["h"]), b(fwd["u"]), b(fwd["a"]),
+                              fwd["offsets"], w_gate, w_up, w_down)
+    dx = unpermute_sum(g["dx_perm"], fwd["slot_of_pair"], T, k)
+    out = dict(dy_perm=dy_perm, dgate=dgate, dx_experts=dx, **g)
+    if router:
+        dz, dw_r, dx_r = route_bwd(dgate, fwd["gate"], fwd["idx"], x, w_r)
+        out.update(dz=dz, dw_r=dw_r)
+        dx = dx + dx_r
+    if shared is not None:
+        out.update(shared_expert_bwd_mx(dY, x, fwd, shared))
+        dx = dx + out["shared_dx"]
+    out["dx"] = dx
+    return out
