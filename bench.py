@@ -32,6 +32,8 @@ WORKLOADS = {
     "e8_fwd_bwd": (8192, 2048, 8, 4, 1024, False, "router"),
     "e128_t16k_skew_fwd_bwd": (16384, 2048, 128, 4, 1024, True, "router"),
     "e128_t16k_uniform_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "uniform"),
+    # the MXFP8 workload's shapes and inputs in bf16 (the pair that MXFP8 is compared within)
+    "e128_t16k_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "router"),
     # a smaller case of the same kernels for profiler captures (still larger than L2)
     "profile_e32_t4k": (4096, 2048, 32, 4, 1024, False, "router"),
     # 256 rows per expert, as at T=8192, E=128, k=4
@@ -45,6 +47,11 @@ WORKLOADS = {
     "e128_recompute_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "native", {"recompute": True}),
 }
 DEFAULT = "e128_fwd_bwd"
+# Timed after the main workload, each in a short run of its own, and reported beside it: the
+# pages' two comparisons -- 8 against 128 experts at equal active FLOPs (qidao123.com, section
+# "新闻原文"), and MXFP8 against bf16 (unite.ai, section "Παραλληλισμός, Ακρίβεια και
+# Τεχνικές Μνήμης") -- on this layer.
+SWEEP = ("e128_fwd_bwd", "e8_fwd_bwd", "e128_t16k_fwd_bwd", "e128_t16k_mxfp8_fwd_bwd")
 
 
 def peaks():
@@ -153,6 +160,85 @@ def to_dev_bf16(a, torch):
     return torch.from_numpy(gen.bf16_bits(a).view(np.int16)).view(torch.bfloat16).cuda()
 
 
+def _workload_spec(name):
+    T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
+    prec = WORKLOADS[name][7] if len(WORKLOADS[name]) > 7 else "native"
+    opts = WORKLOADS[name][8] if len(WORKLOADS[name]) > 8 else {}
+    return T, d, E, k, f, skew, routing, prec, bool(opts.get("shared")), bool(opts.get("recompute"))
+
+
+class Layer:
+    """One workload's device buffers and its step (moe_layer_fwd + moe_layer_bwd)."""
+
+    def __init__(self, name, inp):
+        import torch
+
+        import routing_grouped_expert_softmax_b200 as moe
+        self.moe, self.name, self.inp = moe, name, inp
+        T, d, E, k, f, skew, routing, prec, shared, recompute = _workload_spec(name)
+        self.T, self.d, self.E, self.k, self.f, self.prec = T, d, E, k, f, prec
+        self.routing, self.shared, self.recompute = routing, shared, recompute
+        self.cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
+        self.st = torch.cuda.current_stream()
+        self.ws = moe.alloc_workspace(self.cfg)
+        self.saved = moe.alloc_saved(self.cfg, logits=False, shared=shared, recompute=recompute)
+        self.grads = moe.alloc_grads(self.cfg, router=(routing == "router"), shared=shared)
+        self.x = to_dev_bf16(inp.x, torch)
+        self.dy = to_dev_bf16(inp.dy, torch)
+        self.wr, self.wg, self.wu, self.wd = (to_dev_bf16(a, torch) for a in (inp.w_r, inp.w_gate, inp.w_up,
+                                                                              inp.w_down))
+        self.bias = torch.from_numpy(inp.bias).cuda() if inp.bias is not None else None
+        sh = None
+        if shared:
+            from routing_grouped_expert_softmax_b200 import inputs as gen
+            sh = tuple(to_dev_bf16(a, torch) for a in gen.make_shared_expert(d, f, seed=1))
+        self.w = moe.layer_weights(self.wr, self.bias, self.wg, self.wu, self.wd, shared=sh)
+        self.y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        self.fwd_fn = moe.moe_layer_fwd
+        if routing == "uniform":
+            self.saved["topk_idx"].copy_(torch.from_numpy(inp.extra["idx"]))
+            self.saved["topk_gate"].copy_(torch.from_numpy(inp.extra["gate"]))
+            self.fwd_fn = moe.moe_layer_fwd_routed
+        self.launches_per_step = count_launches(routing, prec, shared, recompute)
+
+    def step(self, x=None, dy=None, y=None, grads=None):
+        self.fwd_fn(self.cfg, self.w, self.x if x is None else x, self.y if y is None else y, self.saved, self.ws,
+                    self.st)
+        self.moe.moe_layer_bwd(self.cfg, self.w, self.x if x is None else x, self.dy if dy is None else dy,
+                               self.saved, self.grads if grads is None else grads, self.ws, self.st)
+
+    def layer_bytes(self):
+        """Device bytes the layer's own buffers hold: workspace, forward context, gradients."""
+        n = self.ws.numel()
+        for dct in (self.saved, self.grads):
+            n += sum(t.numel() * t.element_size() for t in dct.values() if t is not None)
+        return n
+
+    def load(self):
+        c = self.saved["counts"].cpu().numpy().astype(np.int64)
+        m = c.mean()
+        return {"max_over_mean": float(c.max() / m), "min_over_mean": float(c.min() / m),
+                "empty_experts": int((c == 0).sum()), "counts": c.tolist()}
+
+
+def time_steps(layer, steps, warmup, barrier):
+    """Device time of `steps` back-to-back steps (CUDA events on the launching stream), ms per step."""
+    import torch
+    for _ in range(warmup):
+        layer.step()
+    torch.cuda.synchronize()
+    assert layer.moe.moe_get_error(layer.ws) == 0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    e0.record(layer.st)
+    for _ in range(steps):
+        layer.step()
+    e1.record(layer.st)
+    barrier()
+    assert layer.moe.moe_get_error(layer.ws) == 0
+    return e0.elapsed_time(e1) / steps
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -165,36 +251,17 @@ def run_ours(args):
     torch.cuda.set_device(local)
     build.build()
     name = args.workload
-    T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
-    prec = WORKLOADS[name][7] if len(WORKLOADS[name]) > 7 else "native"
-    opts = WORKLOADS[name][8] if len(WORKLOADS[name]) > 8 else {}
-    shared, recompute = bool(opts.get("shared")), bool(opts.get("recompute"))
+    T, d, E, k, f, skew, routing, prec, shared, recompute = _workload_spec(name)
     inp = make_inputs(name, seed=0)
-    cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
-    st = torch.cuda.current_stream()
-    ws = moe.alloc_workspace(cfg)
-    saved = moe.alloc_saved(cfg, logits=False, shared=shared, recompute=recompute)
-    grads = moe.alloc_grads(cfg, router=(routing == "router"), shared=shared)
-    x = to_dev_bf16(inp.x, torch)
-    dy = to_dev_bf16(inp.dy, torch)
-    wr, wg, wu, wd = (to_dev_bf16(a, torch) for a in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down))
-    bias = torch.from_numpy(inp.bias).cuda() if inp.bias is not None else None
-    sh = None
-    if shared:
-        from routing_grouped_expert_softmax_b200 import inputs as gen
-        sh = tuple(to_dev_bf16(a, torch) for a in gen.make_shared_expert(d, f, seed=1))
-    w = moe.layer_weights(wr, bias, wg, wu, wd, shared=sh)
-    y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
-    fwd_fn = moe.moe_layer_fwd
-    if routing == "uniform":
-        saved["topk_idx"].copy_(torch.from_numpy(inp.extra["idx"]))
-        saved["topk_gate"].copy_(torch.from_numpy(inp.extra["gate"]))
-        fwd_fn = moe.moe_layer_fwd_routed
-    launches_per_step = count_launches(routing, prec, shared, recompute)
-
-    def step():
-        fwd_fn(cfg, w, x, y, saved, ws, st)
-        moe.moe_layer_bwd(cfg, w, x, dy, saved, grads, ws, st)
+    torch.cuda.reset_peak_memory_stats()
+    base_mem = torch.cuda.memory_allocated()
+    L = Layer(name, inp)
+    st = L.st
+    cfg, saved, grads, ws = L.cfg, L.saved, L.grads, L.ws
+    wg, wu, wd = L.wg, L.wu, L.wd
+    x, dy, y = L.x, L.dy, L.y
+    step = L.step
+    launches_per_step = L.launches_per_step
 
     def barrier():
         if ws_n > 1:
@@ -221,6 +288,8 @@ def run_ours(args):
     clk.window(t_start, time.time())
     clk.__exit__()
     ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
+    peak_mem = torch.cuda.max_memory_allocated() - base_mem
+    load = L.load()
 
     # ---- step-time spread: up to 50 more steps, each between its own pair of events
     n_spread = min(args.steps, 50)
@@ -289,8 +358,7 @@ def run_ours(args):
         st.wait_event(ev["in"][b])
         if i >= 2:
             st.wait_event(ev["out"][b])                  # step i-2's outputs have left
-        fwd_fn(cfg, w, xs[b], ys[b], saved, ws, st)
-        moe.moe_layer_bwd(cfg, w, xs[b], dys[b], saved, gs[b], ws, st)
+        step(xs[b], dys[b], ys[b], gs[b])
         ev["comp"][b].record(st)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["comp"][b])
@@ -302,6 +370,29 @@ def run_ours(args):
     barrier()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
     assert moe.moe_get_error(ws) == 0
+    layer_gib = L.layer_bytes() / 2 ** 30
+    del L, xs, dys, ys, gs, saved, grads, ws, x, dy, y, hx, hdy, hy, hdx
+    torch.cuda.empty_cache()
+
+    # ---- the sweep's other points, each in its own short timed run: E=8 at equal active
+    # FLOPs (the pages' 8 -> 128 experts comparison) and the T=16384 shapes in bf16 and in
+    # MXFP8 (the pages' MXFP8 against bf16 comparison)
+    sweep = {}
+    if not args.no_sweep:
+        cache = {}
+        for other in SWEEP:
+            if other == name:
+                sweep[other] = ms_max
+                continue
+            key = _workload_spec(other)[:7]
+            if key not in cache:
+                cache.clear()
+                cache[key] = make_inputs(other, seed=0)
+            lo = Layer(other, cache[key])
+            sweep[other] = max_over_ranks(time_steps(lo, min(args.steps, 30), max(args.warmup, 3), barrier), "cuda")
+            del lo
+            torch.cuda.empty_cache()
+        cache.clear()
 
     P = T * k
     flops_fwd = 6.0 * P * d * f
@@ -309,11 +400,10 @@ def run_ours(args):
     pk = peaks()
     gemm_ms = fwd_ms + bwd_ms
     tflops = (flops_fwd + flops_bwd) / (gemm_ms * 1e-3) / 1e12
-    # The GEMMs are timed back to back for `steps` iterations (a long, power-capped loop), so
-    # the tensor roof is the sustained bf16 figure.  An MXFP8 contraction is measured against
-    # the fp8 peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25).
-    bf16_peak = pk["bf16_sus"] or pk["bf16"]
-    peak_tc = bf16_peak * (2.0 if prec == "mxfp8" else 1.0)
+    # The six GEMMs are timed per step between events, a loop of well under a second: the
+    # tensor roof is the burst bf16 figure.  An MXFP8 contraction is measured against the fp8
+    # peak: the measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25).
+    peak_tc = pk["bf16"] * (2.0 if prec == "mxfp8" else 1.0)
     bytes_fwd, bytes_bwd = gemm_algorithmic_bytes(P, d, f, E, prec)
     gbs = (bytes_fwd + bytes_bwd) / (gemm_ms * 1e-3) / 1e9
     # the binding roof: whichever of the FLOP time and the byte time is longer
@@ -349,12 +439,12 @@ def run_ours(args):
                      "unit": "GB/s" if hbm_bound else "TFLOP/s",
                      "frac": gbs / pk["hbm"] if hbm_bound else tflops / peak_tc,
                      "peak_source": (f"{pk['src']} HBM copy" if hbm_bound else
-                                     f"{pk['src']} bf16 {'sustained' if pk['bf16_sus'] else 'burst'}"
-                                     + (" x 2 (nominal fp8/bf16)" if prec == "mxfp8" else "")),
+                                     f"{pk['src']} bf16 burst" + (" x 2 (nominal fp8/bf16)" if prec == "mxfp8" else "")),
                      "traffic": traffic,
                      "algorithmic_bytes_per_step": bytes_fwd + bytes_bwd,
                      "flops_per_step": flops_fwd + flops_bwd,
                      "tensor_tflops": tflops, "tensor_frac": tflops / peak_tc,
+                     "tensor_peak_source": f"{pk['src']} bf16 burst" + (" x 2" if prec == "mxfp8" else ""),
                      "hbm_gbs": gbs, "hbm_frac": gbs / pk["hbm"],
                      "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                      "fwd_tflops": flops_fwd / (fwd_ms * 1e-3) / 1e12,
@@ -363,9 +453,21 @@ def run_ours(args):
                 "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": 2 * T * d * 2},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk.summary(),
+        "load": load,
+        "memory": {"peak_gib": peak_mem / 2 ** 30, "layer_buffers_gib": layer_gib,
+                   "what": "peak torch-allocated device memory of the workload (inputs, weights, forward "
+                           "context, gradients, workspace; the library allocates nothing)"},
     }
+    if sweep:
+        out["sweep_ms_per_step"] = sweep
+        r = {}
+        if "e8_fwd_bwd" in sweep and "e128_fwd_bwd" in sweep:
+            r["e128_over_e8_time"] = sweep["e128_fwd_bwd"] / sweep["e8_fwd_bwd"]
+        if "e128_t16k_fwd_bwd" in sweep and "e128_t16k_mxfp8_fwd_bwd" in sweep:
+            r["mxfp8_speedup_over_bf16"] = sweep["e128_t16k_fwd_bwd"] / sweep["e128_t16k_mxfp8_fwd_bwd"]
+        out["sweep_ratios"] = r
     if rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(inp, k, args.cpu_tokens)
+        out["cpu_baseline"] = cpu_baseline(inp, k, routing)
     if ws_n > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -431,27 +533,72 @@ def count_launches(routing, prec="native", shared=False, recompute=False):
     return n
 
 
-def cpu_baseline(inp, k, n_tokens):
-    """The CPU oracle (float64 NumPy, per-expert loops) on the first n_tokens tokens of the
-    same workload, forward + backward; tokens/s."""
-    from oracle import moe_ref as ref
+def _oracle_step(ref, inp, k, routing, fwd_only=False):
+    """One layer step of the oracle on inp (the whole batch it holds)."""
+    if routing == "uniform":
+        fwd = ref.layer_fwd_routed(inp.x, inp.extra["idx"], inp.extra["gate"], inp.w_gate, inp.w_up, inp.w_down)
+        if not fwd_only:
+            ref.layer_bwd_routed(fwd, inp.dy, inp.w_gate, inp.w_up, inp.w_down)
+    else:
+        fwd = ref.layer_fwd(inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
+        if not fwd_only:
+            ref.layer_bwd(fwd, inp.dy, inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
+
+
+def _token_sample(inp, n):
+    import dataclasses
+    extra = dict(inp.extra)
+    if "idx" in extra:
+        extra["idx"], extra["gate"] = extra["idx"][:n], extra["gate"][:n]
+    return dataclasses.replace(inp, T=n, x=inp.x[:n], dy=inp.dy[:n], extra=extra)
+
+
+def _blas_threads():
     try:
         from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
     except Exception:
-        cores = os.cpu_count()
-    xs, dys = inp.x[:n_tokens], inp.dy[:n_tokens]
-    t0 = time.perf_counter()
-    fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
-    ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
-    dt = time.perf_counter() - t0
-    return {"value": n_tokens / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n_tokens} tokens of the workload, full weights, fwd+bwd, float64",
-            "seconds": dt}
+        return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(inp, k, routing):
+    """The CPU oracle (NumPy, per-expert loops, BLAS matmuls) in its float32 working precision
+    on the host cores: the workload's whole batch, forward and forward + backward (median of
+    two timed runs after one warm-up), and a 512-token sample of it on one thread."""
+    from oracle import moe_ref as ref
+    with ref.working_precision(np.float32):
+        _oracle_step(ref, inp, k, routing)
+        tf, tb = [], []
+        for _ in range(2):
+            t0 = time.perf_counter()
+            _oracle_step(ref, inp, k, routing, fwd_only=True)
+            tf.append(time.perf_counter() - t0)
+            t0 = time.perf_counter()
+            _oracle_step(ref, inp, k, routing)
+            tb.append(time.perf_counter() - t0)
+        one = None
+        try:
+            from threadpoolctl import threadpool_limits
+            small = _token_sample(inp, min(512, inp.T))
+            with threadpool_limits(limits=1):
+                _oracle_step(ref, small, k, routing)
+                t0 = time.perf_counter()
+                _oracle_step(ref, small, k, routing)
+                one = {"value": small.T / (time.perf_counter() - t0), "unit": "tokens/s", "cores": 1,
+                       "sample": f"first {small.T} tokens of the workload, all weights, fwd+bwd, float32"}
+        except ImportError:
+            pass
+    t_fb, t_f = float(np.median(tb)), float(np.median(tf))
+    return {"value": inp.T / t_fb, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"the whole workload ({inp.T} tokens), fwd+bwd, float32 NumPy with BLAS, "
+                      "median of 2 runs after 1 warm-up",
+            "seconds_per_step": t_fb, "fwd_tokens_per_s": inp.T / t_f, "affinity_cores": len(os.sched_getaffinity(0)),
+            "one_thread": one}
 
 
 def run_reference(args):
-    """The reference arm is the CPU oracle itself, timed on the host cores."""
+    """The reference arm is the CPU oracle itself (float32 working precision, BLAS matmuls),
+    timed on the host cores."""
     ws_n, rank, local = dist_env()
     if rank != 0:
         return
@@ -459,40 +606,34 @@ def run_reference(args):
     T, d, E, k, f, skew, routing = WORKLOADS[name][:7]
     inp = make_inputs(name, seed=0)
     from oracle import moe_ref as ref
-    # size each step's token sample so that the W warm-up and K timed steps take about two
-    # minutes together
-    probe = 16
-    t0 = time.perf_counter()
-    fwd = ref.layer_fwd(inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
-    ref.layer_bwd(fwd, inp.dy[:probe], inp.x[:probe], inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
-    t_probe = time.perf_counter() - t0
-    n_steps = max(args.steps + args.warmup, 1)
-    n = int(max(4, min(args.cpu_tokens, probe * (120.0 / n_steps) / max(t_probe, 1e-3))))
-    xs, dys = inp.x[:n], inp.dy[:n]
-    for _ in range(args.warmup):
-        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
-        ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
-    times = []
-    for _ in range(args.steps):
+    with ref.working_precision(np.float32):
+        # size each step's token sample so that the W warm-up and K timed steps take about two
+        # minutes together
+        probe = _token_sample(inp, min(1024, T))
         t0 = time.perf_counter()
-        fwd = ref.layer_fwd(xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias)
-        ref.layer_bwd(fwd, dys, xs, inp.w_r, inp.w_gate, inp.w_up, inp.w_down)
-        times.append(time.perf_counter() - t0)
+        _oracle_step(ref, probe, k, routing)
+        t_probe = time.perf_counter() - t0
+        n_steps = max(args.steps + args.warmup, 1)
+        n = int(max(64, min(T, probe.T * (120.0 / n_steps) / max(t_probe, 1e-3))))
+        sample = _token_sample(inp, n)
+        for _ in range(args.warmup):
+            _oracle_step(ref, sample, k, routing)
+        times = []
+        for _ in range(args.steps):
+            t0 = time.perf_counter()
+            _oracle_step(ref, sample, k, routing)
+            times.append(time.perf_counter() - t0)
     dt = float(np.mean(times))
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
-    except Exception:
-        cores = os.cpu_count()
     v = n / dt
     print(json.dumps({
         "impl": "reference", "metric": "MoE-layer tokens/s (E=128,k=4,bf16 fwd+bwd) 1xB200; grouped-GEMM % TC peak",
         "value": v, "unit": "tokens/s", "n_gpus": ws_n, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic", "config": {"workload": name, "T": T, "d_model": d, "experts": E,
+        "dtype": "f32", "data": "synthetic", "config": {"workload": name, "T": T, "d_model": d, "experts": E,
                                                           "top_k": k, "ffn": f},
-        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-                         "sample": f"first {n} tokens per step, full weights, fwd+bwd, float64"},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"first {n} tokens of the workload per step, all weights, fwd+bwd, float32 "
+                                   "NumPy with BLAS"},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }))
 
@@ -504,8 +645,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
-    ap.add_argument("--cpu-tokens", type=int, default=128)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="time the main workload only")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

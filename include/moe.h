@@ -101,6 +101,18 @@ MOE_API size_t moe_workspace_size(const moe_config *cfg);
  * *code receives 0 or an OR of MOE_ERR_DEVICE_* bits. */
 MOE_API int moe_get_error(void *ws, moe_stream_t stream, int32_t *code);
 
+/* (the pages have no counterpart: failure detection)
+ * Test hook for the kernels' bounded waits.  ns > 0: every grouped GEMM (and the tensor-core
+ * router) launched afterwards from this process with single-CTA tiles first waits up to ns
+ * nanoseconds on a barrier that nothing arrives on; the wait runs out, every role of the
+ * kernel stops, the copies and MMAs already in flight are drained, TMEM is freed, the kernel
+ * returns, and MOE_ERR_DEVICE_TIMEOUT is OR-ed into the workspace's error word.  Launches with
+ * CTA-pair tiles ignore it.  The outputs of such a launch are undefined.  ns = 0 (the default)
+ * turns it off.  ns above MOE_DEBUG_STALL_MAX_NS returns MOE_ERR_INVALID_ARG.  Process-wide,
+ * not synchronised with launches already enqueued. */
+#define MOE_DEBUG_STALL_MAX_NS 1000000000ull
+MOE_API int moe_debug_set_gemm_stall_ns(uint64_t ns);
+
 /* ---------------------------------------------------------------- routing */
 
 /* Router forward (source: qidao123.com, section "新闻原文", 4 of E experts per token; unite.ai, section "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης").
@@ -140,9 +152,14 @@ MOE_API int moe_build_offsets(const moe_config *cfg, const int32_t *topk_idx, in
  * (The pages have no counterpart: this is a calling convention, not a step of the method.)
  *   Scratch: a fixed 256 KiB array inside the library, held on every GPU that loads the
  *   library until the process exits; it must hold ceil(T*k/1024) * E int32 histogram
- *   entries, so larger shapes return MOE_ERR_UNSUPPORTED (e.g. T*k = 262144 at E = 256).
+ *   entries (65536 at most), so larger shapes return MOE_ERR_UNSUPPORTED and launch
+ *   nothing (e.g. T*k = 262145 at E = 256; T*k = 262144 at E = 256 is the largest fit).
  *   The first call made with a given device current looks up the array's device address
- *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   (cudaGetSymbolAddress) and keeps it for that device; make that first call before any
+ *   stream capture.  The address kept is the one in the context current at that first call,
+ *   which is the device's primary context for callers of the CUDA runtime; a caller that
+ *   later makes another context of the same device current (through the driver API) is not
+ *   supported.
  *   Every call shares the one array: calls whose work can overlap on the GPU (different
  *   streams, different host threads) race and must be ordered by the caller.
  *   An expert index outside [0, E) leaves the outputs undefined and is not reported.

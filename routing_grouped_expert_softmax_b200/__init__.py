@@ -36,7 +36,7 @@ EXPORTED = [
     "moe_build_offsets", "moe_build_offsets_noalloc", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
     "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd", "moe_mx_quantize_rows",
-    "moe_mx_quantize_cols", "moe_permute_mxfp8",
+    "moe_mx_quantize_cols", "moe_permute_mxfp8", "moe_debug_set_gemm_stall_ns",
 ]
 
 
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "moe_workspace_size": (ctypes.c_size_t, [_CFG]),
             "moe_get_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
+            "moe_debug_set_gemm_stall_ns": (ctypes.c_int, [ctypes.c_uint64]),
             "moe_route_topk": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]),
             "moe_topk_gating": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P]),
             "moe_build_offsets": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P]),
@@ -161,6 +162,12 @@ def moe_get_error(ws, stream=None) -> int:
     code = ctypes.c_int32(0)
     _call("moe_get_error", ptr(ws), stream_handle(stream), ctypes.byref(code))
     return code.value
+
+
+def moe_debug_set_gemm_stall_ns(ns: int):
+    """Failure-detection test hook: later single-CTA grouped GEMM launches wait up to ns on a
+    barrier nothing arrives on and take their abort path (0 turns it off)."""
+    _call("moe_debug_set_gemm_stall_ns", ns)
 
 
 def moe_route_topk(cfg, x, w_router, bias, logits, topk_idx, topk_gate, ws, stream=None):

@@ -137,6 +137,10 @@ __device__ __forceinline__ void set_error(int *err, int bit) {
   if (err) atomicOr(err, bit);
 }
 
+// Failure-detection test hook of the grouped GEMMs (grouped_gemm.cu): ns > 0 makes every later
+// single-CTA launch wait up to ns on a barrier nothing arrives on and take its abort path.
+void set_gemm_stall_ns(uint64_t ns);
+
 // ---- internal launchers (host side), implemented in routing.cu / rowops.cu / grouped_gemm.cu
 cudaError_t launch_route_topk(const Shape &s, const void *x, const void *w_r, const float *bias,
                               float *logits, int32_t *idx, float *gate, int *err, cudaStream_t st);

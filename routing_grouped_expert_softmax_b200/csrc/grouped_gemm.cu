@@ -126,6 +126,11 @@ struct Params {
   int sfa_ld, sfb_ld;
   int *err;
   int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
+  // Failure-detection test hook, 0 in normal use: the MMA issuer of a single-CTA launch first
+  // waits up to stall_ns on a barrier nothing arrives on, so that the wait runs out and the
+  // kernel takes its abort path (every role stops, in-flight copies and MMAs are drained,
+  // MOE_ERR_DEVICE_TIMEOUT is reported).
+  uint64_t stall_ns;
 };
 
 __device__ __forceinline__ void note_fail(const Params &p, int role, int t, int kb, int site) {
@@ -149,6 +154,7 @@ struct Ctrl {
   uint64_t tempty[2];
   uint64_t tailbar[8];    // weight gradients: a stage's loads ran past the expert's rows
   uint64_t drain;
+  uint64_t never;         // the failure-detection hook's barrier: nothing ever arrives on it
   uint64_t xfull[4];      // router: one lane quarter's second-half picks are in xbuf
   uint64_t xempty[4];     // router: ... and have been merged
   uint32_t tmem_base;
@@ -374,6 +380,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int s = 0; s < C::STAGES; ++s) ptx::mbar_init(ptx::smem_u32(&c.tailbar[s]), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
+    ptx::mbar_init(ptx::smem_u32(&c.never), 1);
     for (int q = 0; q < 4; ++q) {
       ptx::mbar_init(ptx::smem_u32(&c.xfull[q]), 32);
       ptx::mbar_init(ptx::smem_u32(&c.xempty[q]), 32);
@@ -556,27 +563,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
         }
         if (tail) {
-          // the tail fixer warp zeroes the rows past the expert and releases the stage
+          // the tail fixer warp zeroes the rows past the expert and releases the stage; the
+          // copies of this fill are counted on the tail barrier, which the drain waits on
           tarmed |= 1u << stage;
           tlast = (tlast & ~(1u << stage)) | (tnext & (1u << stage));
           tnext ^= 1u << stage;
+          armed &= ~(1u << stage);
+        } else {
+          // this stage's full barrier completes (or has completed) the phase of this pass
+          armed |= 1u << stage;
+          if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
         }
-        // this stage's full barrier completes (or has completed) the phase of this pass
-        armed |= 1u << stage;
-        if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
-    // Drain: every TMA fill this warp issued must land before the CTA may exit.  (Pairs:
-    // the leader's full barriers count the peer's bytes too; the peer only has tails.)
+    // Drain: every TMA fill this warp issued must land before the CTA may exit, also after
+    // an abort (these waits ignore the abort flag and give up only at the limit).  The last
+    // fill of each stage is counted on its full barrier, or on its tail barrier for a tail
+    // fill; earlier fills of a stage had landed before the stage was refilled.  (Pairs: the
+    // leader's full barriers count the peer's bytes too; the peer only has tails.)
     if (lane == 0) {
       for (int s = 0; s < C::STAGES; ++s)
         if (rank == 0 && ((armed >> s) & 1u))
-          if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
+          if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, nullptr, WAIT_LIMIT_NS))
             note_fail(p, 0, 0, s, 2);
       for (int s = 0; s < C::STAGES; ++s)
         if (((tarmed >> s) & 1u) &&
-            !ptx::mbar_wait(ptx::smem_u32(&c.tailbar[s]), (tlast >> s) & 1u, abort_flag, WAIT_LIMIT_NS))
+            !ptx::mbar_wait(ptx::smem_u32(&c.tailbar[s]), (tlast >> s) & 1u, nullptr, WAIT_LIMIT_NS))
           note_fail(p, 0, 0, s, 3);
     }
   } else if (warp == 1) {
@@ -593,6 +606,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
+      if (CG == 1 && p.stall_ns) {
+        // failure-detection hook: a wait that nothing ends runs out, and every role aborts
+        ok = ptx::mbar_wait(ptx::smem_u32(&c.never), 0, abort_flag, p.stall_ns);
+        if (!ok) note_fail(p, 1, 0, 0, 3);
+      }
       for (int t = tile0; t < ntiles && ok; t += tstep, ++it) {
         Tile tl;
         get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
@@ -659,10 +677,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.tfull[acc]), 0x3);
         else ptx::tc_commit(ptx::smem_u32(&c.tfull[acc]));
       }
-      // Drain: all MMAs issued here complete before TMEM is freed.
+      // Drain: all MMAs issued here complete before TMEM is freed, also after an abort.
       if constexpr (CG == 2) ptx::tc_commit_pair(ptx::smem_u32(&c.drain));
       else ptx::tc_commit(ptx::smem_u32(&c.drain));
-      if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, abort_flag, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
+      if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, nullptr, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
     }
     __syncwarp();
   } else if (warp == FIX_WARP) {
@@ -1114,13 +1132,19 @@ static int sm_count() {
   return n;
 }
 
+// Failure-detection test hook (moe_debug_set_gemm_stall_ns), 0 in normal use: process-wide,
+// read at each launch, applied to single-CTA launches only.
+static std::atomic<uint64_t> g_stall_ns{0};
+
 // Persistent launch: one CTA per SM (CG = 1), or one CTA pair per two SMs in clusters
 // of two (CG = 2); never more CTAs (pairs) than tiles.
 template <typename T, int BN, int MODE, int CG = 1>
-static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p,
+static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p_in,
                   int64_t max_tiles, cudaStream_t st, const CUtensorMap *o0 = nullptr,
                   const CUtensorMap *o1 = nullptr) {
   using C = Cfg<T, BN, CG, extra_smem<MODE>()>;
+  Params p = p_in;
+  p.stall_ns = CG == 1 ? g_stall_ns.load(std::memory_order_relaxed) : 0;
   auto kern = grouped_gemm_kernel<T, BN, MODE, CG>;
   constexpr int SMEM = C::SMEM_BYTES;
   static_assert(SMEM <= SMEM_LIMIT, "shared memory");
@@ -1457,6 +1481,8 @@ static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, 
 }
 
 }  // namespace gg
+
+void set_gemm_stall_ns(uint64_t ns) { gg::g_stall_ns.store(ns, std::memory_order_relaxed); }
 
 int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float *bias, float *logits,
                      int32_t *idx, float *gate, int *err, cudaStream_t st) {

@@ -74,6 +74,12 @@ int moe_get_error(void *ws, moe_stream_t stream, int32_t *code) {
   return MOE_OK;
 }
 
+int moe_debug_set_gemm_stall_ns(uint64_t ns) {
+  if (ns > MOE_DEBUG_STALL_MAX_NS) return MOE_ERR_INVALID_ARG;
+  set_gemm_stall_ns(ns);
+  return MOE_OK;
+}
+
 int moe_route_topk(const moe_config *cfg, const void *x, const void *w_router, const float *bias,
                    float *logits, int32_t *topk_idx, float *topk_gate, void *ws, moe_stream_t stream) {
   RETURN_IF(check_cfg(cfg));

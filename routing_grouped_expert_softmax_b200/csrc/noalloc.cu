@@ -26,7 +26,9 @@ void *g_scratch_ptr[MAX_DEVICES] = {};
 
 // The array's name in host code is only a host-side handle, not a device address: the
 // kernels must be given the address cudaGetSymbolAddress returns for the current device.
-// Resolved once per device, on the first call made with that device current.
+// Resolved once per device, on the first call made with that device current, in the context
+// current then (the primary context, for callers of the runtime API); the address is only
+// valid in that context.
 int scratch_for_current_device(void **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return MOE_ERR_CUDA;

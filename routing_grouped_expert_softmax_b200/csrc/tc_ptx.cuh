@@ -45,16 +45,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` (or as soon as *abort is set by another role), sets *abort and
-// returns false.  No wait in these kernels is unbounded.
+// returns false.  abort == nullptr: a drain wait, which ignores other roles'
+// aborts (it waits for asynchronous work this thread started) and only gives up
+// at the limit.  No wait in these kernels is unbounded.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
+    if (abort && *abort) return false;
     if (globaltimer() - t0 > limit_ns) {
-      *abort = 1;
+      if (abort) *abort = 1;
       return false;
     }
   }

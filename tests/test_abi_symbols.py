@@ -134,3 +134,10 @@ def test_shared_expert_and_recompute_host_validation(lib):
     w0 = moe.LayerWeights(16, None, 16, 16, 16, None, None, None)
     assert lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(w0), 16, 16, ctypes.byref(sv), 16, None) \
         == moe.MOE_ERR_INVALID_ARG
+
+
+def test_debug_stall_hook_validates_its_limit(lib):
+    # host only: the hook is a process-wide setting read at the next launch
+    assert lib.moe_debug_set_gemm_stall_ns(2_000_000_000) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_debug_set_gemm_stall_ns(1_000_000) == moe.MOE_OK
+    assert lib.moe_debug_set_gemm_stall_ns(0) == moe.MOE_OK

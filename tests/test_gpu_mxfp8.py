@@ -7,7 +7,8 @@ import pytest
 import routing_grouped_expert_softmax_b200 as moe
 from oracle import moe_ref as ref
 from routing_grouped_expert_softmax_b200 import inputs as gen
-from tests.gpu_util import dev, dev_f32, dev_i32, grid, host, offsets_of, random_counts, rel_err
+from tests.gpu_util import (check_layer, check_logits_and_routing, dev, dev_f32, dev_i32, gpu_decided_oracle, grid,
+                             host, offsets_of, random_counts, rel_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -220,10 +221,10 @@ def test_mx_grouped_swiglu_bwd(d, f, E, kind):
         assert np.all(host(dwg[e]) == 0) and np.all(host(dwd[e]) == 0)
 
 
-def test_mx_layer_against_oracle_and_bf16_path():
+@pytest.mark.parametrize("T,d,E,k,f,skew", [(512, 256, 16, 4, 256, False), (700, 384, 8, 2, 256, True)])
+def test_mx_layer_against_oracle_and_bf16_path(T, d, E, k, f, skew):
     import torch
-    T, d, E, k, f = 512, 256, 16, 4, 256
-    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=5)
+    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=5, skew=skew)
     outs = {}
     for prec in ("native", "mxfp8"):
         cfg = moe.config(T, d, E, k, f, dtype="bf16", prec=prec)
@@ -231,33 +232,22 @@ def test_mx_layer_against_oracle_and_bf16_path():
         saved = moe.alloc_saved(cfg)
         grads = moe.alloc_grads(cfg)
         w = [dev(a_, "bf16") for a_ in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down)]
-        wts = moe.layer_weights(w[0], None, w[1], w[2], w[3])
+        bias = dev_f32(inp.bias) if inp.bias is not None else None
+        wts = moe.layer_weights(w[0], bias, w[1], w[2], w[3])
         x = dev(inp.x, "bf16")
         y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
         moe.moe_layer_fwd(cfg, wts, x, y, saved, ws)
         moe.moe_layer_bwd(cfg, wts, x, dev(inp.dy, "bf16"), saved, grads, ws)
         assert moe.moe_get_error(ws) == 0
-        outs[prec] = (host(y), {n: host(grads[n]) for n in ("dx", "dw_gate", "dw_up", "dw_down", "dw_router")},
-                      host(saved["topk_idx"]))
-    # the oracle with every GEMM operand quantised, on the routing both paths share
-    fwd = ref.layer_fwd(inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k)
-    assert np.array_equal(outs["mxfp8"][2], fwd["idx"])
-    h, u, a, y_perm = ref.grouped_swiglu_mx(fwd["x_perm"], fwd["offsets"], inp.w_gate, inp.w_up, inp.w_down)
-    Y = ref.combine(y_perm, fwd["slot_of_pair"], fwd["gate"])
-    dy_perm, dgate = ref.combine_bwd(inp.dy, y_perm, fwd["slot_of_pair"], fwd["gate"])
-    # the layer keeps h, u, a and dy_perm in bf16; the backward GEMMs quantise those tensors
-    b = ref.bf16_rne
-    g = ref.grouped_swiglu_bwd_mx(b(dy_perm), fwd["x_perm"], b(h), b(u), b(a), fwd["offsets"], inp.w_gate,
-                                  inp.w_up, inp.w_down)
-    dx = ref.unpermute_sum(g["dx_perm"], fwd["slot_of_pair"], T, k)
-    dz, dwr, dxr = ref.route_bwd(dgate, fwd["gate"], fwd["idx"], inp.x, inp.w_r)
-    want = dict(dx=dx + dxr, dw_gate=g["dw_gate"], dw_up=g["dw_up"], dw_down=g["dw_down"], dw_router=dwr)
-    ymx, gmx, _ = outs["mxfp8"]
-    assert rel_err(ymx, Y) <= TOL_MX
-    for n, ref_v in want.items():
-        assert rel_err(gmx[n], ref_v) <= TOL_MX, n
+        outs[prec] = (y, saved, grads)
+    # the oracle's MXFP8 layer (every GEMM operand quantised along its own K, the five stored
+    # tensors in bf16), on the routing decided as the GPU decides it
+    y, sv, g = outs["mxfp8"]
+    zg = check_logits_and_routing(inp, sv)
+    fwd, bwd_fn = gpu_decided_oracle(inp, zg, mx=True)
+    check_layer(y, sv, g, fwd, bwd_fn(fwd), f, TOL_MX, TOL_MX, tag="mxfp8 ")
     # and MXFP8 stays close to the bf16 path (quantisation error only)
-    ybf, gbf, _ = outs["native"]
-    assert 0 < rel_err(ymx, ybf) <= 0.1
+    ybf, _, gbf = outs["native"]
+    assert 0 < rel_err(host(y), host(ybf)) <= 0.1
     for n in ("dx", "dw_gate", "dw_down"):
-        assert rel_err(gmx[n], gbf[n]) <= 0.15, n
+        assert rel_err(host(g[n]), host(gbf[n])) <= 0.15, n

@@ -1,20 +1,21 @@
 """The shared expert and the recomputing backward through moe_layer_fwd / moe_layer_bwd.
 
 Shared expert: parity with the oracle (every output and gradient, including the shared
-expert's activations and weight gradients).  Recompute (saved h | u left out): the same
-kernels on the same inputs, so forward outputs and every gradient must equal those of the
-saving path bit for bit."""
+expert's activations and weight gradients).  Recompute (saved h | u left out): parity with
+the oracle (bf16 and MXFP8), and, since the same kernels run on the same inputs, forward
+outputs and every gradient bit for bit equal to those of the saving path."""
 import numpy as np
 import pytest
 
 import routing_grouped_expert_softmax_b200 as moe
-from oracle import moe_ref as ref
 from routing_grouped_expert_softmax_b200 import inputs as gen
-from tests.gpu_util import dev, dev_f32, host, rel_err
+from tests.gpu_util import check_layer, check_logits_and_routing, dev, dev_f32, gpu_decided_oracle, host
 
 pytestmark = pytest.mark.gpu
 
 TOL = 2e-2
+TOL_COMBINE = 1e-2
+TOL_MX = 6e-2
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -59,21 +60,9 @@ def test_layer_with_shared_expert_against_oracle(T, d, E, k, f, skew):
     inp = gen.make_layer_inputs(T, d, E, k, f, seed=T + 7, skew=skew)
     sh = gen.make_shared_expert(d, f, seed=T + 8)
     y, sv, g = _run(inp, shared=sh)
-    fwd = ref.layer_fwd(inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, k, inp.bias, shared=sh)
-    gi = host(sv["topk_idx"])
-    if not np.array_equal(gi, fwd["idx"]):
-        pytest.skip("near-tie routing differs from the fp64 oracle; the whole-layer comparison needs it equal")
-    shu = host(sv["shared_hu"])
-    assert rel_err(shu[:, :f], fwd["shared_h"]) <= TOL and rel_err(shu[:, f:], fwd["shared_u"]) <= TOL
-    assert rel_err(host(sv["shared_a"]), fwd["shared_a"]) <= TOL
-    assert rel_err(host(y), fwd["y"]) <= TOL
-    bwd = ref.layer_bwd(fwd, inp.dy, inp.x, inp.w_r, inp.w_gate, inp.w_up, inp.w_down, shared=sh)
-    sdhu = host(g["shared_dhu"])
-    assert rel_err(sdhu[:, :f], bwd["shared_dh"]) <= TOL and rel_err(sdhu[:, f:], bwd["shared_du"]) <= TOL
-    for n, key in (("dx", "dx"), ("dw_gate", "dw_gate"), ("dw_up", "dw_up"), ("dw_down", "dw_down"),
-                   ("dw_router", "dw_r"), ("dw_shared_gate", "dw_shared_gate"),
-                   ("dw_shared_up", "dw_shared_up"), ("dw_shared_down", "dw_shared_down")):
-        assert rel_err(host(g[n]), bwd[key]) <= TOL, n
+    zg = check_logits_and_routing(inp, sv)
+    fwd, bwd_fn = gpu_decided_oracle(inp, zg, shared=sh)
+    check_layer(y, sv, g, fwd, bwd_fn(fwd), f, TOL, TOL_COMBINE)
 
 
 def test_shared_expert_with_uniform_random_routing():
@@ -82,11 +71,8 @@ def test_shared_expert_with_uniform_random_routing():
     sh = gen.make_shared_expert(d, f, seed=6)
     idx, gate = gen.uniform_random_routing(T, E, k, seed=5)
     y, sv, g = _run(inp, shared=sh, routed=(idx, gate))
-    fwd = ref.layer_fwd_routed(inp.x, idx, gate, inp.w_gate, inp.w_up, inp.w_down, shared=sh)
-    bwd = ref.layer_bwd_routed(fwd, inp.dy, inp.w_gate, inp.w_up, inp.w_down, x=inp.x, shared=sh)
-    assert rel_err(host(y), fwd["y"]) <= TOL
-    for n in ("dx", "dw_gate", "dw_up", "dw_down", "dw_shared_gate", "dw_shared_up", "dw_shared_down"):
-        assert rel_err(host(g[n]), bwd[n]) <= TOL, n
+    fwd, bwd_fn = gpu_decided_oracle(inp, None, shared=sh, routed=(idx, gate))
+    check_layer(y, sv, g, fwd, bwd_fn(fwd), f, TOL, TOL_COMBINE)
 
 
 @pytest.mark.parametrize("T,d,E,k,f,shared,prec", [
@@ -94,13 +80,23 @@ def test_shared_expert_with_uniform_random_routing():
     (1100, 256, 4, 2, 128, True, "native"),
     (300, 128, 128, 4, 128, True, "native"),
     (256, 256, 8, 2, 256, True, "mxfp8"),
+    (700, 256, 16, 4, 256, False, "mxfp8"),
 ])
-def test_recompute_equals_saving_bit_for_bit(T, d, E, k, f, shared, prec):
+def test_recompute_against_oracle_and_saving_path(T, d, E, k, f, shared, prec):
+    """The recomputing backward against the oracle, and bit for bit against the saving path
+    (the same kernels on the same inputs)."""
     inp = gen.make_layer_inputs(T, d, E, k, f, seed=T + 1)
     sh = gen.make_shared_expert(d, f, seed=T + 2) if shared else None
     y0, s0, g0 = _run(inp, shared=sh, prec=prec)
     y1, s1, g1 = _run(inp, shared=sh, recompute=True, prec=prec)
     assert s1["hu"] is None and s1["shared_hu"] is None
+    # against the oracle (the MXFP8 layer's oracle for prec="mxfp8")
+    mx = prec == "mxfp8"
+    zg = check_logits_and_routing(inp, s1)
+    fwd, bwd_fn = gpu_decided_oracle(inp, zg, shared=sh, mx=mx)
+    tol, tol_c = (TOL_MX, TOL_MX) if mx else (TOL, TOL_COMBINE)
+    check_layer(y1, s1, g1, fwd, bwd_fn(fwd), f, tol, tol_c, tag="recompute ")
+    # and bit for bit against the path that keeps h | u
     assert np.array_equal(host(y0), host(y1))
     for n in ("a", "y_perm", "x_perm") + (("shared_a",) if shared else ()):
         assert np.array_equal(host(s0[n]), host(s1[n])), n
