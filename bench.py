@@ -221,6 +221,23 @@ class Layer:
                 "empty_experts": int((c == 0).sum()), "counts": c.tolist()}
 
 
+def profiled_launches(step):
+    """Kernels of this library (namespace moe) that one step launches, counted by CUPTI through
+    torch.profiler on one untimed step; None if the profiler is unavailable."""
+    import torch
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            step()
+            torch.cuda.synchronize()
+        names = [e.name for e in prof.events() if e.device_type == torch.autograd.DeviceType.CUDA]
+        n = sum(1 for nm in names if "moe::" in nm)
+        return n if n > 0 else None
+    except Exception:
+        return None
+
+
 def time_steps(layer, steps, warmup, barrier):
     """Device time of `steps` back-to-back steps (CUDA events on the launching stream), ms per step."""
     import torch
@@ -290,6 +307,9 @@ def run_ours(args):
     ms_max = max_over_ranks(e0.elapsed_time(e1) / args.steps, "cuda")
     peak_mem = torch.cuda.max_memory_allocated() - base_mem
     load = L.load()
+    counted = None if args.no_cupti else profiled_launches(step)
+    if counted is not None:
+        launches_per_step = counted
 
     # ---- step-time spread: up to 50 more steps, each between its own pair of events
     n_spread = min(args.steps, 50)
@@ -452,6 +472,8 @@ def run_ours(args):
         "e2e": {"value": job_tokens_per_s(T, ws_n, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": 2 * T * d * 2, "d2h_bytes_per_step": 2 * T * d * 2},
         "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches_per_step": launches_per_step,
+        "gpu_launches_source": "CUPTI count of one untimed step" if counted is not None else "formula",
         "clocks": clk.summary(),
         "load": load,
         "memory": {"peak_gib": peak_mem / 2 ** 30, "layer_buffers_gib": layer_gib,
@@ -516,20 +538,24 @@ def gemm_algorithmic_bytes(P, d, f, E, prec):
 
 
 def count_launches(routing, prec="native", shared=False, recompute=False):
-    """Kernels one step launches: forward (router 1, metadata 3, permute 1, grouped GEMMs 2,
-    combine 1) and backward (combine-bwd 1, grouped GEMMs 4, router transpose 1, router
-    weight-gradient 3, unpermute-sum 1); MXFP8 adds 4 quantisers forward, 8 backward.  A
-    shared expert adds its group offsets and 2 GEMMs forward, offsets and 4 GEMMs backward
-    (MXFP8: 4 + 8 more quantisers); recompute adds one GEMM per expert set backward (MXFP8:
-    with its 2 quantisers)."""
+    """Kernels one step launches (the fallback when the CUPTI count is unavailable): forward
+    (router 1, metadata 3, permute 1, grouped GEMMs 2, combine 1) and backward (combine-bwd 1,
+    grouped GEMMs 4, router transpose 1, router weight-gradient 3, unpermute-sum 1).  MXFP8
+    with the forward's weight copies kept for the backward adds 2 weight quantisers forward
+    (the permute and the gate/up epilogue quantise x and a) and 2 token-axis quantisers
+    backward (the combine's backward and the down projection's epilogue quantise dy and
+    [dh | du]).  A shared expert adds its group offsets and 2 GEMMs forward, offsets and 4
+    GEMMs backward (MXFP8: its operands through 3 + 7 quantisers); recompute adds one GEMM per
+    expert set backward (MXFP8: with the quantiser of its input)."""
     fwd = (1 if routing == "router" else 0) + 3 + 1 + 2 + 1
     bwd = 1 + 4 + (5 if routing == "router" else 1)
-    n = fwd + bwd + (12 if prec == "mxfp8" else 0)
+    mx = prec == "mxfp8"
+    n = fwd + bwd + (4 if mx else 0)
     sets = 2 if shared else 1
     if shared:
-        n += 1 + 2 + 1 + 4 + (12 if prec == "mxfp8" else 0)
+        n += 1 + 2 + 1 + 4 + (10 if mx else 0)
     if recompute:
-        n += sets * (1 + (2 if prec == "mxfp8" else 0))
+        n += sets * (1 + (1 if mx else 0))
     return n
 
 
@@ -647,6 +673,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="time the main workload only")
+    ap.add_argument("--no-cupti", action="store_true",
+                    help="count launches by formula, not with the CUDA profiler (e.g. under ncu)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

@@ -96,6 +96,10 @@ typedef struct moe_config {
  * (cudaMemset) before its first use; the library keeps it consistent after. */
 MOE_API size_t moe_workspace_size(const moe_config *cfg);
 
+/* (the pages have no counterpart: calling-convention plumbing)
+ * Bytes of moe_layer_saved.mx_saved for this config: 0 unless prec is MOE_PREC_MXFP8. */
+MOE_API size_t moe_mx_saved_bytes(const moe_config *cfg);
+
 /* (the pages have no counterpart: error reporting)
  * Synchronise `stream`, then report and clear the device error word in `ws`.
  * *code receives 0 or an OR of MOE_ERR_DEVICE_* bits. */
@@ -305,6 +309,12 @@ typedef struct moe_layer_saved {
   void *y_perm;           /* [P,d] */
   void *shared_hu;        /* [T,2f] with a shared expert, or NULL: recomputed */
   void *shared_a;         /* [T,f] with a shared expert */
+  /* MOE_PREC_MXFP8 only, or NULL: moe_mx_saved_bytes(cfg) bytes (256-byte aligned) that the
+   * forward fills with MXFP8 copies (E4M3 codes with E8M0 scales, the layout is internal) the
+   * backward reads instead of quantising again: the routed experts' weights in the orientation
+   * of every GEMM that reads them, and x_perm and a along the token axis.  The weights must not
+   * change between the two calls.  NULL: each call quantises what it needs in the workspace. */
+  void *mx_saved;
 } moe_layer_saved;
 
 /* Outputs of the backward, plus its intermediates (caller-owned). */

@@ -36,7 +36,7 @@ EXPORTED = [
     "moe_build_offsets", "moe_build_offsets_noalloc", "moe_permute", "moe_grouped_swiglu_fwd", "moe_grouped_swiglu_bwd",
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
     "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd", "moe_mx_quantize_rows",
-    "moe_mx_quantize_cols", "moe_permute_mxfp8", "moe_debug_set_gemm_stall_ns",
+    "moe_mx_quantize_cols", "moe_permute_mxfp8", "moe_debug_set_gemm_stall_ns", "moe_mx_saved_bytes",
 ]
 
 
@@ -53,7 +53,7 @@ class MoeConfig(ctypes.Structure):
 WEIGHT_FIELDS = ("w_router", "bias", "w_gate", "w_up", "w_down", "w_shared_gate", "w_shared_up",
                  "w_shared_down")
 SAVED_FIELDS = ("logits", "topk_idx", "topk_gate", "counts", "offsets", "slot_of_pair",
-                "pair_of_slot", "x_perm", "hu", "a", "y_perm", "shared_hu", "shared_a")
+                "pair_of_slot", "x_perm", "hu", "a", "y_perm", "shared_hu", "shared_a", "mx_saved")
 GRAD_FIELDS = ("dx", "dw_router", "dw_gate", "dw_up", "dw_down", "dy_perm", "dgate", "dhu",
                "dx_perm", "dw_shared_gate", "dw_shared_up", "dw_shared_down", "shared_dhu")
 
@@ -91,6 +91,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         sig = {
             "moe_workspace_size": (ctypes.c_size_t, [_CFG]),
+            "moe_mx_saved_bytes": (ctypes.c_size_t, [_CFG]),
             "moe_get_error": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int32)]),
             "moe_debug_set_gemm_stall_ns": (ctypes.c_int, [ctypes.c_uint64]),
             "moe_route_topk": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, _P, _P, _P]),
@@ -156,6 +157,10 @@ def config(T, d, E, k, f, dtype="bf16", prec="native") -> MoeConfig:
 
 def moe_workspace_size(cfg: MoeConfig) -> int:
     return lib().moe_workspace_size(ctypes.byref(cfg))
+
+
+def moe_mx_saved_bytes(cfg: MoeConfig) -> int:
+    return lib().moe_mx_saved_bytes(ctypes.byref(cfg))
 
 
 def moe_get_error(ws, stream=None) -> int:
@@ -289,9 +294,10 @@ def alloc_workspace(cfg, device="cuda"):
     return torch.zeros(max(moe_workspace_size(cfg), 256), dtype=torch.uint8, device=device)
 
 
-def alloc_saved(cfg, device="cuda", logits=True, shared=False, recompute=False) -> dict:
+def alloc_saved(cfg, device="cuda", logits=True, shared=False, recompute=False, mx_saved=True) -> dict:
     """Forward buffers.  shared: room for a shared expert's activations; recompute: keep no
-    [h | u] (the backward recomputes them), which leaves hu (and shared_hu) None."""
+    [h | u] (the backward recomputes them), which leaves hu (and shared_hu) None; mx_saved
+    (MXFP8 only): keep the weights' MXFP8 copies from the forward for the backward."""
     import torch
     dt = torch_dtype(cfg)
     T, d, E, k, f, P = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.T * cfg.k
@@ -309,6 +315,8 @@ def alloc_saved(cfg, device="cuda", logits=True, shared=False, recompute=False) 
         y_perm=torch.empty(P, d, dtype=dt, device=device),
         shared_hu=torch.empty(T, 2 * f, dtype=dt, device=device) if shared and keep_hu else None,
         shared_a=torch.empty(T, f, dtype=dt, device=device) if shared else None,
+        mx_saved=(torch.empty(moe_mx_saved_bytes(cfg), dtype=torch.uint8, device=device)
+                  if mx_saved and cfg.prec == MOE_PREC_MXFP8 else None),
     )
 
 

@@ -59,7 +59,10 @@ struct WsLayout {
 };
 // bytes of an MXFP8 operand [rows][cols] with scales along the row / down the rows
 inline size_t mx_bytes_r(int64_t rows, int64_t cols) { return align_up((size_t)(rows * cols + rows * (cols / 32)), 256); }
-inline size_t mx_bytes_t(int64_t rows, int64_t cols) { return align_up((size_t)(rows * cols + (rows / 32) * cols), 256); }
+// (token-axis scales in the GEMMs' tile layout cover the rows rounded up to 128)
+inline size_t mx_bytes_t(int64_t rows, int64_t cols) {
+  return align_up((size_t)(rows * cols + ((rows + 127) / 128) * 4 * cols), 256);
+}
 constexpr int RB_SPLIT = 16;          // token splits of the router weight-gradient reduction
 
 
@@ -92,6 +95,30 @@ inline WsLayout ws_layout(const Shape &s) {
     L.wgu_r = off;  off += mx_bytes_r(ed, 2 * s.f);
   }
   L.group_offsets = off; off += 256;   // {0, T}: the shared expert's single group
+  L.total = off;
+  return L;
+}
+
+// Layout of moe_layer_saved.mx_saved: the routed experts' weights in MXFP8 in the four
+// orientations the grouped GEMMs read, and the layer input x_perm and the activation a in
+// MXFP8 down the expert-padded token axis (the weight-gradient GEMMs' operands), each as
+// codes then scales in the GEMMs' tile layout.
+struct MxSavedLayout {
+  size_t wgu_c, wd_c, wd_r, wgu_r;   // as the workspace's regions of the same names
+  size_t xq_t, aq_t;                 // [Ppad][d], [Ppad][f]
+  size_t total;
+};
+inline MxSavedLayout mx_saved_layout(const Shape &s) {
+  MxSavedLayout L{};
+  if (s.prec != MOE_PREC_MXFP8) return L;
+  const int64_t ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f, R = s.Ppad();
+  size_t off = 0;
+  L.wgu_c = off; off += mx_bytes_t(ed, 2 * s.f);
+  L.wd_c = off;  off += mx_bytes_t(ef, s.d);
+  L.wd_r = off;  off += mx_bytes_r(ef, s.d);
+  L.wgu_r = off; off += mx_bytes_r(ed, 2 * s.f);
+  L.xq_t = off;  off += mx_bytes_t(R, s.d);
+  L.aq_t = off;  off += mx_bytes_t(R, s.f);
   L.total = off;
   return L;
 }
@@ -160,8 +187,22 @@ cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const i
 cudaError_t launch_group_offsets(int32_t *o, int64_t T, cudaStream_t st);
 // FP8 dispatch: the permute that also writes each routed row in MXFP8 (blocks of 32 along d)
 // into the expert buffers padded to 128 rows (bf16 storage, d % 32 == 0)
+// tiled: scales in the block-scaled GEMMs' tile layout (quant.cu) instead of the plain one
 cudaError_t launch_mx_permute(const void *x, const int32_t *sop, const int32_t *offsets, int E, int64_t T, int k,
-                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st);
+                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st,
+                              bool tiled = false);
+// The combine's backward for the MXFP8 layer (bf16 storage, d % 128 == 0): dy_perm, dgate as
+// launch_combine_bwd, and dy_perm in MXFP8 along d (codes_r) and down the expert-padded token
+// axis (codes_c), scales in the GEMMs' tile layout; pos = pair_of_slot; rows_bound = Ppad.
+cudaError_t launch_mx_combine_bwd(const void *dy, const void *y_perm, const int32_t *pos, const int32_t *offsets,
+                                  const float *gate, int E, int k, int d, int64_t rows_bound, void *dy_perm,
+                                  float *dgate, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
+                                  uint8_t *scales_c, cudaStream_t st);
+// FP8 dispatch, slot-major: x_perm (a bit copy of each routed row) and x_perm in MXFP8 along d
+// (codes_r) and down the expert-padded token axis (codes_c), scales in the GEMMs' tile layout.
+cudaError_t launch_mx_dispatch(const void *x, const int32_t *pos, const int32_t *offsets, int E, int k, int d,
+                               int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r,
+                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st);
 cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm,
                                const int32_t *sop, const float *gate, void *dy_perm,
                                float *dgate, cudaStream_t st);
@@ -177,26 +218,44 @@ cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, cons
 cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
                                 const int32_t *idx, const void *x, float *partial,
                                 float *dw_r, cudaStream_t st);
-// x_quantized (MXFP8 only): the workspace already holds x_perm's MXFP8 rows, written by
-// launch_mx_permute into the layout ws_layout(s) gives them.
+// MXFP8 only:
+//   x_quantized: the workspace already holds x_perm's MXFP8 rows, written by
+//     launch_mx_permute into the layout ws_layout(s) gives them;
+//   wsaved (layout mx_saved_layout(s)) or nullptr: the weights' MXFP8 copies; wfill: the
+//     forward writes all four orientations there (else it reads the ones it needs).
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets,
                        const void *w_gate, const void *w_up, const void *w_down, void *hu,
-                       void *a, void *y_perm, void *ws, cudaStream_t st, bool x_quantized = false);
+                       void *a, void *y_perm, void *ws, cudaStream_t st, bool x_quantized = false,
+                       uint8_t *wsaved = nullptr, bool wfill = false);
 // dst[b][c][r] = src[b][r][c] (fp32)
 cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R, int C, cudaStream_t st);
 // MXFP8 quantisers (quant.cu).  offsets != nullptr: source rows are expert groups written
 // into buffers padded to 128 rows per expert (rows_bound: rows the buffer holds).
+// tiled: scales in the tile layout the block-scaled GEMMs read (needs K % 128 == 0 along rows).
 cudaError_t launch_mx_quant_rows(const void *src, int64_t R, int K, const int32_t *offsets, int E, int64_t rows_bound,
-                                 uint8_t *codes, uint8_t *scales, cudaStream_t st);
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st, bool tiled = false);
 cudaError_t launch_mx_quant_cols(const void *src, int64_t R, int C, const int32_t *offsets, int E, int64_t rows_bound,
-                                 uint8_t *codes, uint8_t *scales, cudaStream_t st);
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st, bool tiled = false);
 cudaError_t launch_mx_quant_cols_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
-                                    uint8_t *scales, cudaStream_t st);
+                                    uint8_t *scales, cudaStream_t st, bool tiled = false);
 cudaError_t launch_mx_quant_rows_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
-                                    uint8_t *scales, cudaStream_t st);
+                                    uint8_t *scales, cudaStream_t st, bool tiled = false);
+// Expert weights in both MXFP8 orientations from one read, scales in the tile layout:
+// gu: (w0, w1) = (W_gate, W_up) [R = E*d][C = f] -> codes_c [R][2f] (blocks down the rows, gate
+// and up interleaved in 64-column chunks) and codes_r [R][2f] (row r = [W_gate[r] | W_up[r]],
+// blocks along it); else w0 = W_down [R = E*f][C = d] -> codes_c, codes_r [R][C].  R % 128 == 0,
+// C % 128 == 0.
+cudaError_t launch_mx_quant_weights(const void *w0, const void *w1, int64_t R, int C, bool gu, uint8_t *codes_c,
+                                    uint8_t *scales_c, uint8_t *codes_r, uint8_t *scales_r, cudaStream_t st);
+// MXFP8 only:
+//   wsaved: the weights' MXFP8 copies a forward wrote (layout mx_saved_layout(s)), read
+//     instead of quantising the weights again; nullptr: quantised here, in the workspace;
+//   dy_quantized: the workspace already holds dy_perm's MXFP8 copies in both orientations
+//     (written by launch_mx_combine_bwd into the layout ws_layout(s) gives them).
 int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                        const void *a, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *dhu, void *dx_perm,
-                       void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st);
+                       void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st,
+                       const uint8_t *wsaved = nullptr, bool dy_quantized = false);
 
 }  // namespace moe

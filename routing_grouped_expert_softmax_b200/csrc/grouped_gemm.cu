@@ -36,6 +36,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "mxfp8.cuh"
 #include "tc_ptx.cuh"
 
 namespace moe {
@@ -119,11 +120,19 @@ struct Params {
   void *out2;
   const void *aux;
   int k;       // router: experts per token
-  // MXFP8 scale factors: K-major operands [rows][K/32] (ld = K/32), MN-major operands
-  // [K/32][MN] (ld = MN)
+  // MXFP8 scale factors in the tile layout the quantisers write (tiles of 128 M or N indices
+  // by 4 K-blocks, 512 bytes, in the arrangement of tcgen05.cp's 32x128b.warpx4 copy); the
+  // tile of (MN block b, K group g) is at (b * nk + g) * 512, nk = the operand's K extent in
+  // groups of 128 elements
   const uint8_t *sfa;
   const uint8_t *sfb;
-  int sfa_ld, sfb_ld;
+  int nka, nkb;
+  // MXFP8 epilogues that quantise their own bf16 output for the next GEMMs (nullptr: none),
+  // rows padded to 128 per expert as the row-grouped MXFP8 GEMMs index them, scales in the
+  // tile layout: q_row* blocks of 32 along the row (nk_row = K groups of a row), q_col*
+  // blocks of 32 down the rows (nk_col = K groups of the padded token axis)
+  uint8_t *q_row_codes, *q_row_scales, *q_col_codes, *q_col_scales;
+  int nk_row, nk_col;
   int *err;
   int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
   // Failure-detection test hook, 0 in normal use: the MMA issuer of a single-CTA launch first
@@ -294,32 +303,6 @@ __device__ __forceinline__ void load32(const T *src, float (&v)[32]) {
 
 __device__ __forceinline__ float sigmoidf_(float h) { return 1.0f / (1.0f + __expf(-h)); }
 
-// MXFP8 scale blocks in shared memory: 128 rows (or columns) x 4 K-blocks in 512 bytes,
-// row m's four scales forming the 32-bit word at byte 16*(m%32) + 4*(m/32).  Lane l of the
-// producer warp builds the 16 bytes at 16*l (rows l, l+32, l+64, l+96).
-// K-major operand: scales [rows][ld], the stage's four bytes of row m at (rowbase+m)*ld + 4*kb.
-__device__ __forceinline__ void sf_gather_kmajor(const uint8_t *sf, int64_t rowbase, int ld, int kb, uint8_t *dst,
-                                                 int lane) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-    w[i] = __ldg(reinterpret_cast<const uint32_t *>(sf + (rowbase + lane + 32 * i) * ld + 4 * kb));
-  *reinterpret_cast<uint4 *>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-// MN-major operand: scales [K/32][ld], K-block kblk+kc of column colbase+m at (kblk+kc)*ld + colbase + m.
-__device__ __forceinline__ void sf_gather_mnmajor(const uint8_t *sf, int64_t kblk, int ld, int64_t colbase,
-                                                  uint8_t *dst, int lane) {
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t v = 0;
-#pragma unroll
-    for (int kc = 0; kc < 4; ++kc) v |= (uint32_t)__ldg(sf + (kblk + kc) * ld + colbase + lane + 32 * i) << (8 * kc);
-    w[i] = v;
-  }
-  *reinterpret_cast<uint4 *>(dst + 16 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // Router order key: an unsigned 32-bit number that grows with the logit (-0 counts as +0),
 // 1 for NaN (below every number) and 0 for "no expert".  Among equal keys the lower expert
 // index ranks first.
@@ -369,9 +352,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // ------------------------------------------------------------------ prologue
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
-      // MXFP8: a second arrival once the producer warp has written the stage's scales
-      // pairs: one arrival, the leader's arrive.expect_tx for both CTAs' bytes
-      ptx::mbar_init(ptx::smem_u32(&c.full[s]), C::MX ? 2 : 1);
+      // one arrival: the producer's arrive.expect_tx (pairs: the leader's, for both CTAs' bytes)
+      ptx::mbar_init(ptx::smem_u32(&c.full[s]), 1);
       ptx::mbar_init(ptx::smem_u32(&c.empty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -474,7 +456,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         };
         if (lane == 0) {
           if (tail) ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-          else if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES);
+          else if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES + C::SF_BYTES);
+          if constexpr (C::MX) {
+            // the stage's scale-factor tiles, A then B (512 bytes each), straight into the
+            // arrangement the MMA issuer's tcgen05.cp reads
+            int64_t a_mn, a_kg, b_mn, b_kg;
+            if constexpr (MT::A_MN) { a_mn = tl.m_blk; a_kg = tl.row0 / 128 + kb; }
+            else { a_mn = tl.row0 / 128; a_kg = kb; }
+            if constexpr (MODE == FWD_GU || MODE == FWD_DOWN) {
+              b_mn = (int64_t)tl.n_blk * BN / 128; b_kg = (int64_t)tl.e * p.K / 128 + kb;
+            } else if constexpr (MODE == DGRAD_DOWN) {
+              b_mn = ((int64_t)tl.e * p.f + (int64_t)tl.n_blk * BN) / 128; b_kg = kb;
+            } else if constexpr (MODE == DGRAD_GU) {
+              b_mn = ((int64_t)tl.e * p.d + (int64_t)tl.n_blk * BN) / 128; b_kg = kb;
+            } else {
+              b_mn = (int64_t)tl.n_blk * BN / 128; b_kg = tl.row0 / 128 + kb;
+            }
+            const uint32_t sf_dst = ptx::smem_u32(sf_ring + stage * C::SF_BYTES);
+            ptx::bulk_load(sf_dst, p.sfa + (a_mn * p.nka + a_kg) * 512, 512, full_local);
+            ptx::bulk_load(sf_dst + 512, p.sfb + (b_mn * p.nkb + b_kg) * 512, 512, full_local);
+          }
           // ---- A
           if constexpr (MT::A_MN) {
 #pragma unroll
@@ -537,30 +538,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             for (int i = 0; i < BNC / C::BOX_MN; ++i)
               ld(b_dst + i * C::BOX_BYTES, &tmB0, tl.n_blk * BN + rank * BNC + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
           }
-        }
-        if constexpr (C::MX) {
-          // this stage's scales: A then B, 512 bytes each
-          uint8_t *sfa_s = sf_ring + stage * C::SF_BYTES;
-          uint8_t *sfb_s = sfa_s + 512;
-          if constexpr (MT::A_MN)
-            sf_gather_mnmajor(p.sfa, (tl.row0 + kb * C::KBLK) / 32, p.sfa_ld, (int64_t)tl.m_blk * BM, sfa_s, lane);
-          else
-            sf_gather_kmajor(p.sfa, tl.row0, p.sfa_ld, kb, sfa_s, lane);
-          if constexpr (MODE == FWD_GU)
-            sf_gather_mnmajor(p.sfb, ((int64_t)tl.e * p.K + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN,
-                              sfb_s, lane);
-          else if constexpr (MODE == FWD_DOWN)
-            sf_gather_mnmajor(p.sfb, ((int64_t)tl.e * p.K + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN,
-                              sfb_s, lane);
-          else if constexpr (MODE == DGRAD_DOWN)
-            sf_gather_kmajor(p.sfb, (int64_t)tl.e * p.f + tl.n_blk * BN, p.sfb_ld, kb, sfb_s, lane);
-          else if constexpr (MODE == DGRAD_GU)
-            sf_gather_kmajor(p.sfb, (int64_t)tl.e * p.d + tl.n_blk * BN, p.sfb_ld, kb, sfb_s, lane);
-          else
-            sf_gather_mnmajor(p.sfb, (tl.row0 + kb * C::KBLK) / 32, p.sfb_ld, (int64_t)tl.n_blk * BN, sfb_s, lane);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(ptx::smem_u32(&c.full[stage]));
         }
         if (tail) {
           // the tail fixer warp zeroes the rows past the expert and releases the stage; the
@@ -952,6 +929,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) a[i] = valid ? h[i] * sigmoidf_(h[i]) * u[i] : 0.f;
             store_slab(aa + srow * p.f + col, p.f, nvalid, a);
+            if constexpr (C::MX) {
+              if (p.q_row_codes) {
+                // the down projection's operand: the stored bf16 a, in MXFP8 along f, at the
+                // padded row (pad rows hold zeros)
+                const int64_t prow = (int64_t)tl.row0 + r;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) a[i] = __bfloat162float(__float2bfloat16_rn(a[i]));
+                mx_block32_store(a, p.q_row_codes + prow * p.f + col,
+                                 p.q_row_scales + sf_tiled_off(prow, col / 32, p.nk_row));
+                if (p.q_col_codes)   // and down the padded token axis (the weight gradient's operand)
+                  mx_slab32_cols_store(a, p.q_col_codes + prow * p.f + col,
+                                       p.q_col_scales + sf_tiled_off(col + lane, prow / 32, p.nk_col));
+              }
+            }
           }
         }
       } else if constexpr (MODE == FWD_DOWN || MODE == DGRAD_GU) {
@@ -1010,6 +1001,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int col = tl.n_blk * BN + cc;
           store_slab(dhu + srow * 2 * p.f + col, 2 * p.f, nvalid, dh);
           store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
+          if constexpr (C::MX) {
+            if (p.q_row_codes) {
+              // the gate/up GEMMs' operand: the stored bf16 [dh | du] in MXFP8 along 2f (for the
+              // data gradient) and down the padded token axis (for the weight gradient); pad
+              // rows hold zeros
+              const int64_t prow = (int64_t)tl.row0 + r;
+              const int64_t ld = 2 * p.f;
+#pragma unroll
+              for (int i = 0; i < 32; ++i) {
+                dh[i] = valid ? __bfloat162float(__float2bfloat16_rn(dh[i])) : 0.f;
+                du[i] = valid ? __bfloat162float(__float2bfloat16_rn(du[i])) : 0.f;
+              }
+              mx_block32_store(dh, p.q_row_codes + prow * ld + col,
+                               p.q_row_scales + sf_tiled_off(prow, col / 32, p.nk_row));
+              mx_block32_store(du, p.q_row_codes + prow * ld + p.f + col,
+                               p.q_row_scales + sf_tiled_off(prow, (p.f + col) / 32, p.nk_row));
+              const int64_t kb = prow / 32;   // every lane of the warp: the same 32-row block
+              mx_slab32_cols_store(dh, p.q_col_codes + prow * ld + col,
+                                   p.q_col_scales + sf_tiled_off(col + lane, kb, p.nk_col));
+              mx_slab32_cols_store(du, p.q_col_codes + prow * ld + p.f + col,
+                                   p.q_col_scales + sf_tiled_off(p.f + col + lane, kb, p.nk_col));
+            }
+          }
         }
       } else {  // weight gradients: rows q*32.. of the [M x N] block of expert e
         // Each 32 x 64 piece goes through one of the warp's two staging boxes in the layout
@@ -1385,19 +1399,37 @@ static MxOp mx_r(void *ws, size_t off, int64_t rows, int64_t cols) {
   return {b, b + rows * cols};
 }
 
-// Forward with both operands of both GEMMs quantised to MXFP8 (blocks along K).
+// Forward with both operands of both GEMMs quantised to MXFP8 (blocks along K).  Every
+// quantiser writes its scales in the tile layout the GEMMs fetch with bulk copies.
 static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
-                       cudaStream_t st, bool x_quantized) {
+                       cudaStream_t st, bool x_quantized, uint8_t *wsaved, bool wfill) {
   const WsLayout L = ws_layout(s);
   const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
   const MxOp xq = mx_r(ws, L.xq_r, R, s.d), aq = mx_r(ws, L.aq_r, R, s.f);
-  const MxOp wgu = mx_r(ws, L.wgu_c, ed, 2 * s.f), wd = mx_r(ws, L.wd_c, ef, s.d);
   // x_quantized: the FP8 dispatch (launch_mx_permute) already wrote xq's rows
-  if ((!x_quantized && launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st)) ||
-      launch_mx_quant_cols_gu(w_gate, w_up, ed, s.f, wgu.codes, wgu.scales, st) ||
-      (y_perm && launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st)))
+  if (!x_quantized && launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st, true))
     return MOE_ERR_CUDA;
+  MxOp wgu, wd;
+  if (wsaved) {
+    // the caller's buffer: every orientation from one read of each weight (wfill), or the
+    // copies an earlier forward wrote there
+    const MxSavedLayout M = mx_saved_layout(s);
+    wgu = mx_r(wsaved, M.wgu_c, ed, 2 * s.f);
+    wd = mx_r(wsaved, M.wd_c, ef, s.d);
+    const MxOp wgur = mx_r(wsaved, M.wgu_r, ed, 2 * s.f), wdr = mx_r(wsaved, M.wd_r, ef, s.d);
+    if (wfill && (launch_mx_quant_weights(w_gate, w_up, ed, s.f, true, wgu.codes, wgu.scales, wgur.codes,
+                                          wgur.scales, st) ||
+                  launch_mx_quant_weights(w_down, nullptr, ef, s.d, false, wd.codes, wd.scales, wdr.codes,
+                                          wdr.scales, st)))
+      return MOE_ERR_CUDA;
+  } else {
+    wgu = mx_r(ws, L.wgu_c, ed, 2 * s.f);
+    wd = mx_r(ws, L.wd_c, ef, s.d);
+    if (launch_mx_quant_cols_gu(w_gate, w_up, ed, s.f, wgu.codes, wgu.scales, st, true) ||
+        (y_perm && launch_mx_quant_cols(w_down, ef, s.d, nullptr, s.E, ef, wd.codes, wd.scales, st, true)))
+      return MOE_ERR_CUDA;
+  }
   int *err = err_word(ws);
   Params p{};
   p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
@@ -1407,28 +1439,46 @@ static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offset
   if (!make_tmap(&tA, xq.codes, 1, s.d, R, 128, BM) || !make_tmap(&tB, wgu.codes, 1, 2 * s.f, ed, 128, 128))
     return MOE_ERR_CUDA;
   p.K = s.d; p.N = 2 * s.f; p.out0 = hu; p.out1 = a;
-  p.sfa = xq.scales; p.sfa_ld = s.d / 32; p.sfb = wgu.scales; p.sfb_ld = 2 * s.f;
+  p.sfa = xq.scales; p.nka = s.d / 128; p.sfb = wgu.scales; p.nkb = (int)(ed / 128);
+  if (a && y_perm) {
+    // the epilogue also writes a in MXFP8 along f, the down projection's operand, and (into
+    // the caller's buffer, for the backward) down the padded token axis
+    p.q_row_codes = aq.codes; p.q_row_scales = aq.scales; p.nk_row = s.f / 128;
+    if (wsaved && wfill) {
+      const MxOp aqt = mx_r(wsaved, mx_saved_layout(s).aq_t, R, s.f);
+      p.q_col_codes = aqt.codes; p.q_col_scales = aqt.scales; p.nk_col = (int)((R + 127) / 128);
+    }
+  }
   int rc = launch<e4m3, 128, FWD_GU>(tA, tB, tB, p, mblocks * (p.N / 128), st);
+  p.q_row_codes = p.q_row_scales = p.q_col_codes = p.q_col_scales = nullptr;
   if (rc || !y_perm) return rc;   // no y_perm: [h | u] only (the backward's recompute)
   // GEMM 2: y_perm = a Wd
-  if (launch_mx_quant_rows(a, P, s.f, offsets, s.E, R, aq.codes, aq.scales, st)) return MOE_ERR_CUDA;
   if (!make_tmap(&tA, aq.codes, 1, s.f, R, 128, BM) || !make_tmap(&tB, wd.codes, 1, s.d, ef, 128, 128))
     return MOE_ERR_CUDA;
   p.K = s.f; p.N = s.d; p.out0 = y_perm; p.out1 = nullptr;
-  p.sfa = aq.scales; p.sfa_ld = s.f / 32; p.sfb = wd.scales; p.sfb_ld = s.d;
+  p.sfa = aq.scales; p.nka = s.f / 128; p.sfb = wd.scales; p.nkb = (int)(ef / 128);
   return launch<e4m3, 128, FWD_DOWN>(tA, tB, tB, p, mblocks * (p.N / 128), st);
 }
 
 // Backward with every GEMM operand quantised to MXFP8 along that GEMM's own K.
 static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu, const void *a,
                        const int32_t *offsets, const void *w_gate, const void *w_up, const void *w_down, void *dhu,
-                       void *dx_perm, void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st) {
+                       void *dx_perm, void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st,
+                       const uint8_t *wsaved, bool dy_quantized) {
   const WsLayout L = ws_layout(s);
   const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
+  const int nkt = (int)((R + 127) / 128);   // K groups of the token-axis operands
   const MxOp dyq = mx_r(ws, L.dyq_r, R, s.d), dhuq = mx_r(ws, L.dhuq_r, R, 2 * s.f);
-  const MxOp xqt = mx_r(ws, L.xq_t, R, s.d), aqt = mx_r(ws, L.aq_t, R, s.f);
+  // the token-axis copies of x_perm and a: from the forward when it kept them
+  uint8_t *wsv0 = const_cast<uint8_t *>(wsaved);
+  const MxOp xqt = wsaved ? mx_r(wsv0, mx_saved_layout(s).xq_t, R, s.d) : mx_r(ws, L.xq_t, R, s.d);
+  const MxOp aqt = wsaved ? mx_r(wsv0, mx_saved_layout(s).aq_t, R, s.f) : mx_r(ws, L.aq_t, R, s.f);
   const MxOp dyqt = mx_r(ws, L.dyq_t, R, s.d), dhuqt = mx_r(ws, L.dhuq_t, R, 2 * s.f);
-  const MxOp wdr = mx_r(ws, L.wd_r, ef, s.d), wgur = mx_r(ws, L.wgu_r, ed, 2 * s.f);
+  // the weights' data-gradient orientations: from the forward's copies when given
+  const MxSavedLayout M = mx_saved_layout(s);
+  uint8_t *wsv = const_cast<uint8_t *>(wsaved);
+  const MxOp wdr = wsaved ? mx_r(wsv, M.wd_r, ef, s.d) : mx_r(ws, L.wd_r, ef, s.d);
+  const MxOp wgur = wsaved ? mx_r(wsv, M.wgu_r, ed, 2 * s.f) : mx_r(ws, L.wgu_r, ed, 2 * s.f);
   int *err = err_word(ws);
   Params p{};
   p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
@@ -1436,47 +1486,50 @@ static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, 
   CUtensorMap tA, tB;
   int rc;
   // (1) da = dy Wd^T -> SwiGLU backward -> dhu
-  if (launch_mx_quant_rows(dy_perm, P, s.d, offsets, s.E, R, dyq.codes, dyq.scales, st) ||
-      launch_mx_quant_rows(w_down, ef, s.d, nullptr, s.E, ef, wdr.codes, wdr.scales, st))
+  // dy_quantized: the combine's backward already wrote dy_perm's codes in both orientations
+  if ((!dy_quantized && launch_mx_quant_rows(dy_perm, P, s.d, offsets, s.E, R, dyq.codes, dyq.scales, st, true)) ||
+      (!wsaved && launch_mx_quant_rows(w_down, ef, s.d, nullptr, s.E, ef, wdr.codes, wdr.scales, st, true)))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, dyq.codes, 1, s.d, R, 128, BM) || !make_tmap(&tB, wdr.codes, 1, s.d, ef, 128, 128))
     return MOE_ERR_CUDA;
   p.K = s.d; p.N = s.f; p.out0 = dhu; p.aux = hu;
-  p.sfa = dyq.scales; p.sfa_ld = s.d / 32; p.sfb = wdr.scales; p.sfb_ld = s.d / 32;
+  p.sfa = dyq.scales; p.nka = s.d / 128; p.sfb = wdr.scales; p.nkb = s.d / 128;
+  // the epilogue also writes [dh | du] in MXFP8 in both orientations the gate/up GEMMs read
+  p.q_row_codes = dhuq.codes; p.q_row_scales = dhuq.scales; p.nk_row = 2 * s.f / 128;
+  p.q_col_codes = dhuqt.codes; p.q_col_scales = dhuqt.scales; p.nk_col = nkt;
   rc = launch<e4m3, 128, DGRAD_DOWN>(tA, tB, tB, p, mblocks * (s.f / 128), st);
+  p.q_row_codes = p.q_row_scales = p.q_col_codes = p.q_col_scales = nullptr;
   if (rc) return rc;
   // (2) dWd = a^T dy, K = the tokens of each expert
-  if (launch_mx_quant_cols(a, P, s.f, offsets, s.E, R, aqt.codes, aqt.scales, st) ||
-      launch_mx_quant_cols(dy_perm, P, s.d, offsets, s.E, R, dyqt.codes, dyqt.scales, st))
+  if ((!wsaved && launch_mx_quant_cols(a, P, s.f, offsets, s.E, R, aqt.codes, aqt.scales, st, true)) ||
+      (!dy_quantized && launch_mx_quant_cols(dy_perm, P, s.d, offsets, s.E, R, dyqt.codes, dyqt.scales, st, true)))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, aqt.codes, 1, s.f, R, 128, 128) || !make_tmap(&tB, dyqt.codes, 1, s.d, R, 128, 128))
     return MOE_ERR_CUDA;
   CUtensorMap tO0, tO1;
   if (!make_tmap(&tO0, dw_down, 2, s.d, ef, 64, 32)) return MOE_ERR_CUDA;
   p.M = s.f; p.N = s.d; p.out0 = dw_down; p.aux = nullptr;
-  p.sfa = aqt.scales; p.sfa_ld = s.f; p.sfb = dyqt.scales; p.sfb_ld = s.d;
+  p.sfa = aqt.scales; p.nka = nkt; p.sfb = dyqt.scales; p.nkb = nkt;
   rc = launch<e4m3, 128, WGRAD_DOWN>(tA, tB, tB, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st, &tO0, &tO0);
   if (rc) return rc;
   // (3) dx_perm = [dh | du] [Wg | Wu]^T
-  if (launch_mx_quant_rows(dhu, P, 2 * s.f, offsets, s.E, R, dhuq.codes, dhuq.scales, st) ||
-      launch_mx_quant_rows_gu(w_gate, w_up, ed, s.f, wgur.codes, wgur.scales, st))
+  if (!wsaved && launch_mx_quant_rows_gu(w_gate, w_up, ed, s.f, wgur.codes, wgur.scales, st, true))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, dhuq.codes, 1, 2 * s.f, R, 128, BM) || !make_tmap(&tB, wgur.codes, 1, 2 * s.f, ed, 128, 128))
     return MOE_ERR_CUDA;
   p.K = 2 * s.f; p.N = s.d; p.out0 = dx_perm;
-  p.sfa = dhuq.scales; p.sfa_ld = 2 * s.f / 32; p.sfb = wgur.scales; p.sfb_ld = 2 * s.f / 32;
+  p.sfa = dhuq.scales; p.nka = 2 * s.f / 128; p.sfb = wgur.scales; p.nkb = 2 * s.f / 128;
   rc = launch<e4m3, 128, DGRAD_GU>(tA, tB, tB, p, mblocks * (s.d / 128), st);
   if (rc) return rc;
   // (4) [dWg | dWu] = x^T [dh | du], K = the tokens of each expert
-  if (launch_mx_quant_cols(x_perm, P, s.d, offsets, s.E, R, xqt.codes, xqt.scales, st) ||
-      launch_mx_quant_cols(dhu, P, 2 * s.f, offsets, s.E, R, dhuqt.codes, dhuqt.scales, st))
+  if (!wsaved && launch_mx_quant_cols(x_perm, P, s.d, offsets, s.E, R, xqt.codes, xqt.scales, st, true))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, xqt.codes, 1, s.d, R, 128, 128) || !make_tmap(&tB, dhuqt.codes, 1, 2 * s.f, R, 128, 128))
     return MOE_ERR_CUDA;
   if (!make_tmap(&tO0, dw_gate, 2, s.f, ed, 64, 32) || !make_tmap(&tO1, dw_up, 2, s.f, ed, 64, 32))
     return MOE_ERR_CUDA;
   p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
-  p.sfa = xqt.scales; p.sfa_ld = s.d; p.sfb = dhuqt.scales; p.sfb_ld = 2 * s.f;
+  p.sfa = xqt.scales; p.nka = nkt; p.sfb = dhuqt.scales; p.nkb = nkt;
   return launch<e4m3, 128, WGRAD_GU>(tA, tB, tB, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st, &tO0, &tO1);
 }
 
@@ -1491,9 +1544,10 @@ int launch_router_tc(const Shape &s, const void *x, const void *w_r, const float
 
 int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *hu, void *a, void *y_perm, void *ws,
-                       cudaStream_t st, bool x_quantized) {
+                       cudaStream_t st, bool x_quantized, uint8_t *wsaved, bool wfill) {
   if (s.prec == MOE_PREC_MXFP8)
-    return gg::mx_fwd_impl(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st, x_quantized);
+    return gg::mx_fwd_impl(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st, x_quantized, wsaved,
+                           wfill);
   if (s.dtype == MOE_BF16)
     return gg::fwd_impl<bf16>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
   return gg::fwd_impl<float>(s, x_perm, offsets, w_gate, w_up, w_down, hu, a, y_perm, ws, st);
@@ -1502,13 +1556,13 @@ int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offset
 int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                        const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
                        const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
-                       void *dw_down, void *ws, cudaStream_t st) {
+                       void *dw_down, void *ws, cudaStream_t st, const uint8_t *wsaved, bool dy_quantized) {
   // The weight-gradient GEMMs reduce over tokens, which makes both operands MN-major;
   // tf32 MMAs take K-major operands only, so the fp32 backward is not offered.
   if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (s.prec == MOE_PREC_MXFP8)
     return gg::mx_bwd_impl(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm, dw_gate,
-                           dw_up, dw_down, ws, st);
+                           dw_up, dw_down, ws, st, wsaved, dy_quantized);
   return gg::bwd_impl<bf16>(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
                             dw_gate, dw_up, dw_down, err_word(ws), st);
 }

@@ -63,6 +63,11 @@ size_t moe_workspace_size(const moe_config *cfg) {
   return ws_layout(shape_of(cfg)).total;
 }
 
+size_t moe_mx_saved_bytes(const moe_config *cfg) {
+  if (!cfg || cfg->T < 0 || cfg->E <= 0 || cfg->d <= 0 || cfg->f <= 0 || cfg->k <= 0) return 0;
+  return mx_saved_layout(shape_of(cfg)).total;
+}
+
 int moe_get_error(void *ws, moe_stream_t stream, int32_t *code) {
   if (!ws || !code) return MOE_ERR_INVALID_ARG;
   int32_t h = 0;
@@ -266,6 +271,7 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   RETURN_IF(check_ptrs4({sv->counts, sv->offsets}));
   if (route) RETURN_IF(check_ptrs4({w->w_router}));
   if (shared) RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down}));
+  if (s.prec == MOE_PREC_MXFP8) RETURN_IF(check_ptrs_or_null({sv->mx_saved}));
   if (cfg->T > 0) {
     RETURN_IF(check_ptrs({x, y, sv->x_perm, sv->a, sv->y_perm}));
     RETURN_IF(check_ptrs_or_null({sv->hu}));
@@ -286,16 +292,25 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
                                          sv->pair_of_slot, bc, err, st)));
   if (cfg->T == 0) return MOE_OK;
   const bool mx = s.prec == MOE_PREC_MXFP8;
+  uint8_t *mxs = mx ? static_cast<uint8_t *>(sv->mx_saved) : nullptr;
   if (mx) {
-    // FP8 dispatch: the permute also writes x_perm's MXFP8 rows where the forward GEMM reads them
+    // FP8 dispatch: the permute also writes x_perm's MXFP8 rows where the forward GEMM reads
+    // them, and, when the caller keeps the MXFP8 copies for the backward, its token-axis copy
     uint8_t *xq = static_cast<uint8_t *>(ws) + L.xq_r;
-    RETURN_IF(cuda_rc(launch_mx_permute(x, sv->slot_of_pair, sv->offsets, s.E, s.T, s.k, s.d, sv->x_perm, xq,
-                                        xq + s.Ppad() * s.d, st)));
+    const int64_t R = s.Ppad();
+    if (mxs) {
+      uint8_t *xqt = mxs + mx_saved_layout(s).xq_t;
+      RETURN_IF(cuda_rc(launch_mx_dispatch(x, sv->pair_of_slot, sv->offsets, s.E, s.k, s.d, R, sv->x_perm, xq,
+                                           xq + R * s.d, xqt, xqt + R * s.d, st)));
+    } else {
+      RETURN_IF(cuda_rc(launch_mx_permute(x, sv->slot_of_pair, sv->offsets, s.E, s.T, s.k, s.d, sv->x_perm, xq,
+                                          xq + R * s.d, st, /*tiled=*/true)));
+    }
   } else {
     RETURN_IF(cuda_rc(launch_permute(s, x, sv->slot_of_pair, sv->x_perm, st)));
   }
   RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, sv->hu, sv->a,
-                               sv->y_perm, ws, st, mx));
+                               sv->y_perm, ws, st, mx, mxs, /*wfill=*/true));
   if (shared) {
     // the shared expert's output goes straight into y; the combine then adds to it
     int32_t *go = reinterpret_cast<int32_t *>(static_cast<char *>(ws) + L.group_offsets);
@@ -330,10 +345,11 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   RETURN_IF(check_ptrs({w->w_gate, w->w_up, w->w_down, g->dw_gate, g->dw_up, g->dw_down}));
   RETURN_IF(check_ptrs4({sv->offsets}));
   if (router) RETURN_IF(check_ptrs4({w->w_router, g->dw_router}));
-  if (router && cfg->T > 0) RETURN_IF(check_ptrs4({sv->pair_of_slot}));
+  if ((router || s.prec == MOE_PREC_MXFP8) && cfg->T > 0) RETURN_IF(check_ptrs4({sv->pair_of_slot}));
   if (shared)
     RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down, g->dw_shared_gate,
                           g->dw_shared_up, g->dw_shared_down}));
+  if (s.prec == MOE_PREC_MXFP8) RETURN_IF(check_ptrs_or_null({sv->mx_saved}));
   if (cfg->T > 0) {
     RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
     RETURN_IF(check_ptrs_or_null({sv->hu}));
@@ -355,17 +371,31 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
     if (e == cudaSuccess && shared) e = cudaMemsetAsync(g->dw_shared_down, 0, sb, st);
     return cuda_rc(e);
   }
-  RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
-                                       g->dgate, st)));
+  const bool mx = s.prec == MOE_PREC_MXFP8;
+  if (mx) {
+    // FP8 dispatch of the backward: dy_perm's MXFP8 copies for both down-projection GEMMs come
+    // out of the combine's backward itself
+    const WsLayout L = ws_layout(s);
+    uint8_t *w8 = static_cast<uint8_t *>(ws);
+    const int64_t R = s.Ppad();
+    uint8_t *dyq = w8 + L.dyq_r, *dyqt = w8 + L.dyq_t;
+    RETURN_IF(cuda_rc(launch_mx_combine_bwd(dy, sv->y_perm, sv->pair_of_slot, sv->offsets, sv->topk_gate, s.E, s.k,
+                                            s.d, R, g->dy_perm, g->dgate, dyq, dyq + R * s.d, dyqt, dyqt + R * s.d,
+                                            st)));
+  } else {
+    RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
+                                         g->dgate, st)));
+  }
   // recompute: [h | u] = x_perm [Wg | Wu] into dhu, where the SwiGLU backward then runs in place
+  uint8_t *mxs = s.prec == MOE_PREC_MXFP8 ? static_cast<uint8_t *>(sv->mx_saved) : nullptr;
   const void *hu = sv->hu;
   if (!hu) {
     RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, g->dhu, nullptr,
-                                 nullptr, ws, st));
+                                 nullptr, ws, st, false, mxs, /*wfill=*/false));
     hu = g->dhu;
   }
   RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, hu, sv->a, sv->offsets, w->w_gate, w->w_up,
-                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st));
+                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st, mxs, mx));
   if (shared) {
     // one group of all tokens: its dy is dY itself (weight 1) and its dx, in token order,
     // is written to dx, to which the routed experts' rows are then added

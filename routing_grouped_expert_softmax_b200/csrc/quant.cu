@@ -16,26 +16,10 @@
 // Activation operands are written into expert buffers padded to 128 rows: padded row
 // 128*pre[e] + i holds source row offsets[e] + i for i < count_e and zeros after, where
 // pre[e] = sum_{e' < e} ceil(count_e' / 128).
-#include <cuda_fp8.h>
-
 #include "common.cuh"
+#include "mxfp8.cuh"
 
 namespace moe {
-
-// E8M0 exponent s (scale 2^s) of a block from its largest magnitude.
-__device__ __forceinline__ int mx_scale_exp(float amax) {
-  const uint32_t bits = __float_as_uint(amax);
-  const int e = (int)((bits >> 23) & 0xFF);
-  if (e == 0) return -127;                 // zero or fp32-subnormal amax
-  return max(e - 127 - 8, -127);           // floor(log2 amax) - 8 (at most 119 for finite amax)
-}
-
-// 2^-s as a float, for s in [-127, 119]
-__device__ __forceinline__ float exp2_neg(int s) { return __uint_as_float((uint32_t)(127 - s) << 23); }
-
-__device__ __forceinline__ uint16_t e4m3x2(float lo, float hi) {
-  return (uint16_t)__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3);
-}
 
 // Padded-row bookkeeping: exclusive prefix of 128-row blocks per expert, by one warp.
 __device__ void mx_block_prefix(const int32_t *offsets, int E, int *pre) {
@@ -82,7 +66,7 @@ __device__ __forceinline__ int64_t mx_src_row(int64_t pr, const int32_t *offsets
 __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16 *__restrict__ src, int64_t R, int K,
                                                             const int32_t *__restrict__ offsets, int E,
                                                             uint8_t *__restrict__ codes,
-                                                            uint8_t *__restrict__ scales) {
+                                                            uint8_t *__restrict__ scales, bool tiled) {
   __shared__ int pre[MAX_E + 1];
   if (offsets) {
     if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
@@ -121,7 +105,7 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16 *__restri
     uint4 *d4 = reinterpret_cast<uint4 *>(codes + pr * K + c0 + lane * 32);
     d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
     d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    scales[pr * (K / 32) + blk] = (uint8_t)(s + 127);
+    scales[tiled ? sf_tiled_off(pr, blk, K / 128) : pr * (K / 32) + blk] = (uint8_t)(s + 127);
   }
 }
 
@@ -131,8 +115,8 @@ __global__ void __launch_bounds__(256) mx_quant_rows_kernel(const bf16 *__restri
 __device__ __forceinline__ uint2 mx_row8(const bf16 *src, int64_t ld_src, int i, int nvalid) {
   return i < nvalid ? __ldg(reinterpret_cast<const uint2 *>(src + i * ld_src)) : make_uint2(0u, 0u);
 }
-__device__ __forceinline__ void mx_cols4(const bf16 *src, int64_t ld_src, int nvalid, uint8_t *codes,
-                                         int64_t ld_codes, uint8_t *scales) {
+__device__ __forceinline__ uint32_t mx_cols4(const bf16 *src, int64_t ld_src, int nvalid, uint8_t *codes,
+                                             int64_t ld_codes) {
   float amax[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
@@ -157,15 +141,28 @@ __device__ __forceinline__ void mx_cols4(const bf16 *src, int64_t ld_src, int nv
         ((uint32_t)e4m3x2(__uint_as_float(r.y << 16) * inv[2], __uint_as_float(r.y & 0xFFFF0000u) * inv[3]) << 16);
     *reinterpret_cast<uint32_t *>(codes + i * ld_codes) = w;
   }
-  *reinterpret_cast<uint32_t *>(scales) = (uint32_t)(sc[0] + 127) | ((uint32_t)(sc[1] + 127) << 8) |
-                                          ((uint32_t)(sc[2] + 127) << 16) | ((uint32_t)(sc[3] + 127) << 24);
+  // the four columns' scale bytes, column j in byte j
+  return (uint32_t)(sc[0] + 127) | ((uint32_t)(sc[1] + 127) << 8) | ((uint32_t)(sc[2] + 127) << 16) |
+         ((uint32_t)(sc[3] + 127) << 24);
+}
+
+// Scale bytes of four adjacent columns c..c+3 (K-block kb): plain, one 4-byte store at
+// row kb of [.][C]; tiled, one byte each.
+__device__ __forceinline__ void mx_put_scales4(uint8_t *scales, uint32_t sc4, int64_t kb, int c, int C, bool tiled,
+                                               int64_t nkg) {
+  if (!tiled) {
+    *reinterpret_cast<uint32_t *>(scales + kb * C + c) = sc4;
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) scales[sf_tiled_off(c + j, kb, nkg)] = (uint8_t)(sc4 >> (8 * j));
+  }
 }
 
 // ---- cols: one thread per (4 adjacent columns, 32-row block).  C % 4 == 0.
 __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restrict__ src, int64_t R, int C,
                                                             const int32_t *__restrict__ offsets, int E,
                                                             uint8_t *__restrict__ codes,
-                                                            uint8_t *__restrict__ scales) {
+                                                            uint8_t *__restrict__ scales, bool tiled, int64_t nkg) {
   __shared__ int pre[MAX_E + 1];
   if (offsets) {
     if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
@@ -191,7 +188,8 @@ __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restri
     }
   }
   if (sr0 < 0) sr0 = 0;   // nothing is read from it then
-  mx_cols4(src + sr0 * C + c, C, nvalid, codes + rb * 32 * C + c, C, scales + rb * C + c);
+  const uint32_t sc4 = mx_cols4(src + sr0 * C + c, C, nvalid, codes + rb * 32 * C + c, C);
+  mx_put_scales4(scales, sc4, rb, c, C, tiled, nkg);
 }
 
 // ---- weights of the gate/up GEMM, blocked down the rows, with gate and up columns
@@ -201,7 +199,7 @@ __global__ void __launch_bounds__(256) mx_quant_cols_kernel(const bf16 *__restri
 __global__ void __launch_bounds__(256) mx_quant_cols_gu_kernel(const bf16 *__restrict__ wg,
                                                                const bf16 *__restrict__ wu, int64_t R, int f,
                                                                uint8_t *__restrict__ codes,
-                                                               uint8_t *__restrict__ scales) {
+                                                               uint8_t *__restrict__ scales, bool tiled) {
   const int oc = 4 * (blockIdx.x * 256 + threadIdx.x);   // output column in [0, 2f)
   const int64_t rb = blockIdx.y;
   if (oc >= 2 * f || rb * 32 >= R) return;
@@ -209,7 +207,8 @@ __global__ void __launch_bounds__(256) mx_quant_cols_gu_kernel(const bf16 *__res
   const bf16 *src = i < 64 ? wg : wu;
   const int c = 64 * j + (i & 63);
   const int nvalid = (int)(R - rb * 32 < 32 ? R - rb * 32 : 32);
-  mx_cols4(src + rb * 32 * f + c, f, nvalid, codes + rb * 32 * (2 * f) + oc, 2 * f, scales + rb * (2 * f) + oc);
+  const uint32_t sc4 = mx_cols4(src + rb * 32 * f + c, f, nvalid, codes + rb * 32 * (2 * f) + oc, 2 * f);
+  mx_put_scales4(scales, sc4, rb, oc, 2 * f, tiled, (R + 127) / 128);
 }
 
 // ---- weights of the gate/up data-gradient GEMM, blocked along the rows of [W_gate | W_up]
@@ -217,7 +216,7 @@ __global__ void __launch_bounds__(256) mx_quant_cols_gu_kernel(const bf16 *__res
 __global__ void __launch_bounds__(256) mx_quant_rows_gu_kernel(const bf16 *__restrict__ wg,
                                                                const bf16 *__restrict__ wu, int64_t R, int f,
                                                                uint8_t *__restrict__ codes,
-                                                               uint8_t *__restrict__ scales) {
+                                                               uint8_t *__restrict__ scales, bool tiled) {
   const int lane = threadIdx.x & 31;
   const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
   if (r >= R) return;
@@ -243,8 +242,91 @@ __global__ void __launch_bounds__(256) mx_quant_rows_gu_kernel(const bf16 *__res
     uint4 *d4 = reinterpret_cast<uint4 *>(codes + r * K + col);
     d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
     d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    scales[r * (K / 32) + col / 32] = (uint8_t)(sc + 127);
+    scales[tiled ? sf_tiled_off(r, col / 32, K / 128) : r * (K / 32) + col / 32] = (uint8_t)(sc + 127);
   }
+}
+
+// ---- weights in both orientations from one read.  A block takes a tile of 32 rows x 128
+// columns: for the gate/up pair (gu) 64 columns of W_gate and the same 64 of W_up, else 128
+// columns of one tensor [R][C].  From the tile it writes
+//   codes_c: blocks of 32 down the rows (the forward GEMMs' K), [R][C'] with C' = 2f for the
+//            pair (gate and up interleaved in 64-column chunks: output column 128 J + i is gate
+//            column 64 J + i for i < 64, up column 64 J + i - 64 otherwise) or C;
+//   codes_r: blocks of 32 along the row (the data-gradient GEMMs' K), [R][C'] with row r of the
+//            pair [W_gate[r] | W_up[r]];
+// scales of both in the tile layout.  Same arithmetic as the single-orientation kernels.
+constexpr int WQ_ROWS = 32, WQ_COLS = 128;
+__global__ void __launch_bounds__(256) mx_quant_weights_kernel(const bf16 *__restrict__ w0, const bf16 *__restrict__ w1,
+                                                               int64_t R, int C, bool gu,
+                                                               uint8_t *__restrict__ codes_c,
+                                                               uint8_t *__restrict__ scales_c,
+                                                               uint8_t *__restrict__ codes_r,
+                                                               uint8_t *__restrict__ scales_r) {
+  __shared__ float tile[WQ_ROWS][WQ_COLS + 1];
+  __shared__ float inv_c[WQ_COLS], inv_r[WQ_ROWS][4];
+  const int t = threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.y * WQ_ROWS;
+  const int CO = gu ? 2 * C : C;                    // output columns per row
+  // source column of tile column j: (tensor, column)
+  auto src_of = [&](int j, const bf16 *&w, int &col) {
+    if (gu) { w = j < 64 ? w0 : w1; col = blockIdx.x * 64 + (j & 63); }
+    else { w = w0; col = blockIdx.x * WQ_COLS + j; }
+  };
+  // output column of tile column j in the row-blocked layout
+  auto rcol_of = [&](int j) { return gu ? (j < 64 ? 0 : C) + (int)blockIdx.x * 64 + (j & 63)
+                                        : (int)blockIdx.x * WQ_COLS + j; };
+  const int ccol0 = blockIdx.x * WQ_COLS;           // first output column in the column-blocked layout
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {                     // 512 16-byte pieces, two per thread
+    const int idx = t + 256 * i, row = idx >> 4, j = (idx & 15) * 8;
+    const bf16 *w;
+    int col;
+    src_of(j, w, col);
+    float v[8];
+    Vec<bf16>::load(__ldg(reinterpret_cast<const uint4 *>(w + (r0 + row) * C + col)), v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) tile[row][j + e] = v[e];
+  }
+  __syncthreads();
+  if (t < WQ_COLS) {                                 // column scales: one 32-row block per column
+    float amax = 0.f;
+#pragma unroll 8
+    for (int r = 0; r < WQ_ROWS; ++r) amax = fmaxf(amax, fabsf(tile[r][t]));
+    const int sc = mx_scale_exp(amax);
+    inv_c[t] = exp2_neg(sc);
+    scales_c[sf_tiled_off(ccol0 + t, r0 / 32, R / 128)] = (uint8_t)(sc + 127);
+  } else {                                          // row scales: 4 blocks of 32 columns per row
+    const int u = t - WQ_COLS, row = u >> 2, b = u & 3;
+    float amax = 0.f;
+#pragma unroll 8
+    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(tile[row][32 * b + j]));
+    const int sc = mx_scale_exp(amax);
+    inv_r[row][b] = exp2_neg(sc);
+    scales_r[sf_tiled_off(r0 + row, rcol_of(32 * b) / 32, CO / 128)] = (uint8_t)(sc + 127);
+  }
+  __syncthreads();
+  // codes: thread t writes 16 consecutive tile columns of one row in both layouts
+  const int row = t >> 3, j0 = (t & 7) * 16;
+  uint32_t wc[4], wr[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int j = j0 + 4 * q;
+    const float ir = inv_r[row][j >> 5];
+    wc[q] = (uint32_t)e4m3x2(tile[row][j] * inv_c[j], tile[row][j + 1] * inv_c[j + 1]) |
+            ((uint32_t)e4m3x2(tile[row][j + 2] * inv_c[j + 2], tile[row][j + 3] * inv_c[j + 3]) << 16);
+    wr[q] = (uint32_t)e4m3x2(tile[row][j] * ir, tile[row][j + 1] * ir) |
+            ((uint32_t)e4m3x2(tile[row][j + 2] * ir, tile[row][j + 3] * ir) << 16);
+  }
+  *reinterpret_cast<uint4 *>(codes_c + (r0 + row) * CO + ccol0 + j0) = make_uint4(wc[0], wc[1], wc[2], wc[3]);
+  *reinterpret_cast<uint4 *>(codes_r + (r0 + row) * CO + rcol_of(j0)) = make_uint4(wr[0], wr[1], wr[2], wr[3]);
+}
+
+cudaError_t launch_mx_quant_weights(const void *w0, const void *w1, int64_t R, int C, bool gu, uint8_t *codes_c,
+                                    uint8_t *scales_c, uint8_t *codes_r, uint8_t *scales_r, cudaStream_t st) {
+  dim3 grid((unsigned)(gu ? C / 64 : C / WQ_COLS), (unsigned)(R / WQ_ROWS));
+  mx_quant_weights_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(w0), static_cast<const bf16 *>(w1), R, C,
+                                                gu, codes_c, scales_c, codes_r, scales_r);
+  return cudaGetLastError();
 }
 
 // ---- FP8 dispatch: x_perm[slot(t,j)] = x[t] (a bit copy) and, in the same pass, the row in
@@ -255,7 +337,8 @@ __global__ void __launch_bounds__(256) mx_quant_rows_gu_kernel(const bf16 *__res
 __global__ void __launch_bounds__(256) mx_permute_kernel(const bf16 *__restrict__ x, const int32_t *__restrict__ sop,
                                                          const int32_t *__restrict__ offsets, int E, int64_t T,
                                                          int k, int d, bf16 *__restrict__ x_perm,
-                                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales) {
+                                                         uint8_t *__restrict__ codes, uint8_t *__restrict__ scales,
+                                                         bool tiled) {
   __shared__ int pre[MAX_E + 1];
   if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
   __syncthreads();
@@ -307,49 +390,201 @@ __global__ void __launch_bounds__(256) mx_permute_kernel(const bf16 *__restrict_
         uint4 *d4 = reinterpret_cast<uint4 *>(codes + prow[j] * d + col);
         d4[0] = make_uint4(w[0], w[1], w[2], w[3]);
         d4[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        scales[prow[j] * (d / 32) + col / 32] = (uint8_t)(sc + 127);
+        scales[tiled ? sf_tiled_off(prow[j], col / 32, d / 128) : prow[j] * (d / 32) + col / 32] =
+            (uint8_t)(sc + 127);
       }
     }
   }
 }
 
+// ---- Slot-major FP8 dispatch, forward and backward.  One block per 32 padded rows of one
+// expert; warp w takes rows 4w..4w+3; the columns go in chunks of 256, 8 per lane.  For the
+// routed pair in slot s (token t, gate g) the row is
+//   forward (BWD = false):  x_perm[s] = x[t]             (src = x; a bit copy)
+//   backward (BWD = true):  dy_perm[s] = bf16(g dY[t])    (src = dY), dgate = <dY[t], y_perm[s]>
+// and in the same pass the row in MXFP8 along d (codes_r, blocks of 32 columns; may be null)
+// and down the token axis (codes_c, blocks of 32 rows of the expert-padded layout), scales in
+// the GEMMs' tile layout.  Pad rows are zeros.
+constexpr int CB_CHUNK = 256;
+template <bool BWD>
+__global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
+    const bf16 *__restrict__ src, const bf16 *__restrict__ y_perm, const int32_t *__restrict__ pos,
+    const int32_t *__restrict__ offsets, const float *__restrict__ gate, int E, int k, int d, int64_t nkt,
+    bf16 *__restrict__ out_perm, float *__restrict__ dgate, uint8_t *__restrict__ codes_r,
+    uint8_t *__restrict__ scales_r, uint8_t *__restrict__ codes_c, uint8_t *__restrict__ scales_c) {
+  __shared__ int pre[MAX_E + 1];
+  __shared__ float colmax[8][CB_CHUNK];
+  __shared__ float inv_col[CB_CHUNK];
+  if (threadIdx.x < 32) mx_block_prefix(offsets, E, pre);
+  __syncthreads();
+  const int64_t blk = blockIdx.x;                    // 32-row block of the padded layout
+  if (blk * 32 >= (int64_t)pre[E] * 128) return;     // (uniform over the block)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // this block's expert: pre[e] <= blk / 4 < pre[e + 1]
+  const int g = (int)(blk >> 2);
+  int lo = 0, hi = E;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pre[mid] <= g) lo = mid; else hi = mid;
+  }
+  const int cnt = offsets[lo + 1] - offsets[lo];
+  int64_t prow[4], tok[4], pair[4];
+  float gt[4], dot[4];
+  bool valid[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    prow[i] = blk * 32 + warp * 4 + i;
+    const int64_t local = prow[i] - (int64_t)pre[lo] * 128;
+    valid[i] = local < cnt;
+    const int64_t slot = offsets[lo] + (valid[i] ? local : 0);
+    pair[i] = valid[i] ? pos[slot] : 0;
+    tok[i] = pair[i] / k;
+    gt[i] = (BWD && valid[i]) ? gate[pair[i]] : 0.f;
+    dot[i] = 0.f;
+  }
+  for (int c0 = 0; c0 < d; c0 += CB_CHUNK) {
+    const int c = c0 + lane * 8;
+    const bool cin = c < d;       // d % 128 == 0: a 32-column block is wholly in or out
+    float v[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t slot = offsets[lo] + (prow[i] - (int64_t)pre[lo] * 128);
+      if (valid[i] && cin) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src + tok[i] * d + c));
+        if constexpr (BWD) {
+          float fd[8], fy[8];
+          Vec<bf16>::load(raw, fd);
+          Vec<bf16>::load(__ldg(reinterpret_cast<const uint4 *>(y_perm + slot * d + c)), fy);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            dot[i] = fmaf(fd[j], fy[j], dot[i]);
+            v[i][j] = gt[i] * fd[j];
+          }
+          const uint4 o = Vec<bf16>::store(v[i]);                // the stored bf16 dy_perm row
+          *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = o;
+          Vec<bf16>::load(o, v[i]);
+        } else {
+          *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = raw;   // the permute: a bit copy
+          Vec<bf16>::load(raw, v[i]);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[i][j] = 0.f;
+      }
+    }
+    // along d: a block of 32 columns is 4 lanes x 8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float amax = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[i][j]));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+      amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+      const int sc = mx_scale_exp(amax);
+      const float inv = exp2_neg(sc);
+      uint2 w;
+      w.x = (uint32_t)e4m3x2(v[i][0] * inv, v[i][1] * inv) | ((uint32_t)e4m3x2(v[i][2] * inv, v[i][3] * inv) << 16);
+      w.y = (uint32_t)e4m3x2(v[i][4] * inv, v[i][5] * inv) | ((uint32_t)e4m3x2(v[i][6] * inv, v[i][7] * inv) << 16);
+      if (cin && codes_r) {
+        *reinterpret_cast<uint2 *>(codes_r + prow[i] * d + c) = w;
+        if ((lane & 3) == 0) scales_r[sf_tiled_off(prow[i], c / 32, d / 128)] = (uint8_t)(sc + 127);
+      }
+    }
+    // down the token axis: the block's 32 rows of each column
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      colmax[warp][lane * 8 + j] =
+          fmaxf(fmaxf(fabsf(v[0][j]), fabsf(v[1][j])), fmaxf(fabsf(v[2][j]), fabsf(v[3][j])));
+    __syncthreads();
+    {
+      float amax = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) amax = fmaxf(amax, colmax[w][threadIdx.x]);
+      const int sc = mx_scale_exp(amax);
+      inv_col[threadIdx.x] = exp2_neg(sc);
+      if (c0 + (int)threadIdx.x < d) scales_c[sf_tiled_off(c0 + threadIdx.x, blk, nkt)] = (uint8_t)(sc + 127);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float *iv = &inv_col[lane * 8];
+      uint2 w;
+      w.x = (uint32_t)e4m3x2(v[i][0] * iv[0], v[i][1] * iv[1]) | ((uint32_t)e4m3x2(v[i][2] * iv[2], v[i][3] * iv[3]) << 16);
+      w.y = (uint32_t)e4m3x2(v[i][4] * iv[4], v[i][5] * iv[5]) | ((uint32_t)e4m3x2(v[i][6] * iv[6], v[i][7] * iv[7]) << 16);
+      if (cin) *reinterpret_cast<uint2 *>(codes_c + prow[i] * d + c) = w;
+    }
+    __syncthreads();   // colmax and inv_col are rewritten by the next chunk
+  }
+  if constexpr (BWD) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float s = dot[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0 && valid[i]) dgate[pair[i]] = s;
+    }
+  }
+}
+
+cudaError_t launch_mx_combine_bwd(const void *dy, const void *y_perm, const int32_t *pos, const int32_t *offsets,
+                                  const float *gate, int E, int k, int d, int64_t rows_bound, void *dy_perm,
+                                  float *dgate, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
+                                  uint8_t *scales_c, cudaStream_t st) {
+  if (rows_bound <= 0) return cudaSuccess;
+  mx_slot_dispatch_kernel<true><<<(unsigned)((rows_bound + 31) / 32), 256, 0, st>>>(
+      static_cast<const bf16 *>(dy), static_cast<const bf16 *>(y_perm), pos, offsets, gate, E, k, d,
+      (rows_bound + 127) / 128, static_cast<bf16 *>(dy_perm), dgate, codes_r, scales_r, codes_c, scales_c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_dispatch(const void *x, const int32_t *pos, const int32_t *offsets, int E, int k, int d,
+                               int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r,
+                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st) {
+  if (rows_bound <= 0) return cudaSuccess;
+  mx_slot_dispatch_kernel<false><<<(unsigned)((rows_bound + 31) / 32), 256, 0, st>>>(
+      static_cast<const bf16 *>(x), nullptr, pos, offsets, nullptr, E, k, d, (rows_bound + 127) / 128,
+      static_cast<bf16 *>(x_perm), nullptr, codes_r, scales_r, codes_c, scales_c);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mx_permute(const void *x, const int32_t *sop, const int32_t *offsets, int E, int64_t T, int k,
-                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st) {
+                              int d, void *x_perm, uint8_t *codes, uint8_t *scales, cudaStream_t st, bool tiled) {
   if (T == 0) return cudaSuccess;
   mx_permute_kernel<<<(unsigned)((T + 7) / 8), 256, 0, st>>>(static_cast<const bf16 *>(x), sop, offsets, E, T, k, d,
-                                                             static_cast<bf16 *>(x_perm), codes, scales);
+                                                             static_cast<bf16 *>(x_perm), codes, scales, tiled);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_rows(const void *src, int64_t R, int K, const int32_t *offsets, int E, int64_t rows_bound,
-                                 uint8_t *codes, uint8_t *scales, cudaStream_t st) {
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st, bool tiled) {
   if (rows_bound <= 0) return cudaSuccess;
   dim3 grid((unsigned)((rows_bound + 7) / 8), (unsigned)((K + 1023) / 1024));
-  mx_quant_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(src), R, K, offsets, E, codes, scales);
+  mx_quant_rows_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(src), R, K, offsets, E, codes, scales, tiled);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_cols(const void *src, int64_t R, int C, const int32_t *offsets, int E, int64_t rows_bound,
-                                 uint8_t *codes, uint8_t *scales, cudaStream_t st) {
+                                 uint8_t *codes, uint8_t *scales, cudaStream_t st, bool tiled) {
   if (rows_bound <= 0) return cudaSuccess;
   dim3 grid((unsigned)((C / 4 + 255) / 256), (unsigned)((rows_bound + 31) / 32));
-  mx_quant_cols_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(src), R, C, offsets, E, codes, scales);
+  mx_quant_cols_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(src), R, C, offsets, E, codes, scales, tiled,
+                                             (rows_bound + 127) / 128);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_cols_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
-                                    uint8_t *scales, cudaStream_t st) {
+                                    uint8_t *scales, cudaStream_t st, bool tiled) {
   dim3 grid((unsigned)((2 * f / 4 + 255) / 256), (unsigned)((R + 31) / 32));
   mx_quant_cols_gu_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(wg), static_cast<const bf16 *>(wu), R, f,
-                                                codes, scales);
+                                                codes, scales, tiled);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_rows_gu(const void *wg, const void *wu, int64_t R, int f, uint8_t *codes,
-                                    uint8_t *scales, cudaStream_t st) {
+                                    uint8_t *scales, cudaStream_t st, bool tiled) {
   mx_quant_rows_gu_kernel<<<(unsigned)((R + 7) / 8), 256, 0, st>>>(static_cast<const bf16 *>(wg),
                                                                     static_cast<const bf16 *>(wu), R, f, codes,
-                                                                    scales);
+                                                                    scales, tiled);
   return cudaGetLastError();
 }
 

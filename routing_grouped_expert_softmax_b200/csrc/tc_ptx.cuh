@@ -146,6 +146,13 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const void *tmap,
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
+// Untiled bulk copy global -> this CTA's shared memory, bytes counted on `bar`.  Both
+// addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+               : "memory");
+}
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (TMA and the tensor cores).
 __device__ __forceinline__ void fence_proxy_async_smem() {

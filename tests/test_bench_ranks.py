@@ -100,6 +100,6 @@ def test_launch_count():
     import bench
     assert bench.count_launches("router") == 18
     assert bench.count_launches("uniform") == 13
-    assert bench.count_launches("router", "mxfp8") == 30
+    assert bench.count_launches("router", "mxfp8") == 22
     assert bench.count_launches("router", "native", shared=True) == 26
     assert bench.count_launches("router", "native", recompute=True) == 19

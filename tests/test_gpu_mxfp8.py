@@ -251,3 +251,30 @@ def test_mx_layer_against_oracle_and_bf16_path(T, d, E, k, f, skew):
     assert 0 < rel_err(host(y), host(ybf)) <= 0.1
     for n in ("dx", "dw_gate", "dw_down"):
         assert rel_err(host(g[n]), host(gbf[n])) <= 0.15, n
+
+
+@pytest.mark.parametrize("recompute", [False, True])
+def test_mx_saved_weights_give_the_same_bits(recompute):
+    """The forward's MXFP8 weight copies (all four orientations from one read of each weight)
+    reused by the backward give exactly what quantising each orientation where it is used
+    gives."""
+    import torch
+    T, d, E, k, f = 600, 256, 8, 4, 256
+    inp = gen.make_layer_inputs(T, d, E, k, f, dtype="bf16", seed=17)
+    outs = []
+    for keep in (False, True):
+        cfg = moe.config(T, d, E, k, f, dtype="bf16", prec="mxfp8")
+        ws = moe.alloc_workspace(cfg)
+        saved = moe.alloc_saved(cfg, recompute=recompute, mx_saved=keep)
+        assert (saved["mx_saved"] is not None) == keep
+        grads = moe.alloc_grads(cfg)
+        w = [dev(a_, "bf16") for a_ in (inp.w_r, inp.w_gate, inp.w_up, inp.w_down)]
+        wts = moe.layer_weights(w[0], None, w[1], w[2], w[3])
+        x = dev(inp.x, "bf16")
+        y = torch.empty(T, d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_layer_fwd(cfg, wts, x, y, saved, ws)
+        moe.moe_layer_bwd(cfg, wts, x, dev(inp.dy, "bf16"), saved, grads, ws)
+        assert moe.moe_get_error(ws) == 0
+        outs.append([host(y)] + [host(grads[n]) for n in ("dx", "dw_gate", "dw_up", "dw_down", "dw_router")])
+    for a_, b_ in zip(*outs):
+        assert np.array_equal(a_, b_)
