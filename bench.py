@@ -41,6 +41,8 @@ WORKLOADS = {
     # the same shapes with every grouped-GEMM operand in MXFP8 (E4M3 + E8M0 per 32)
     "e128_t16k_mxfp8_fwd_bwd": (16384, 2048, 128, 4, 1024, False, "router", "mxfp8"),
     "e128_mxfp8_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "mxfp8"),
+    # E=8 (4096 rows per expert: the GEMMs are compute-bound) with MXFP8 grouped GEMMs
+    "e8_mxfp8_fwd_bwd": (8192, 2048, 8, 4, 1024, False, "router", "mxfp8"),
     # the C3 shapes plus one shared expert (every token, weight 1) of the routed experts' shape
     "e128_shared_fwd_bwd": (8192, 2048, 128, 4, 1024, False, "router", "native", {"shared": True}),
     # the C3 shapes keeping no [h | u] between forward and backward (recomputed there)
@@ -51,7 +53,7 @@ DEFAULT = "e128_fwd_bwd"
 # pages' two comparisons -- 8 against 128 experts at equal active FLOPs (qidao123.com, section
 # "新闻原文"), and MXFP8 against bf16 (unite.ai, section "Παραλληλισμός, Ακρίβεια και
 # Τεχνικές Μνήμης") -- on this layer.
-SWEEP = ("e128_fwd_bwd", "e8_fwd_bwd", "e128_t16k_fwd_bwd", "e128_t16k_mxfp8_fwd_bwd")
+SWEEP = ("e128_fwd_bwd", "e8_fwd_bwd", "e8_mxfp8_fwd_bwd", "e128_t16k_fwd_bwd", "e128_t16k_mxfp8_fwd_bwd")
 
 
 def peaks():
@@ -487,6 +489,8 @@ def run_ours(args):
             r["e128_over_e8_time"] = sweep["e128_fwd_bwd"] / sweep["e8_fwd_bwd"]
         if "e128_t16k_fwd_bwd" in sweep and "e128_t16k_mxfp8_fwd_bwd" in sweep:
             r["mxfp8_speedup_over_bf16"] = sweep["e128_t16k_fwd_bwd"] / sweep["e128_t16k_mxfp8_fwd_bwd"]
+        if "e8_fwd_bwd" in sweep and "e8_mxfp8_fwd_bwd" in sweep:
+            r["mxfp8_speedup_over_bf16_e8"] = sweep["e8_fwd_bwd"] / sweep["e8_mxfp8_fwd_bwd"]
         out["sweep_ratios"] = r
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(inp, k, routing)

@@ -52,6 +52,9 @@ struct WsLayout {
   //   *_r: blocks along the row (K-major use), *_t: blocks down the rows (token axis)
   size_t xq_r, aq_r, dyq_r, dhuq_r, xq_t, aq_t, dyq_t, dhuq_t;  // activations, Ppad rows
   size_t wgu_c, wd_c, wd_r, wgu_r;                              // weights
+  // bf16 weight-gradient GEMMs: every expert's last partial K-block of their two operands,
+  // [E * 64][C] each (rows past the expert zero), C up to max(d, f) and max(d, 2f)
+  size_t wg_tail_a, wg_tail_b;
   // int32 {0, T}: the shared expert's single group.  Last, so that a layout for the shared
   // expert's shape (E = 1, k = 1: every region no larger) never reaches it.
   size_t group_offsets;
@@ -64,6 +67,7 @@ inline size_t mx_bytes_t(int64_t rows, int64_t cols) {
   return align_up((size_t)(rows * cols + ((rows + 127) / 128) * 4 * cols), 256);
 }
 constexpr int RB_SPLIT = 16;          // token splits of the router weight-gradient reduction
+constexpr int WGRAD_TAIL_ROWS = 64;   // rows of a bf16 weight-gradient K-block (one tail per expert)
 
 
 inline WsLayout ws_layout(const Shape &s) {
@@ -93,6 +97,12 @@ inline WsLayout ws_layout(const Shape &s) {
     L.wd_c = off;   off += mx_bytes_t(ef, s.d);
     L.wd_r = off;   off += mx_bytes_r(ef, s.d);
     L.wgu_r = off;  off += mx_bytes_r(ed, 2 * s.f);
+  }
+  L.wg_tail_a = L.wg_tail_b = 0;
+  if (s.dtype == MOE_BF16 && s.prec == MOE_PREC_NATIVE) {
+    const size_t rows = (size_t)s.E * WGRAD_TAIL_ROWS;
+    L.wg_tail_a = off; off = align_up(off + rows * (size_t)(s.d > s.f ? s.d : s.f) * 2, 256);
+    L.wg_tail_b = off; off = align_up(off + rows * (size_t)(s.d > 2 * s.f ? s.d : 2 * s.f) * 2, 256);
   }
   L.group_offsets = off; off += 256;   // {0, T}: the shared expert's single group
   L.total = off;
@@ -218,6 +228,10 @@ cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, cons
 cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
                                 const int32_t *idx, const void *x, float *partial,
                                 float *dw_r, cudaStream_t st);
+// bf16 weight gradients: tails[e*64 + i] = src[offsets[e] + 64*(count_e/64) + i] for
+// i < count_e % 64 and zeros for the rest of the expert's 64 rows (src [P][C] bf16); experts
+// whose count is a multiple of 64 are left alone (they have no partial K-block).
+cudaError_t launch_wgrad_tails(const void *src, int C, const int32_t *offsets, int E, void *tails, cudaStream_t st);
 // MXFP8 only:
 //   x_quantized: the workspace already holds x_perm's MXFP8 rows, written by
 //     launch_mx_permute into the layout ws_layout(s) gives them;

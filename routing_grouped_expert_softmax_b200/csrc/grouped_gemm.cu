@@ -8,7 +8,7 @@
 // стек обучения MoE от Ai2 ...", section "Три числа, три знаменателя" (the gains sit in
 // the feed-forward compute).
 //
-// One persistent kernel, one CTA per SM, 11 warps:
+// One persistent kernel, one CTA per SM, 10 warps:
 //   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) K-blocks in shared
 //               memory (128-byte swizzle), one mbarrier per stage;
 //   warp 1      allocates TMEM; its lane 0 issues tcgen05.mma (128 x BN x 16 per
@@ -19,16 +19,16 @@
 //               the columns), apply the fused elementwise step and store to global
 //               memory (weight gradients: through shared memory and TMA stores), then
 //               release the accumulator;
-//   warp 10     weight gradients: zeroes the K rows of an expert's last stage that lie
-//               past the expert's end, then releases that stage to the MMA issuer.
 // The epilogue of tile i overlaps the MMAs of tile i+1 (double-buffered accumulator).
 //
 // Tile schedule.  Row-grouped GEMMs (forward and data-gradient) tile every expert's row
 // range [offsets[e], offsets[e+1]) in 128-row blocks; each CTA rebuilds the per-expert
 // block prefix from `offsets` on the device, so the host never learns the counts.
 // Rows of a block that belong to the next expert are computed and not stored.
-// Weight-gradient GEMMs reduce over one expert's rows; the last K-block of an expert
-// is zero-filled in shared memory past the expert's end before the MMA reads it.
+// Weight-gradient GEMMs reduce over one expert's rows; the expert's last, partial K-block is
+// read from a per-expert tail buffer that holds its rows and zeros after them (bf16; the
+// MXFP8 operands are padded to 128 rows per expert instead), so every stage is an ordinary
+// load.
 // CTA pairs (cta_group::2): a 256-row tile whose MMAs the even CTA issues for both.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -46,8 +46,7 @@ enum Mode { FWD_GU = 0, FWD_DOWN = 1, DGRAD_DOWN = 2, DGRAD_GU = 3, WGRAD_DOWN =
 
 constexpr int BM = 128;
 constexpr int EPI_WARPS = 8;
-constexpr int FIX_WARP = 2 + EPI_WARPS;           // weight gradients: zeroes K rows past an expert
-constexpr int NUM_THREADS = 32 * (FIX_WARP + 1);  // producer, MMA issuer, epilogue warps, tail fixer
+constexpr int NUM_THREADS = 32 * (2 + EPI_WARPS);  // producer, MMA issuer, epilogue warps
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s: far above any tile's time
 
 template <int MODE> struct ModeTraits {
@@ -161,7 +160,6 @@ struct Ctrl {
   uint64_t empty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
-  uint64_t tailbar[8];    // weight gradients: a stage's loads ran past the expert's rows
   uint64_t drain;
   uint64_t never;         // the failure-detection hook's barrier: nothing ever arrives on it
   uint64_t xfull[4];      // router: one lane quarter's second-half picks are in xbuf
@@ -171,21 +169,28 @@ struct Ctrl {
   union {
     int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
     float bias[MAX_E];      // router: the logit bias (0 past E)
+    int offs[MAX_E + 1];    // bf16 weight gradients: a copy of offsets (prefix is unused there)
   };
 };
 static_assert(sizeof(Ctrl) <= CTRL_BYTES, "control block");
 // Router: shared buffer for the second-half picks, [MAX_K][BM] keys then [MAX_K][BM] experts
 constexpr int ROUTER_XBYTES = 2 * MAX_K * BM * 4;
-// Weight gradients: each epilogue warp stages its output in two boxes of 32 rows x 64 bf16
-// columns (128-byte rows, 128-byte swizzle) that TMA stores write out.
+// Weight gradients: each epilogue warp stages its output in one box of 32 rows x 64 bf16
+// columns (128-byte rows, 128-byte swizzle) that TMA stores write out.  One box per warp
+// (32 KB in all) leaves room for six pipeline stages of 32 KB.
 constexpr int EPI_BOX_BYTES = 32 * 128;
-constexpr int WGRAD_XBYTES = EPI_WARPS * 2 * EPI_BOX_BYTES;
+constexpr int WGRAD_XBYTES = EPI_WARPS * EPI_BOX_BYTES;
+// Row-grouped GEMMs: a copy of offsets [E+1] after the control block, read by every role's
+// tile lookup (one global load per tile per role otherwise, on the MMA issuer's critical path).
+constexpr int OFFS_BYTES = 1152;
 template <int MODE> constexpr int extra_smem() {
-  return MODE == ROUTER ? ROUTER_XBYTES : ModeTraits<MODE>::WGRAD ? WGRAD_XBYTES : 0;
+  return MODE == ROUTER ? ROUTER_XBYTES : ModeTraits<MODE>::WGRAD ? WGRAD_XBYTES : OFFS_BYTES;
 }
 
+// offs: offsets [E+1] (a shared-memory copy where the kernel keeps one)
 template <int MODE, int BN, int KBLK, bool MX, int CG = 1>
-__device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, Tile &tl, int rank = 0) {
+__device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, const int *offs, Tile &tl,
+                                         int rank = 0) {
   constexpr int BMP = BM * CG;
   if constexpr (MODE == ROUTER) {
     tl.e = 0;
@@ -201,7 +206,7 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.m_blk = r / nt;
     tl.n_blk = r - tl.m_blk * nt;
     tl.mcol0 = tl.m_blk * BMP + rank * BM;
-    int lo = p.offsets[tl.e], hi = p.offsets[tl.e + 1];
+    int lo = offs[tl.e], hi = offs[tl.e + 1];
     tl.rows = hi - lo;
     if constexpr (MX) {
       // quantised operands live in expert buffers padded to 128 rows (zeros past the end)
@@ -224,7 +229,7 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     }
     tl.e = lo;
     tl.m_blk = g - c.prefix[lo];
-    int off = p.offsets[lo], cnt = p.offsets[lo + 1] - off;
+    int off = offs[lo], cnt = offs[lo + 1] - off;
     tl.orow0 = off + tl.m_blk * BMP + rank * BM;   // this CTA's rows of the (pair) tile
     tl.row0 = MX ? g * BM : tl.orow0;   // quantised A: expert buffers padded to 128 rows
     tl.rows = min(BM, cnt - tl.m_blk * BMP - rank * BM);   // may be <= 0 for the second CTA
@@ -326,7 +331,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                         const __grid_constant__ CUtensorMap tmB0,
                         const __grid_constant__ CUtensorMap tmB1,
                         const __grid_constant__ CUtensorMap tmO0,   // weight gradients: outputs
-                        const __grid_constant__ CUtensorMap tmO1, const Params p) {
+                        const __grid_constant__ CUtensorMap tmO1,
+                        const __grid_constant__ CUtensorMap tmAT,   // bf16 weight gradients: tail
+                        const __grid_constant__ CUtensorMap tmBT,   // buffers of A and B
+                        const Params p) {
   using C = Cfg<T, BN, CG, extra_smem<MODE>()>;
   static_assert(CG == 1 || (sizeof(T) == 2 && MODE != ROUTER), "CTA pairs: bf16 grouped GEMMs only");
   constexpr int BMP = C::BMP, BNC = C::BNC;
@@ -360,7 +368,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
       ptx::mbar_init(ptx::smem_u32(&c.tempty[a]), EPI_WARPS * CG);   // one arrival per epilogue warp
     }
-    for (int s = 0; s < C::STAGES; ++s) ptx::mbar_init(ptx::smem_u32(&c.tailbar[s]), 1);
     ptx::mbar_init(ptx::smem_u32(&c.drain), 1);
     ptx::mbar_init(ptx::smem_u32(&c.never), 1);
     for (int q = 0; q < 4; ++q) {
@@ -375,6 +382,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if constexpr (MT::WGRAD) {
       ptx::tma_prefetch(&tmO0);
       ptx::tma_prefetch(&tmO1);
+      if constexpr (!C::MX) {
+        ptx::tma_prefetch(&tmAT);
+        ptx::tma_prefetch(&tmBT);
+      }
     }
   }
   if (warp == 1) {
@@ -391,6 +402,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float *bias = static_cast<const float *>(p.aux);
       for (int e = threadIdx.x - 64; e < MAX_E; e += 32 * EPI_WARPS) c.bias[e] = (bias && e < p.E) ? bias[e] : 0.f;
     }
+  }
+  // shared-memory copy of offsets: bf16 weight gradients in the control block's union (their
+  // prefix is unused), row-grouped GEMMs after the control block; MXFP8 weight gradients read
+  // the global array (their union holds the padded prefix)
+  constexpr bool SMEM_OFFS = MODE != ROUTER && !(MT::WGRAD && C::MX);
+  int *offs_smem = MT::WGRAD ? c.offs : reinterpret_cast<int *>(extra);
+  const int *offs_s = SMEM_OFFS ? offs_smem : p.offsets;
+  if constexpr (SMEM_OFFS) {
+    if (warp == 3)
+      for (int i = lane; i <= p.E; i += 32) offs_smem[i] = p.offsets[i];
   }
   if (warp == 2 && (!MT::WGRAD || C::MX) && MODE != ROUTER) {
     // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
@@ -430,33 +451,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;  // per stage: a fill is in flight / its parity
-    uint32_t tarmed = 0, tlast = 0, tnext = 0;  // per stage: a tail fill was issued / the parity
-                                                // of the last one / of the next one
     bool ok = true;
     for (int t = tile0; t < ntiles && ok; t += tstep) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
+      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
       for (int kb = 0; kb < tl.num_kb && ok; ++kb) {
         if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 0); break; }
         const uint32_t a_dst = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
         const uint32_t b_dst = a_dst + C::A_BYTES;
-        int valid = C::KBLK;
-        if constexpr (MT::WGRAD && !C::MX) valid = min(C::KBLK, tl.rows - kb * C::KBLK);
-        const bool tail = valid < C::KBLK;
+        // bf16 weight gradients: the expert's last K-block, when partial, comes from the tail
+        // buffers (rows e*64 + i: the block's rows, then zeros)
+        bool tail = false;
+        if constexpr (MT::WGRAD && !C::MX) tail = tl.rows - kb * C::KBLK < C::KBLK;
         const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
         // pairs: the bytes of both CTAs' loads are counted on the leader's full barrier
         const uint32_t full_leader = CG == 2 ? ptx::mapa(full_local, 0) : full_local;
-        const uint32_t bar = tail ? ptx::smem_u32(&c.tailbar[stage]) : full_local;
-        const bool pair_load = CG == 2 && !tail;
+        const uint32_t bar = full_local;
         auto ld = [&](uint32_t dst, const CUtensorMap *tm, int x, int y) {
-          if (pair_load) ptx::tma_load_2d_pair(dst, tm, full_leader, x, y);
+          if (CG == 2) ptx::tma_load_2d_pair(dst, tm, full_leader, x, y);
           else ptx::tma_load_2d(dst, tm, bar, x, y);
         };
         if (lane == 0) {
-          if (tail) ptx::mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-          else if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES + C::SF_BYTES);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES + C::SF_BYTES);
           if constexpr (C::MX) {
             // the stage's scale-factor tiles, A then B (512 bytes each), straight into the
             // arrangement the MMA issuer's tcgen05.cp reads
@@ -479,8 +497,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // ---- A
           if constexpr (MT::A_MN) {
 #pragma unroll
-            for (int i = 0; i < BM / C::BOX_MN; ++i)
-              ld(a_dst + i * C::BOX_BYTES, &tmA, tl.mcol0 + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
+            for (int i = 0; i < BM / C::BOX_MN; ++i) {
+              if (tail) ld(a_dst + i * C::BOX_BYTES, &tmAT, tl.mcol0 + i * C::BOX_MN, tl.e * C::KBLK);
+              else ld(a_dst + i * C::BOX_BYTES, &tmA, tl.mcol0 + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
+            }
           } else {
             ld(a_dst, &tmA, kb * C::KBLK, tl.row0);
           }
@@ -535,39 +555,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ld(b_dst, &tmB1, (kb - kb_half) * C::KBLK, tl.e * p.d + tl.n_blk * BN + rank * BNC);
           } else {  // weight gradients: B is the MN-major activation gradient
 #pragma unroll
-            for (int i = 0; i < BNC / C::BOX_MN; ++i)
-              ld(b_dst + i * C::BOX_BYTES, &tmB0, tl.n_blk * BN + rank * BNC + i * C::BOX_MN, tl.row0 + kb * C::KBLK);
+            for (int i = 0; i < BNC / C::BOX_MN; ++i) {
+              const int x = tl.n_blk * BN + rank * BNC + i * C::BOX_MN;
+              if (tail) ld(b_dst + i * C::BOX_BYTES, &tmBT, x, tl.e * C::KBLK);
+              else ld(b_dst + i * C::BOX_BYTES, &tmB0, x, tl.row0 + kb * C::KBLK);
+            }
           }
         }
-        if (tail) {
-          // the tail fixer warp zeroes the rows past the expert and releases the stage; the
-          // copies of this fill are counted on the tail barrier, which the drain waits on
-          tarmed |= 1u << stage;
-          tlast = (tlast & ~(1u << stage)) | (tnext & (1u << stage));
-          tnext ^= 1u << stage;
-          armed &= ~(1u << stage);
-        } else {
-          // this stage's full barrier completes (or has completed) the phase of this pass
-          armed |= 1u << stage;
-          if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
-        }
+        // this stage's full barrier completes (or has completed) the phase of this pass
+        armed |= 1u << stage;
+        if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
         if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
       }
     }
     // Drain: every TMA fill this warp issued must land before the CTA may exit, also after
     // an abort (these waits ignore the abort flag and give up only at the limit).  The last
-    // fill of each stage is counted on its full barrier, or on its tail barrier for a tail
-    // fill; earlier fills of a stage had landed before the stage was refilled.  (Pairs: the
-    // leader's full barriers count the peer's bytes too; the peer only has tails.)
+    // fill of each stage is counted on its full barrier; earlier fills of a stage had landed
+    // before the stage was refilled.  (Pairs: the leader's full barriers count the peer's
+    // bytes too.)
     if (lane == 0) {
       for (int s = 0; s < C::STAGES; ++s)
         if (rank == 0 && ((armed >> s) & 1u))
           if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, nullptr, WAIT_LIMIT_NS))
             note_fail(p, 0, 0, s, 2);
-      for (int s = 0; s < C::STAGES; ++s)
-        if (((tarmed >> s) & 1u) &&
-            !ptx::mbar_wait(ptx::smem_u32(&c.tailbar[s]), (tlast >> s) & 1u, nullptr, WAIT_LIMIT_NS))
-          note_fail(p, 0, 0, s, 3);
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -590,7 +600,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       for (int t = tile0; t < ntiles && ok; t += tstep, ++it) {
         Tile tl;
-        get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
+        get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
         ok = ptx::mbar_wait(ptx::smem_u32(&c.tempty[acc]), aph ^ 1, abort_flag, WAIT_LIMIT_NS);
@@ -603,12 +613,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         for (int kb = 0; kb < tl.num_kb; ++kb) {
-          // Loaded bytes and commit arrivals are ordered by the barrier itself.  A weight-gradient
-          // tail stage was also zeroed by the peer's ordinary stores: that one wait takes a
-          // cluster-scope acquire, to see them before the pair MMA reads the peer's stage.
-          const bool peer_stores = CG == 2 && MT::WGRAD && kb == tl.num_kb - 1 && (tl.rows % C::KBLK) != 0;
-          ok = peer_stores ? ptx::mbar_wait_cluster(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS)
-                           : ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
+          // loaded bytes and commit arrivals are ordered by the barrier itself
+          ok = ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
           if (!ok) { note_fail(p, 1, t, kb, 1); break; }
           ptx::tc_fence_after();
           const uint32_t a_addr = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
@@ -622,7 +628,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tmem_cp_32x128b_x4(sfa_t, ptx::smem_desc_sf(sf_s));
             ptx::tmem_cp_32x128b_x4(sfb_t, ptx::smem_desc_sf(sf_s + 512));
           }
-          // a weight-gradient tail stage: only the UMMA_K-row slices that hold expert rows
+          // a weight-gradient tail stage: only the UMMA_K-row slices that hold expert rows (the
+          // rest of the tail buffer's block is zeros)
           int nk = C::KBLK / C::UMMA_K;
           if constexpr (MT::WGRAD && !C::MX)
             nk = min(nk, (tl.rows - kb * C::KBLK + C::UMMA_K - 1) / C::UMMA_K);
@@ -660,60 +667,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ptx::mbar_wait(ptx::smem_u32(&c.drain), 0, nullptr, WAIT_LIMIT_NS)) note_fail(p, 1, 0, 0, 2);
     }
     __syncwarp();
-  } else if (warp == FIX_WARP) {
-    // ================================================================ tail fixer
-    // Weight gradients reduce over an expert's rows: K rows of a stage past the expert's end
-    // belong to another expert (or lie outside the tensor).  This warp follows the producer's
-    // sequence of stages, zeroes those rows once a tail stage's loads have landed and then
-    // releases the stage to the MMA issuer, so that the producer never waits on a load.
-    if constexpr (MT::WGRAD && !C::MX) {
-      int stage = 0;
-      uint32_t tpar = 0;  // per stage: parity of the next tail completion
-      bool ok = true;
-      for (int t = tile0; t < ntiles && ok; t += tstep) {
-        Tile tl;
-        get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
-        for (int kb = 0; kb < tl.num_kb; ++kb) {
-          const int valid = min(C::KBLK, tl.rows - kb * C::KBLK);
-          if (valid < C::KBLK) {
-            ok = ptx::mbar_wait(ptx::smem_u32(&c.tailbar[stage]), (tpar >> stage) & 1u, abort_flag, WAIT_LIMIT_NS);
-            ok = __all_sync(0xffffffffu, ok);
-            if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
-            tpar ^= 1u << stage;
-            // In an MN-major box each K row is one 128-byte line.  The MMA issuer reads only
-            // the UMMA_K-row slices that hold expert rows, so rows [valid, round_up(valid,
-            // UMMA_K)), the byte range [valid*128, that*128) of every box, are zeroed.
-            const int nbox_a = BM / C::BOX_MN, nbox_b = BNC / C::BOX_MN;
-            const int line0 = valid * 8;                                           // 16-byte units
-            const int lines = ((valid + C::UMMA_K - 1) / C::UMMA_K) * C::UMMA_K * 8;
-            const uint4 z = make_uint4(0, 0, 0, 0);
-            for (int b = 0; b < nbox_a + nbox_b; ++b) {
-              uint8_t *box = ring + stage * C::STAGE_BYTES +
-                             (b < nbox_a ? b * C::BOX_BYTES : C::A_BYTES + (b - nbox_a) * C::BOX_BYTES);
-              for (int i = line0 + lane; i < lines; i += 32) reinterpret_cast<uint4 *>(box)[i] = z;
-            }
-            ptx::fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
-              if constexpr (CG == 2) {
-                // the leader arrives expecting the peer's bytes; the peer posts them once its
-                // zeroed stage is visible (the tensor cores of the pair read it)
-                if (rank == 0) {
-                  ptx::mbar_arrive_expect_tx(full_local, C::STAGE_BYTES);
-                } else {
-                  ptx::fence_acq_rel_cluster();
-                  ptx::mbar_complete_tx_cluster(ptx::mapa(full_local, 0), C::STAGE_BYTES);
-                }
-              } else {
-                ptx::mbar_arrive(full_local);
-              }
-            }
-          }
-          if (++stage == C::STAGES) stage = 0;
-        }
-      }
-    }
   } else {
     // ================================================================ epilogue
     using OutT = typename ElemTraits<T>::Out;
@@ -722,12 +675,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;
     const int half = (warp - 2) >> 2;     // 0 or 1
     const int r = q * 32 + lane;          // tile row owned by this thread
-    uint8_t *epi_box = extra + (warp - 2) * 2 * EPI_BOX_BYTES;   // weight gradients
-    int nst = 0;                          // weight gradients: boxes stored by this warp
+    uint8_t *epi_box = extra + (warp - 2) * EPI_BOX_BYTES;       // weight gradients
     int it = 0;
     for (int t = tile0; t < ntiles; t += tstep, ++it) {
       Tile tl;
-      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, tl, rank);
+      get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
       const int acc = it & 1;
       const uint32_t aph = (it >> 1) & 1;
       bool ok = ptx::mbar_wait(ptx::smem_u32(&c.tfull[acc]), aph, abort_flag, WAIT_LIMIT_NS);
@@ -1026,14 +978,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {  // weight gradients: rows q*32.. of the [M x N] block of expert e
-        // Each 32 x 64 piece goes through one of the warp's two staging boxes in the layout
-        // of a 128-byte-swizzled TMA box (16-byte chunk j of row r at chunk j ^ (r % 8)); one
-        // lane then stores the box with TMA.  A box is refilled only once the store that
-        // last used it has read it.
+        // Each 32 x 64 piece goes through the warp's staging box in the layout of a
+        // 128-byte-swizzled TMA box (16-byte chunk j of row r at chunk j ^ (r % 8)); one lane
+        // then stores the box with TMA.  The box is refilled only once the store that last
+        // used it has read it.
         static_assert(sizeof(OutT) == 2, "weight gradients are stored as bf16");
         const int orow = tl.e * p.M + tl.mcol0 + q * 32;
 #pragma unroll 1
-        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 64, ++nst) {
+        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 64) {
           float v0[32], v1[32];
           if (tl.num_kb > 0) {
             ptx::tmem_ld32(taddr + cc, v0);
@@ -1042,8 +994,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) { v0[i] = 0.f; v1[i] = 0.f; }
           }
-          uint8_t *box = epi_box + (nst & 1) * EPI_BOX_BYTES;
-          if (lane == 0) ptx::bulk_wait_read<1>();
+          uint8_t *box = epi_box;
+          if (lane == 0) ptx::bulk_wait_read<0>();
           __syncwarp();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -1155,7 +1107,8 @@ static std::atomic<uint64_t> g_stall_ns{0};
 template <typename T, int BN, int MODE, int CG = 1>
 static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap &b1, const Params &p_in,
                   int64_t max_tiles, cudaStream_t st, const CUtensorMap *o0 = nullptr,
-                  const CUtensorMap *o1 = nullptr) {
+                  const CUtensorMap *o1 = nullptr, const CUtensorMap *at = nullptr,
+                  const CUtensorMap *bt = nullptr) {
   using C = Cfg<T, BN, CG, extra_smem<MODE>()>;
   Params p = p_in;
   p.stall_ns = CG == 1 ? g_stall_ns.load(std::memory_order_relaxed) : 0;
@@ -1163,7 +1116,9 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   constexpr int SMEM = C::SMEM_BYTES;
   static_assert(SMEM <= SMEM_LIMIT, "shared memory");
   if (ModeTraits<MODE>::WGRAD && (!o0 || !o1)) return MOE_ERR_INVALID_ARG;
+  if (ModeTraits<MODE>::WGRAD && !C::MX && (!at || !bt)) return MOE_ERR_INVALID_ARG;
   const CUtensorMap &out0 = o0 ? *o0 : a, &out1 = o1 ? *o1 : a;
+  const CUtensorMap &atail = at ? *at : a, &btail = bt ? *bt : a;
   // the shared-memory opt-in is a per-device property of the kernel: set once per device
   // (two threads racing here both set it, which is harmless)
   static std::atomic<bool> attr_set[MAX_DEVICES];
@@ -1175,7 +1130,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   }
   if constexpr (CG == 1) {
     const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
-    kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, out0, out1, p);
+    kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, out0, out1, atail, btail, p);
   } else {
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(NUM_THREADS);
@@ -1202,7 +1157,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
     }
     const int64_t units = std::min<int64_t>(max_pairs, std::max<int64_t>(max_tiles, 1));
     cfg.gridDim = dim3((unsigned)(units * CG));
-    if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, out0, out1, p) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, out0, out1, atail, btail, p) != cudaSuccess) return MOE_ERR_CUDA;
   }
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -1287,11 +1242,16 @@ template <typename T>
 static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                     const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
                     const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
-                    void *dw_down, int *err, cudaStream_t st) {
+                    void *dw_down, void *ws, cudaStream_t st) {
   constexpr int ES = sizeof(T);
   constexpr int KBLK = 128 / ES, BOX_MN = 128 / ES;
+  static_assert(KBLK == WGRAD_TAIL_ROWS, "tail buffers hold one K-block per expert");
   const int64_t P = s.P();
-  CUtensorMap tA, tB0, tB1;
+  int *err = err_word(ws);
+  const WsLayout L = ws_layout(s);
+  void *tail_a = static_cast<char *>(ws) + L.wg_tail_a, *tail_b = static_cast<char *>(ws) + L.wg_tail_b;
+  const uint64_t tail_rows = (uint64_t)s.E * WGRAD_TAIL_ROWS;
+  CUtensorMap tA, tB0, tB1, tAT, tBT;
   Params p{};
   p.offsets = offsets; p.E = s.E; p.P = (int)P; p.f = s.f; p.d = s.d; p.err = err; p.where = err + 1;
   const int64_t mblocks = (P + BM - 1) / BM + s.E;
@@ -1315,6 +1275,12 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   }
   // (2) dWd[e] = a^T [f, rows_e] x dy_perm [rows_e, d]
   {
+    // every expert's last partial K-block of a and dy_perm, zero past the expert's rows
+    if (launch_wgrad_tails(a, s.f, offsets, s.E, tail_a, st) || launch_wgrad_tails(dy_perm, s.d, offsets, s.E, tail_b, st))
+      return MOE_ERR_CUDA;
+    if (!make_tmap(&tAT, tail_a, ES, s.f, tail_rows, BOX_MN, KBLK) ||
+        !make_tmap(&tBT, tail_b, ES, s.d, tail_rows, BOX_MN, KBLK))
+      return MOE_ERR_CUDA;
     CUtensorMap tO;
     if (!make_tmap(&tO, dw_down, ES, s.d, (uint64_t)s.E * s.f, 64, 32)) return MOE_ERR_CUDA;
     if (!make_tmap(&tA, a, ES, s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
@@ -1322,13 +1288,16 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
     if (s.d % 256 == 0 && s.f % 256 == 0) {
       // weight-gradient tiles are 256 weight rows (no empty rows): always CTA pairs
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 256, WGRAD_DOWN, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / 256) * (s.d / 256), st, &tO, &tO);
+      rc = launch<T, 256, WGRAD_DOWN, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / 256) * (s.d / 256), st, &tO, &tO,
+                                         &tAT, &tBT);
     } else if (s.d % 256 == 0) {
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st, &tO, &tO);
+      rc = launch<T, 256, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 256), st, &tO, &tO, &tAT,
+                                      &tBT);
     } else {
       if (!make_tmap(&tB0, dy_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
-      rc = launch<T, 128, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st, &tO, &tO);
+      rc = launch<T, 128, WGRAD_DOWN>(tA, tB0, tB0, p, (int64_t)s.E * (s.f / BM) * (s.d / 128), st, &tO, &tO, &tAT,
+                                      &tBT);
     }
     if (rc) return rc;
   }
@@ -1353,6 +1322,12 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   }
   // (4) [dWg | dWu][e] = x_perm^T [d, rows_e] x dhu [rows_e, 2f]
   {
+    if (launch_wgrad_tails(x_perm, s.d, offsets, s.E, tail_a, st) ||
+        launch_wgrad_tails(dhu, 2 * s.f, offsets, s.E, tail_b, st))
+      return MOE_ERR_CUDA;
+    if (!make_tmap(&tAT, tail_a, ES, s.d, tail_rows, BOX_MN, KBLK) ||
+        !make_tmap(&tBT, tail_b, ES, 2 * s.f, tail_rows, BOX_MN, KBLK))
+      return MOE_ERR_CUDA;
     if (!make_tmap(&tA, x_perm, ES, s.d, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     if (!make_tmap(&tB0, dhu, ES, 2 * s.f, P, BOX_MN, KBLK)) return MOE_ERR_CUDA;
     CUtensorMap tO0, tO1;
@@ -1361,11 +1336,14 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
       return MOE_ERR_CUDA;
     p.M = s.d; p.N = 2 * s.f; p.out0 = dw_gate; p.out1 = dw_up;
     if (s.f % 256 == 0 && s.d % 256 == 0)
-      rc = launch<T, 256, WGRAD_GU, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / 256) * (2 * s.f / 256), st, &tO0, &tO1);
+      rc = launch<T, 256, WGRAD_GU, 2>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / 256) * (2 * s.f / 256), st, &tO0, &tO1,
+                                       &tAT, &tBT);
     else if (s.f % 256 == 0)
-      rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st, &tO0, &tO1);
+      rc = launch<T, 256, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 256), st, &tO0, &tO1,
+                                    &tAT, &tBT);
     else
-      rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st, &tO0, &tO1);
+      rc = launch<T, 128, WGRAD_GU>(tA, tB0, tB0, p, (int64_t)s.E * (s.d / BM) * (2 * s.f / 128), st, &tO0, &tO1,
+                                    &tAT, &tBT);
     if (rc) return rc;
   }
   return MOE_OK;
@@ -1564,7 +1542,7 @@ int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, 
     return gg::mx_bwd_impl(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm, dw_gate,
                            dw_up, dw_down, ws, st, wsaved, dy_quantized);
   return gg::bwd_impl<bf16>(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
-                            dw_gate, dw_up, dw_down, err_word(ws), st);
+                            dw_gate, dw_up, dw_down, ws, st);
 }
 
 }  // namespace moe

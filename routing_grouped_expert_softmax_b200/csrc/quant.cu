@@ -16,6 +16,8 @@
 // Activation operands are written into expert buffers padded to 128 rows: padded row
 // 128*pre[e] + i holds source row offsets[e] + i for i < count_e and zeros after, where
 // pre[e] = sum_{e' < e} ceil(count_e' / 128).
+#include <atomic>
+
 #include "common.cuh"
 #include "mxfp8.cuh"
 
@@ -246,87 +248,167 @@ __global__ void __launch_bounds__(256) mx_quant_rows_gu_kernel(const bf16 *__res
   }
 }
 
-// ---- weights in both orientations from one read.  A block takes a tile of 32 rows x 128
-// columns: for the gate/up pair (gu) 64 columns of W_gate and the same 64 of W_up, else 128
-// columns of one tensor [R][C].  From the tile it writes
+// ---- weights in both orientations from one read.  A block takes 128 rows and NC "tile
+// columns": for the gate/up pair (gu) 128 columns of W_gate and the same 128 of W_up (NC = 256,
+// in the interleaved output order below), else NC = 256 (or 128 when C % 256 != 0) columns of
+// one tensor [R][C].  From the tile it writes
 //   codes_c: blocks of 32 down the rows (the forward GEMMs' K), [R][C'] with C' = 2f for the
 //            pair (gate and up interleaved in 64-column chunks: output column 128 J + i is gate
 //            column 64 J + i for i < 64, up column 64 J + i - 64 otherwise) or C;
 //   codes_r: blocks of 32 along the row (the data-gradient GEMMs' K), [R][C'] with row r of the
 //            pair [W_gate[r] | W_up[r]];
-// scales of both in the tile layout.  Same arithmetic as the single-orientation kernels.
-constexpr int WQ_ROWS = 32, WQ_COLS = 128;
-__global__ void __launch_bounds__(256) mx_quant_weights_kernel(const bf16 *__restrict__ w0, const bf16 *__restrict__ w1,
-                                                               int64_t R, int C, bool gu,
-                                                               uint8_t *__restrict__ codes_c,
-                                                               uint8_t *__restrict__ scales_c,
-                                                               uint8_t *__restrict__ codes_r,
-                                                               uint8_t *__restrict__ scales_r) {
-  __shared__ float tile[WQ_ROWS][WQ_COLS + 1];
-  __shared__ float inv_c[WQ_COLS], inv_r[WQ_ROWS][4];
+// and the scales of both in the tile layout.  128 rows hold four 32-row blocks and NC columns
+// whole 128-column groups, so the block owns whole 512-byte scale tiles: it assembles them in
+// shared memory and writes them with 16-byte stores.  Same arithmetic as the single-orientation
+// kernels (block maxima of the bf16 values, scale rule, E4M3 rounding).
+constexpr int WQ_ROWS = 128, WQ_THREADS = 512, WQ_NC_MAX = 256, WQ_PAD = 8;
+constexpr size_t WQ_TILE_BYTES = (size_t)WQ_ROWS * (WQ_NC_MAX + WQ_PAD) * 2;
+// the tile, the inverse scales and the two staged scale tiles of each orientation (two blocks
+// fit on an SM)
+constexpr size_t WQ_SMEM = WQ_TILE_BYTES + 4 * WQ_NC_MAX * 4 + WQ_ROWS * (WQ_NC_MAX / 32) * 4 + 2 * 2 * 512;
+
+struct WqMap {
+  bool gu;
+  int C, NC, c0;
+  // source tensor (0 or 1) and column of tile column j
+  __device__ __forceinline__ int tensor(int j) const { return gu ? (j >> 6) & 1 : 0; }
+  __device__ __forceinline__ int src_col(int j) const { return gu ? c0 + 64 * (j >> 7) + (j & 63) : c0 + j; }
+  // output column of tile column j: column-blocked (interleaved for the pair) and row-blocked
+  __device__ __forceinline__ int ccol(int j) const { return gu ? 2 * c0 + j : c0 + j; }
+  __device__ __forceinline__ int rcol(int j) const { return tensor(j) * C + src_col(j); }
+};
+
+// One block per tile (tile column block blockIdx.x, row block blockIdx.y).
+template <bool GU, int NC>
+__global__ void __launch_bounds__(WQ_THREADS) mx_quant_weights_kernel(
+    const bf16 *__restrict__ w0, const bf16 *__restrict__ w1, int64_t R, int C,
+    uint8_t *__restrict__ codes_c, uint8_t *__restrict__ scales_c, uint8_t *__restrict__ codes_r,
+    uint8_t *__restrict__ scales_r) {
+  extern __shared__ __align__(16) uint8_t wq_smem[];
+  constexpr bool gu = GU;
+  constexpr int pitch = NC + WQ_PAD;                                    // bf16 elements per row
+  bf16 *tile = reinterpret_cast<bf16 *>(wq_smem);                       // [128][pitch]
+  float *inv_c = reinterpret_cast<float *>(wq_smem + WQ_TILE_BYTES);    // [4][NC]
+  float *inv_r = inv_c + 4 * NC;                                        // [128][NC/32]
+  uint8_t *st_c = reinterpret_cast<uint8_t *>(inv_r + WQ_ROWS * (NC / 32));   // [NC/128][512]
+  uint8_t *st_r = st_c + (NC / 128) * 512;                              // [NC/128][512]
+  const WqMap m{gu, C, NC, (int)blockIdx.x * (gu ? 128 : NC)};
   const int t = threadIdx.x;
   const int64_t r0 = (int64_t)blockIdx.y * WQ_ROWS;
-  const int CO = gu ? 2 * C : C;                    // output columns per row
-  // source column of tile column j: (tensor, column)
-  auto src_of = [&](int j, const bf16 *&w, int &col) {
-    if (gu) { w = j < 64 ? w0 : w1; col = blockIdx.x * 64 + (j & 63); }
-    else { w = w0; col = blockIdx.x * WQ_COLS + j; }
-  };
-  // output column of tile column j in the row-blocked layout
-  auto rcol_of = [&](int j) { return gu ? (j < 64 ? 0 : C) + (int)blockIdx.x * 64 + (j & 63)
-                                        : (int)blockIdx.x * WQ_COLS + j; };
-  const int ccol0 = blockIdx.x * WQ_COLS;           // first output column in the column-blocked layout
+  const int CO = gu ? 2 * C : C;
+  // (1) the tile, 16-byte pieces (8 tile columns of one chunk each): every load of the thread
+  // in flight at once, then the shared-memory stores
+  constexpr int vpr = NC / 8, NLD = WQ_ROWS * vpr / WQ_THREADS;
+  uint4 ld[NLD];
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {                     // 512 16-byte pieces, two per thread
-    const int idx = t + 256 * i, row = idx >> 4, j = (idx & 15) * 8;
-    const bf16 *w;
-    int col;
-    src_of(j, w, col);
-    float v[8];
-    Vec<bf16>::load(__ldg(reinterpret_cast<const uint4 *>(w + (r0 + row) * C + col)), v);
+  for (int q = 0; q < NLD; ++q) {
+    const int idx = t + q * WQ_THREADS, row = idx / vpr, j = (idx - row * vpr) * 8;
+    const bf16 *w = m.tensor(j) ? w1 : w0;
+    ld[q] = __ldg(reinterpret_cast<const uint4 *>(w + (r0 + row) * C + m.src_col(j)));
+  }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) tile[row][j + e] = v[e];
+  for (int q = 0; q < NLD; ++q) {
+    const int idx = t + q * WQ_THREADS, row = idx / vpr, j = (idx - row * vpr) * 8;
+    *reinterpret_cast<uint4 *>(tile + row * pitch + j) = ld[q];
   }
   __syncthreads();
-  if (t < WQ_COLS) {                                 // column scales: one 32-row block per column
-    float amax = 0.f;
+  // (2) scales.  Column blocks: 4 row groups x NC columns, two adjacent columns per task
+  // (32 paired loads); row blocks: 128 rows x NC/32, 32 values as 4 vectors per task.
+  for (int u = t; u < 2 * NC; u += WQ_THREADS) {
+    const int grp = u / (NC / 2), j = 2 * (u - grp * (NC / 2));
+    float a0 = 0.f, a1 = 0.f;
 #pragma unroll 8
-    for (int r = 0; r < WQ_ROWS; ++r) amax = fmaxf(amax, fabsf(tile[r][t]));
-    const int sc = mx_scale_exp(amax);
-    inv_c[t] = exp2_neg(sc);
-    scales_c[sf_tiled_off(ccol0 + t, r0 / 32, R / 128)] = (uint8_t)(sc + 127);
-  } else {                                          // row scales: 4 blocks of 32 columns per row
-    const int u = t - WQ_COLS, row = u >> 2, b = u & 3;
+    for (int r = 0; r < 32; ++r) {
+      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + (grp * 32 + r) * pitch + j));
+      a0 = fmaxf(a0, fabsf(v.x));
+      a1 = fmaxf(a1, fabsf(v.y));
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int sc = mx_scale_exp(h ? a1 : a0);
+      inv_c[grp * NC + j + h] = exp2_neg(sc);
+      const int mn = m.ccol(j + h) & 127;                               // the tile's base is a multiple of 128
+      st_c[((j + h) >> 7) * 512 + 16 * (mn & 31) + 4 * (mn >> 5) + grp] = (uint8_t)(sc + 127);
+    }
+  }
+  constexpr int nb = NC / 32;
+  for (int u = t; u < WQ_ROWS * nb; u += WQ_THREADS) {
+    const int row = u / nb, b = u - row * nb, j = 32 * b;
     float amax = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(tile[row][32 * b + j]));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float v[8];
+      Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j + 8 * i), v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    }
     const int sc = mx_scale_exp(amax);
-    inv_r[row][b] = exp2_neg(sc);
-    scales_r[sf_tiled_off(r0 + row, rcol_of(32 * b) / 32, CO / 128)] = (uint8_t)(sc + 127);
+    inv_r[row * nb + b] = exp2_neg(sc);
+    const int kb = m.rcol(j) / 32;                                      // K-block along the row
+    const int ti = gu ? m.tensor(j) : (j >> 7);                         // which staged tile
+    st_r[ti * 512 + 16 * (row & 31) + 4 * (row >> 5) + (kb & 3)] = (uint8_t)(sc + 127);
   }
   __syncthreads();
-  // codes: thread t writes 16 consecutive tile columns of one row in both layouts
-  const int row = t >> 3, j0 = (t & 7) * 16;
-  uint32_t wc[4], wr[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int j = j0 + 4 * q;
-    const float ir = inv_r[row][j >> 5];
-    wc[q] = (uint32_t)e4m3x2(tile[row][j] * inv_c[j], tile[row][j + 1] * inv_c[j + 1]) |
-            ((uint32_t)e4m3x2(tile[row][j + 2] * inv_c[j + 2], tile[row][j + 3] * inv_c[j + 3]) << 16);
-    wr[q] = (uint32_t)e4m3x2(tile[row][j] * ir, tile[row][j + 1] * ir) |
-            ((uint32_t)e4m3x2(tile[row][j + 2] * ir, tile[row][j + 3] * ir) << 16);
+  // (3) the staged scale tiles, whole, with 16-byte stores
+  for (int u = t; u < 2 * (NC / 128) * 32; u += WQ_THREADS) {
+    const int which = u / ((NC / 128) * 32), rest = u - which * (NC / 128) * 32, ti = rest >> 5, q = rest & 31;
+    if (which == 0) {
+      const int64_t mnb = m.ccol(ti * 128) / 128, kg = r0 / 128;
+      reinterpret_cast<uint4 *>(scales_c + (mnb * (R / 128) + kg) * 512)[q] =
+          reinterpret_cast<const uint4 *>(st_c + ti * 512)[q];
+    } else {
+      const int64_t mnb = r0 / 128, kg = m.rcol(gu ? ti * 64 : ti * 128) / 128;
+      reinterpret_cast<uint4 *>(scales_r + (mnb * (CO / 128) + kg) * 512)[q] =
+          reinterpret_cast<const uint4 *>(st_r + ti * 512)[q];
+    }
   }
-  *reinterpret_cast<uint4 *>(codes_c + (r0 + row) * CO + ccol0 + j0) = make_uint4(wc[0], wc[1], wc[2], wc[3]);
-  *reinterpret_cast<uint4 *>(codes_r + (r0 + row) * CO + rcol_of(j0)) = make_uint4(wr[0], wr[1], wr[2], wr[3]);
+  // (4) codes: 16 tile columns of one row per task, in both orientations
+  constexpr int vr = NC / 16;
+  for (int u = t; u < WQ_ROWS * vr; u += WQ_THREADS) {
+    const int row = u / vr, j0 = (u - row * vr) * 16, grp = row >> 5;
+    float v[16];
+    Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j0), v);
+    Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j0 + 8), v + 8);
+    const float ir = inv_r[row * nb + j0 / 32];
+    const float *ic = inv_c + grp * NC + j0;
+    uint32_t wc[4], wr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      wc[q] = (uint32_t)e4m3x2(v[4 * q] * ic[4 * q], v[4 * q + 1] * ic[4 * q + 1]) |
+              ((uint32_t)e4m3x2(v[4 * q + 2] * ic[4 * q + 2], v[4 * q + 3] * ic[4 * q + 3]) << 16);
+      wr[q] = (uint32_t)e4m3x2(v[4 * q] * ir, v[4 * q + 1] * ir) |
+              ((uint32_t)e4m3x2(v[4 * q + 2] * ir, v[4 * q + 3] * ir) << 16);
+    }
+    *reinterpret_cast<uint4 *>(codes_c + (r0 + row) * CO + m.ccol(j0)) = make_uint4(wc[0], wc[1], wc[2], wc[3]);
+    *reinterpret_cast<uint4 *>(codes_r + (r0 + row) * CO + m.rcol(j0)) = make_uint4(wr[0], wr[1], wr[2], wr[3]);
+  }
+}
+
+template <bool GU, int NC>
+static cudaError_t launch_wq(const void *w0, const void *w1, int64_t R, int C, uint8_t *codes_c, uint8_t *scales_c,
+                             uint8_t *codes_r, uint8_t *scales_r, cudaStream_t st) {
+  // the dynamic shared-memory opt-in is a per-device property of the kernel
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!(attr_set.load(std::memory_order_acquire) >> dev & 1ull)) {
+    cudaError_t e = cudaFuncSetAttribute(mx_quant_weights_kernel<GU, NC>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)WQ_SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set.fetch_or(1ull << dev, std::memory_order_acq_rel);
+  }
+  dim3 grid((unsigned)(GU ? C / 128 : C / NC), (unsigned)(R / WQ_ROWS));
+  if (grid.x == 0 || grid.y == 0) return cudaSuccess;
+  mx_quant_weights_kernel<GU, NC><<<grid, WQ_THREADS, WQ_SMEM, st>>>(
+      static_cast<const bf16 *>(w0), static_cast<const bf16 *>(w1), R, C, codes_c, scales_c, codes_r, scales_r);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_mx_quant_weights(const void *w0, const void *w1, int64_t R, int C, bool gu, uint8_t *codes_c,
                                     uint8_t *scales_c, uint8_t *codes_r, uint8_t *scales_r, cudaStream_t st) {
-  dim3 grid((unsigned)(gu ? C / 64 : C / WQ_COLS), (unsigned)(R / WQ_ROWS));
-  mx_quant_weights_kernel<<<grid, 256, 0, st>>>(static_cast<const bf16 *>(w0), static_cast<const bf16 *>(w1), R, C,
-                                                gu, codes_c, scales_c, codes_r, scales_r);
-  return cudaGetLastError();
+  if (gu) return launch_wq<true, 256>(w0, w1, R, C, codes_c, scales_c, codes_r, scales_r, st);
+  if (C % 256 == 0) return launch_wq<false, 256>(w0, w1, R, C, codes_c, scales_c, codes_r, scales_r, st);
+  return launch_wq<false, 128>(w0, w1, R, C, codes_c, scales_c, codes_r, scales_r, st);
 }
 
 // ---- FP8 dispatch: x_perm[slot(t,j)] = x[t] (a bit copy) and, in the same pass, the row in

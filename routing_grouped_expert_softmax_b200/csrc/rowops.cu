@@ -448,6 +448,35 @@ cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, cons
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------------------
+// Tail buffers of the bf16 weight-gradient GEMMs, which reduce over each expert's rows in
+// K-blocks of 64: the expert's last, partial block is copied into its own 64 rows with zeros
+// after the expert's rows, so that the GEMM loads it like any other block.  One block per
+// (row i of the tail, expert e).
+// ---------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) wgrad_tail_kernel(const uint4 *__restrict__ src, int nv,
+                                                         const int32_t *__restrict__ offsets,
+                                                         uint4 *__restrict__ tails) {
+  const int i = blockIdx.x, e = blockIdx.y;
+  const int lo = offsets[e], cnt = offsets[e + 1] - lo;
+  const int full = cnt / WGRAD_TAIL_ROWS * WGRAD_TAIL_ROWS, v = cnt - full;
+  if (v == 0) return;                        // no partial block: the tail rows are never read
+  uint4 *dst = tails + ((int64_t)e * WGRAD_TAIL_ROWS + i) * nv;
+  if (i < v) {
+    const uint4 *row = src + ((int64_t)lo + full + i) * nv;
+    for (int c = threadIdx.x; c < nv; c += 128) dst[c] = __ldg(row + c);
+  } else {
+    for (int c = threadIdx.x; c < nv; c += 128) dst[c] = make_uint4(0, 0, 0, 0);
+  }
+}
+
+cudaError_t launch_wgrad_tails(const void *src, int C, const int32_t *offsets, int E, void *tails, cudaStream_t st) {
+  dim3 grid(WGRAD_TAIL_ROWS, (unsigned)E);
+  wgrad_tail_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4 *>(src), C * 2 / 16, offsets,
+                                          static_cast<uint4 *>(tails));
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------------------ launchers
 static unsigned row_grid(int64_t T) { return (unsigned)((T + ROW_WARPS - 1) / ROW_WARPS); }
 
