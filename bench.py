@@ -328,13 +328,21 @@ def run_ours(args):
     # ---- the grouped GEMMs alone (6 tcgen05 launches per step), same stream and inputs
     g0, g1, g2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
     hu_buf = saved["hu"] if saved["hu"] is not None else grads["dhu"]   # recompute keeps no h | u
+    x_perm, dy_perm = saved["x_perm"], grads["dy_perm"]
+    if x_perm is None:     # the MXFP8 layer moved the rows in MXFP8 only: make the bf16 ones
+        x_perm = torch.empty(L.T * L.k, L.d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_permute(cfg, L.x, saved["slot_of_pair"], x_perm, st)
+    if dy_perm is None:
+        dy_perm = torch.empty(L.T * L.k, L.d, dtype=torch.bfloat16, device="cuda")
+        moe.moe_combine_bwd(cfg, L.dy, saved["y_perm"], saved["slot_of_pair"], saved["topk_gate"], dy_perm,
+                            grads["dgate"], st)
     fwd_ms = bwd_ms = 0.0
     for _ in range(args.steps):
         g0.record(st)
-        moe.moe_grouped_swiglu_fwd(cfg, saved["x_perm"], saved["offsets"], wg, wu, wd, hu_buf,
+        moe.moe_grouped_swiglu_fwd(cfg, x_perm, saved["offsets"], wg, wu, wd, hu_buf,
                                    saved["a"], saved["y_perm"], ws, st)
         g1.record(st)
-        moe.moe_grouped_swiglu_bwd(cfg, grads["dy_perm"], saved["x_perm"], hu_buf, saved["a"],
+        moe.moe_grouped_swiglu_bwd(cfg, dy_perm, x_perm, hu_buf, saved["a"],
                                    saved["offsets"], wg, wu, wd, grads["dhu"], grads["dx_perm"],
                                    grads["dw_gate"], grads["dw_up"], grads["dw_down"], ws, st)
         g2.record(st)
@@ -544,7 +552,8 @@ def gemm_algorithmic_bytes(P, d, f, E, prec):
 def count_launches(routing, prec="native", shared=False, recompute=False):
     """Kernels one step launches (the fallback when the CUPTI count is unavailable): forward
     (router 1, metadata 3, permute 1, grouped GEMMs 2, combine 1) and backward (combine-bwd 1,
-    grouped GEMMs 4, router transpose 1, router weight-gradient 3, unpermute-sum 1).  MXFP8
+    grouped GEMMs 4, router transpose 1, router weight-gradient 3, unpermute-sum 1; bf16: one
+    tail-buffer copy before each weight-gradient GEMM, per expert set).  MXFP8
     with the forward's weight copies kept for the backward adds 2 weight quantisers forward
     (the permute and the gate/up epilogue quantise x and a) and 2 token-axis quantisers
     backward (the combine's backward and the down projection's epilogue quantise dy and
@@ -554,8 +563,8 @@ def count_launches(routing, prec="native", shared=False, recompute=False):
     fwd = (1 if routing == "router" else 0) + 3 + 1 + 2 + 1
     bwd = 1 + 4 + (5 if routing == "router" else 1)
     mx = prec == "mxfp8"
-    n = fwd + bwd + (4 if mx else 0)
     sets = 2 if shared else 1
+    n = fwd + bwd + (4 if mx else 2 * sets)
     if shared:
         n += 1 + 2 + 1 + 4 + (10 if mx else 0)
     if recompute:

@@ -238,6 +238,23 @@ MOE_API int moe_permute_mxfp8(const moe_config *cfg, const void *x, const int32_
                               const int32_t *offsets, void *x_perm, int64_t rows_bound,
                               uint8_t *codes, uint8_t *scales, moe_stream_t stream);
 
+/* FP8 dispatch in both orientations (same passage): each routed row of x is read once, in
+ * slot order through pair_of_slot, and written in MXFP8 twice on the expert-padded layout
+ * (padded row 128*pre[e] + i holds x[pair_of_slot[offsets[e] + i] / k] for i < count_e and
+ * zeros after, up to 128*pre[E]):
+ *   codes_r [rows_bound][d], scales_r [rows_bound][d/32]: blocks of 32 along d (the forward
+ *     GEMM's operand), as moe_mx_quantize_rows with offsets;
+ *   codes_c [rows_bound][d], scales_c [rows_bound/32][d]: blocks of 32 padded rows (the
+ *     weight gradient's operand), as moe_mx_quantize_cols with offsets.
+ * x_perm [P,d] or NULL: the bf16 bit copy of moe_permute as well.  The pad rows are written
+ * (zeros, scale byte 0); rows past 128*pre[E] are left as they were.  bf16 only (else
+ * MOE_ERR_UNSUPPORTED); rows_bound >= T*k + 127*E (else MOE_ERR_INVALID_ARG); x, x_perm, codes 16-byte aligned, pair_of_slot, offsets, scales
+ * 4-byte aligned; pair_of_slot and offsets from moe_build_offsets. */
+MOE_API int moe_dispatch_mxfp8(const moe_config *cfg, const void *x, const int32_t *pair_of_slot,
+                               const int32_t *offsets, int64_t rows_bound, void *x_perm,
+                               uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
+                               uint8_t *scales_c, moe_stream_t stream);
+
 MOE_API int moe_mx_quantize_rows(const void *src, int64_t rows, int32_t cols, const int32_t *offsets,
                                  int32_t E, int64_t rows_bound, uint8_t *codes, uint8_t *scales,
                                  moe_stream_t stream);
@@ -261,6 +278,20 @@ MOE_API int moe_unpermute_combine(const moe_config *cfg, const void *y_perm,
 MOE_API int moe_combine_bwd(const moe_config *cfg, const void *dy, const void *y_perm,
                     const int32_t *slot_of_pair, const float *topk_gate, void *dy_perm,
                     float *dgate, moe_stream_t stream);
+
+/* The combine's backward with its output dispatched in MXFP8 (unite.ai, section
+ * "Παραλληλισμός, Ακρίβεια και Τεχνικές Μνήμης": MXFP8 for the data moved between experts):
+ * for each slot, in the order of pair_of_slot, dy_perm row = bf16(g * dy[t]) (the fp32
+ * product rounded to bf16) and dgate[t,j] = <dy[t], y_perm[slot]> (fp32); the bf16 row is
+ * then written in MXFP8 in both orientations exactly as moe_dispatch_mxfp8 writes x's rows
+ * (codes_r/scales_r along d, codes_c/scales_c down the padded token axis).  dy_perm [P,d] or
+ * NULL: the bf16 rows as well.  Arguments, alignment and errors as moe_dispatch_mxfp8, with
+ * y_perm [P,d] bf16, topk_gate [T,k] fp32 and dgate [T,k] fp32 out (4-byte aligned). */
+MOE_API int moe_combine_bwd_mxfp8(const moe_config *cfg, const void *dy, const void *y_perm,
+                                  const int32_t *pair_of_slot, const int32_t *offsets,
+                                  const float *topk_gate, int64_t rows_bound, void *dy_perm,
+                                  float *dgate, uint8_t *codes_r, uint8_t *scales_r,
+                                  uint8_t *codes_c, uint8_t *scales_c, moe_stream_t stream);
 
 /* (source: as moe_permute; its chain rule)
  * Backward of the permute: dx[t] = sum_j dx_perm[slot(t,j)] (fp32 sum).
@@ -303,7 +334,7 @@ typedef struct moe_layer_saved {
   int32_t *offsets;       /* [E+1] */
   int32_t *slot_of_pair;  /* [P] */
   int32_t *pair_of_slot;  /* [P] */
-  void *x_perm;           /* [P,d] */
+  void *x_perm;           /* [P,d]; unused (may be NULL) with mx_saved */
   void *hu;               /* [P,2f] (h | u), or NULL: the backward recomputes them */
   void *a;                /* [P,f] */
   void *y_perm;           /* [P,d] */
@@ -312,8 +343,11 @@ typedef struct moe_layer_saved {
   /* MOE_PREC_MXFP8 only, or NULL: moe_mx_saved_bytes(cfg) bytes (256-byte aligned) that the
    * forward fills with MXFP8 copies (E4M3 codes with E8M0 scales, the layout is internal) the
    * backward reads instead of quantising again: the routed experts' weights in the orientation
-   * of every GEMM that reads them, and x_perm and a along the token axis.  The weights must not
-   * change between the two calls.  NULL: each call quantises what it needs in the workspace. */
+   * of every GEMM that reads them, the routed rows of x along d and along the token axis, and
+   * a along the token axis.  The routed rows then move in MXFP8 only (the FP8 dispatch): x_perm
+   * is neither written nor read, and the router's weight gradient reads x through
+   * pair_of_slot.  The weights must not change between the two calls.  NULL: the forward also
+   * writes the bf16 x_perm, and each call quantises what it needs in the workspace. */
   void *mx_saved;
 } moe_layer_saved;
 
@@ -324,7 +358,8 @@ typedef struct moe_layer_grads {
   void *dw_gate;     /* [E,d,f] */
   void *dw_up;       /* [E,d,f] */
   void *dw_down;     /* [E,f,d] */
-  void *dy_perm;     /* [P,d] intermediate */
+  void *dy_perm;     /* [P,d] intermediate; unused (may be NULL) with MOE_PREC_MXFP8, where the
+                        combine's backward writes it in MXFP8 only */
   float *dgate;      /* [T,k] intermediate */
   void *dhu;         /* [P,2f] intermediate (also holds recomputed h | u) */
   void *dx_perm;     /* [P,d] intermediate */

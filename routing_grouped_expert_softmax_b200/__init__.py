@@ -37,6 +37,7 @@ EXPORTED = [
     "moe_unpermute_combine", "moe_combine_bwd", "moe_unpermute_sum", "moe_route_bwd",
     "moe_layer_fwd", "moe_layer_fwd_routed", "moe_layer_bwd", "moe_mx_quantize_rows",
     "moe_mx_quantize_cols", "moe_permute_mxfp8", "moe_debug_set_gemm_stall_ns", "moe_mx_saved_bytes",
+    "moe_dispatch_mxfp8", "moe_combine_bwd_mxfp8",
 ]
 
 
@@ -110,6 +111,9 @@ def lib() -> ctypes.CDLL:
             "moe_mx_quantize_cols": (ctypes.c_int, [_P, ctypes.c_int64, ctypes.c_int32, _P, ctypes.c_int32,
                                                     ctypes.c_int64, _P, _P, _P]),
             "moe_permute_mxfp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, ctypes.c_int64, _P, _P, _P]),
+            "moe_dispatch_mxfp8": (ctypes.c_int, [_CFG, _P, _P, _P, ctypes.c_int64, _P, _P, _P, _P, _P, _P]),
+            "moe_combine_bwd_mxfp8": (ctypes.c_int, [_CFG, _P, _P, _P, _P, _P, ctypes.c_int64, _P, _P, _P, _P,
+                                                     _P, _P, _P]),
             "moe_layer_fwd": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
                                              ctypes.POINTER(LayerSaved), _P, _P]),
             "moe_layer_fwd_routed": (ctypes.c_int, [_CFG, ctypes.POINTER(LayerWeights), _P, _P,
@@ -246,6 +250,19 @@ def moe_permute_mxfp8(cfg, x, slot_of_pair, offsets, x_perm, rows_bound, codes, 
           rows_bound, ptr(codes), ptr(scales), stream_handle(stream))
 
 
+def moe_dispatch_mxfp8(cfg, x, pair_of_slot, offsets, rows_bound, x_perm, codes_r, scales_r, codes_c, scales_c,
+                       stream=None):
+    _call("moe_dispatch_mxfp8", ctypes.byref(cfg), ptr(x), ptr(pair_of_slot), ptr(offsets), rows_bound,
+          ptr(x_perm), ptr(codes_r), ptr(scales_r), ptr(codes_c), ptr(scales_c), stream_handle(stream))
+
+
+def moe_combine_bwd_mxfp8(cfg, dy, y_perm, pair_of_slot, offsets, topk_gate, rows_bound, dy_perm, dgate, codes_r,
+                          scales_r, codes_c, scales_c, stream=None):
+    _call("moe_combine_bwd_mxfp8", ctypes.byref(cfg), ptr(dy), ptr(y_perm), ptr(pair_of_slot), ptr(offsets),
+          ptr(topk_gate), rows_bound, ptr(dy_perm), ptr(dgate), ptr(codes_r), ptr(scales_r), ptr(codes_c),
+          ptr(scales_c), stream_handle(stream))
+
+
 def moe_mx_quantize_cols(src, rows, cols, offsets, E, rows_bound, codes, scales, stream=None):
     _call("moe_mx_quantize_cols", ptr(src), rows, cols, ptr(offsets), E, rows_bound, ptr(codes),
           ptr(scales), stream_handle(stream))
@@ -297,30 +314,33 @@ def alloc_workspace(cfg, device="cuda"):
 def alloc_saved(cfg, device="cuda", logits=True, shared=False, recompute=False, mx_saved=True) -> dict:
     """Forward buffers.  shared: room for a shared expert's activations; recompute: keep no
     [h | u] (the backward recomputes them), which leaves hu (and shared_hu) None; mx_saved
-    (MXFP8 only): keep the weights' MXFP8 copies from the forward for the backward."""
+    (MXFP8 only): keep the MXFP8 copies of the weights and the routed rows from the forward
+    for the backward, which leaves x_perm None (the rows move in MXFP8 only)."""
     import torch
     dt = torch_dtype(cfg)
     T, d, E, k, f, P = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.T * cfg.k
     i32 = dict(dtype=torch.int32, device=device)
     keep_hu = not recompute
+    fp8_rows = mx_saved and cfg.prec == MOE_PREC_MXFP8
     return dict(
         logits=torch.empty(T, E, dtype=torch.float32, device=device) if logits else None,
         topk_idx=torch.empty(T, k, **i32),
         topk_gate=torch.empty(T, k, dtype=torch.float32, device=device),
         counts=torch.empty(E, **i32), offsets=torch.empty(E + 1, **i32),
         slot_of_pair=torch.empty(P, **i32), pair_of_slot=torch.empty(P, **i32),
-        x_perm=torch.empty(P, d, dtype=dt, device=device),
+        x_perm=None if fp8_rows else torch.empty(P, d, dtype=dt, device=device),
         hu=torch.empty(P, 2 * f, dtype=dt, device=device) if keep_hu else None,
         a=torch.empty(P, f, dtype=dt, device=device),
         y_perm=torch.empty(P, d, dtype=dt, device=device),
         shared_hu=torch.empty(T, 2 * f, dtype=dt, device=device) if shared and keep_hu else None,
         shared_a=torch.empty(T, f, dtype=dt, device=device) if shared else None,
-        mx_saved=(torch.empty(moe_mx_saved_bytes(cfg), dtype=torch.uint8, device=device)
-                  if mx_saved and cfg.prec == MOE_PREC_MXFP8 else None),
+        mx_saved=torch.empty(moe_mx_saved_bytes(cfg), dtype=torch.uint8, device=device) if fp8_rows else None,
     )
 
 
 def alloc_grads(cfg, device="cuda", router=True, shared=False) -> dict:
+    """Backward buffers.  MXFP8 leaves dy_perm None (the combine's backward writes it in
+    MXFP8 only, into the workspace)."""
     import torch
     dt = torch_dtype(cfg)
     T, d, E, k, f, P = cfg.T, cfg.d, cfg.E, cfg.k, cfg.f, cfg.T * cfg.k
@@ -330,7 +350,7 @@ def alloc_grads(cfg, device="cuda", router=True, shared=False) -> dict:
         dw_gate=torch.empty(E, d, f, dtype=dt, device=device),
         dw_up=torch.empty(E, d, f, dtype=dt, device=device),
         dw_down=torch.empty(E, f, d, dtype=dt, device=device),
-        dy_perm=torch.empty(P, d, dtype=dt, device=device),
+        dy_perm=None if cfg.prec == MOE_PREC_MXFP8 else torch.empty(P, d, dtype=dt, device=device),
         dgate=torch.empty(T, k, dtype=torch.float32, device=device),
         dhu=torch.empty(P, 2 * f, dtype=dt, device=device),
         dx_perm=torch.empty(P, d, dtype=dt, device=device),

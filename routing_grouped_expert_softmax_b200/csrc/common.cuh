@@ -110,12 +110,12 @@ inline WsLayout ws_layout(const Shape &s) {
 }
 
 // Layout of moe_layer_saved.mx_saved: the routed experts' weights in MXFP8 in the four
-// orientations the grouped GEMMs read, and the layer input x_perm and the activation a in
-// MXFP8 down the expert-padded token axis (the weight-gradient GEMMs' operands), each as
-// codes then scales in the GEMMs' tile layout.
+// orientations the grouped GEMMs read, the permuted layer input in MXFP8 along d and down the
+// expert-padded token axis, and the activation a down the token axis (the weight-gradient
+// GEMMs' operands), each as codes then scales in the GEMMs' tile layout.
 struct MxSavedLayout {
   size_t wgu_c, wd_c, wd_r, wgu_r;   // as the workspace's regions of the same names
-  size_t xq_t, aq_t;                 // [Ppad][d], [Ppad][f]
+  size_t xq_r, xq_t, aq_t;           // [Ppad][d] along d, [Ppad][d] and [Ppad][f] along tokens
   size_t total;
 };
 inline MxSavedLayout mx_saved_layout(const Shape &s) {
@@ -127,6 +127,7 @@ inline MxSavedLayout mx_saved_layout(const Shape &s) {
   L.wd_c = off;  off += mx_bytes_t(ef, s.d);
   L.wd_r = off;  off += mx_bytes_r(ef, s.d);
   L.wgu_r = off; off += mx_bytes_r(ed, 2 * s.f);
+  L.xq_r = off;  off += mx_bytes_r(R, s.d);
   L.xq_t = off;  off += mx_bytes_t(R, s.d);
   L.aq_t = off;  off += mx_bytes_t(R, s.f);
   L.total = off;
@@ -204,15 +205,18 @@ cudaError_t launch_mx_permute(const void *x, const int32_t *sop, const int32_t *
 // The combine's backward for the MXFP8 layer (bf16 storage, d % 128 == 0): dy_perm, dgate as
 // launch_combine_bwd, and dy_perm in MXFP8 along d (codes_r) and down the expert-padded token
 // axis (codes_c), scales in the GEMMs' tile layout; pos = pair_of_slot; rows_bound = Ppad.
+// dy_perm may be null (the bf16 rows are not written); tiled: scales in the GEMMs' tile layout,
+// else plain ([rows][d/32] along d, [rows/32][d] down the token axis).
 cudaError_t launch_mx_combine_bwd(const void *dy, const void *y_perm, const int32_t *pos, const int32_t *offsets,
                                   const float *gate, int E, int k, int d, int64_t rows_bound, void *dy_perm,
                                   float *dgate, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
-                                  uint8_t *scales_c, cudaStream_t st);
+                                  uint8_t *scales_c, cudaStream_t st, bool tiled = true);
 // FP8 dispatch, slot-major: x_perm (a bit copy of each routed row) and x_perm in MXFP8 along d
 // (codes_r) and down the expert-padded token axis (codes_c), scales in the GEMMs' tile layout.
+// x_perm may be null (the bf16 rows are not written); tiled as for launch_mx_combine_bwd.
 cudaError_t launch_mx_dispatch(const void *x, const int32_t *pos, const int32_t *offsets, int E, int k, int d,
                                int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r,
-                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st);
+                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st, bool tiled = true);
 cudaError_t launch_combine_bwd(const Shape &s, const void *dy, const void *y_perm,
                                const int32_t *sop, const float *gate, void *dy_perm,
                                float *dgate, cudaStream_t st);
@@ -221,17 +225,23 @@ cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int3
                                  const float *dgate, const float *gate, const int32_t *idx,
                                  const void *w_rt, bool accumulate, void *dx, cudaStream_t st);
 cudaError_t launch_router_transpose(const Shape &s, const void *w_r, void *w_rt, cudaStream_t st);
-// dW_r from the expert-contiguous rows x_perm and the slot maps (layer backward)
+// Multiprocessors of the current device (cached per device; 148 if the query fails).
+int device_sm_count();
+
+// dW_r from the expert-contiguous rows x_perm and the slot maps (layer backward); x != nullptr:
+// the rows are read from the layer input instead, x[pos[slot] / k] (no x_perm kept)
 cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, const int32_t *pos,
                                         const int32_t *offsets, const float *dgate, const float *gate,
-                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st);
+                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st,
+                                        const void *x = nullptr);
 cudaError_t launch_router_wgrad(const Shape &s, const float *dgate, const float *gate,
                                 const int32_t *idx, const void *x, float *partial,
                                 float *dw_r, cudaStream_t st);
 // bf16 weight gradients: tails[e*64 + i] = src[offsets[e] + 64*(count_e/64) + i] for
 // i < count_e % 64 and zeros for the rest of the expert's 64 rows (src [P][C] bf16); experts
 // whose count is a multiple of 64 are left alone (they have no partial K-block).
-cudaError_t launch_wgrad_tails(const void *src, int C, const int32_t *offsets, int E, void *tails, cudaStream_t st);
+cudaError_t launch_wgrad_tails(const void *src_a, int C_a, void *tails_a, const void *src_b, int C_b, void *tails_b,
+                               const int32_t *offsets, int E, cudaStream_t st);
 // MXFP8 only:
 //   x_quantized: the workspace already holds x_perm's MXFP8 rows, written by
 //     launch_mx_permute into the layout ws_layout(s) gives them;

@@ -28,7 +28,10 @@
 // Weight-gradient GEMMs reduce over one expert's rows; the expert's last, partial K-block is
 // read from a per-expert tail buffer that holds its rows and zeros after them (bf16; the
 // MXFP8 operands are padded to 128 rows per expert instead), so every stage is an ordinary
-// load.
+// load.  bf16 weight gradients deal whole strips (one expert's M block: all N tiles that
+// share the A operand) to the CTAs (pairs) and keep A's K-blocks resident in shared memory
+// across the strip, so that only B streams through the ring (A stationary); an expert whose
+// K-blocks outnumber the A slots streams A with B instead.
 // CTA pairs (cta_group::2): a 256-row tile whose MMAs the even CTA issues for both.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -132,6 +135,10 @@ struct Params {
   // blocks of 32 down the rows (nk_col = K groups of the padded token axis)
   uint8_t *q_row_codes, *q_row_scales, *q_col_codes, *q_col_scales;
   int nk_row, nk_col;
+  // bf16 weight gradients (A stationary): na of the ring's slots hold A, the rest are B's
+  // ring; strips: tiles are dealt in whole strips that keep A resident (else tile by tile,
+  // A streaming with B)
+  int na, strips;
   int *err;
   int *where;  // [3]: first failed wait per role, ((tile+1) << 12) | (kb << 2) | site
   // Failure-detection test hook, 0 in normal use: the MMA issuer of a single-CTA launch first
@@ -158,6 +165,8 @@ struct Tile {
 struct Ctrl {
   uint64_t full[8];
   uint64_t empty[8];
+  uint64_t afull[8];      // A-stationary weight gradients: one pair of barriers per A slot
+  uint64_t aempty[8];
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t drain;
@@ -237,6 +246,20 @@ __device__ __forceinline__ bool get_tile(int t, const Params &p, const Ctrl &c, 
     tl.num_kb = p.K / KBLK;
   }
   return true;
+}
+
+// The i-th tile of this CTA (pair), or -1 past the last.  strips: strip s = tile0 + j*tstep
+// holds tiles s*nt .. s*nt + nt-1 (nt = N/BN, the tiles that share one A block).
+template <int BN>
+__device__ __forceinline__ int nth_tile(int i, const Params &p, int tile0, int tstep, int ntiles, bool strips) {
+  int t;
+  if (strips) {
+    const int nt = p.N / BN;
+    t = (tile0 + (i / nt) * tstep) * nt + i % nt;
+  } else {
+    t = tile0 + i * tstep;
+  }
+  return t < ntiles ? t : -1;
 }
 
 template <int MODE, int BN, int CG = 1>
@@ -342,6 +365,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // tf32 operands are only ever K-major: the fp32 forward reads pre-transposed weights
   constexpr bool FWD_B_KMAJOR = (sizeof(T) == 4) && (MODE == FWD_GU || MODE == FWD_DOWN);
   constexpr bool B_MN = MT::B_MN && !FWD_B_KMAJOR;
+  // A stationary (bf16 weight gradients): the ring memory holds NA A slots and then SB B
+  // slots instead of STAGES (A | B) stages.  CTA pairs hold 128 rows of A and 128 columns of
+  // B per CTA, slots of the same size, so the split is the host's choice (p.na); single CTAs
+  // keep STAGES of each.
+  constexpr bool ASTAT = MT::WGRAD && !C::MX;
+  const int NA = ASTAT ? (C::A_BYTES == C::B_BYTES ? p.na : C::STAGES) : 0;
+  const int SB = ASTAT ? (C::A_BYTES == C::B_BYTES ? 2 * C::STAGES - NA : C::STAGES) : C::STAGES;
+  const bool strips = ASTAT && p.strips;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ring = smem;                                   // STAGES x (A | B)
@@ -359,10 +390,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   // ------------------------------------------------------------------ prologue
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < 8; ++s) {
       // one arrival: the producer's arrive.expect_tx (pairs: the leader's, for both CTAs' bytes)
       ptx::mbar_init(ptx::smem_u32(&c.full[s]), 1);
       ptx::mbar_init(ptx::smem_u32(&c.empty[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&c.afull[s]), 1);
+      ptx::mbar_init(ptx::smem_u32(&c.aempty[s]), 1);
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(ptx::smem_u32(&c.tfull[a]), 1);
@@ -451,20 +484,53 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int stage = 0;
     uint32_t phase = 0;
     uint32_t armed = 0, armed_par = 0;  // per stage: a fill is in flight / its parity
+    uint32_t aph = 0, a_armed = 0, a_armed_par = 0;   // A slots: fill parity, in flight, its parity
     bool ok = true;
-    for (int t = tile0; t < ntiles && ok; t += tstep) {
+    for (int i = 0; ok; ++i) {
+      const int t = nth_tile<BN>(i, p, tile0, tstep, ntiles, strips);
+      if (t < 0) break;
       Tile tl;
       get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
+      // A stationary: the strip's first tile loads A (the K-blocks stay in their slots for
+      // the strip's other tiles), unless there are more K-blocks than slots
+      const bool a_res = strips && tl.num_kb <= NA;
+      const bool load_a = ASTAT && (!a_res || i % (p.N / BN) == 0);
       for (int kb = 0; kb < tl.num_kb && ok; ++kb) {
-        if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 0); break; }
-        const uint32_t a_dst = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
-        const uint32_t b_dst = a_dst + C::A_BYTES;
         // bf16 weight gradients: the expert's last K-block, when partial, comes from the tail
         // buffers (rows e*64 + i: the block's rows, then zeros)
         bool tail = false;
         if constexpr (MT::WGRAD && !C::MX) tail = tl.rows - kb * C::KBLK < C::KBLK;
+        if constexpr (ASTAT) {
+          if (load_a) {
+            const int as = a_res ? kb : kb % NA;
+            if (lane == 0)
+              ok = ptx::mbar_wait(ptx::smem_u32(&c.aempty[as]), ((aph >> as) & 1u) ^ 1u, abort_flag, WAIT_LIMIT_NS);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 1); break; }
+            if (lane == 0) {
+              const uint32_t abar = ptx::smem_u32(&c.afull[as]);
+              const uint32_t abar_leader = CG == 2 ? ptx::mapa(abar, 0) : abar;
+              const uint32_t a_dst = ptx::smem_u32(ring + as * C::A_BYTES);
+              if (rank == 0) ptx::mbar_arrive_expect_tx(abar, CG * C::A_BYTES);
+#pragma unroll
+              for (int j = 0; j < BM / C::BOX_MN; ++j) {
+                const CUtensorMap *tm = tail ? &tmAT : &tmA;
+                const int y = tail ? tl.e * C::KBLK : tl.row0 + kb * C::KBLK;
+                if (CG == 2) ptx::tma_load_2d_pair(a_dst + j * C::BOX_BYTES, tm, abar_leader, tl.mcol0 + j * C::BOX_MN, y);
+                else ptx::tma_load_2d(a_dst + j * C::BOX_BYTES, tm, abar, tl.mcol0 + j * C::BOX_MN, y);
+              }
+            }
+            a_armed |= 1u << as;
+            if ((aph >> as) & 1u) a_armed_par |= 1u << as; else a_armed_par &= ~(1u << as);
+            aph ^= 1u << as;
+          }
+        }
+        if (lane == 0) ok = ptx::mbar_wait(ptx::smem_u32(&c.empty[stage]), phase ^ 1, abort_flag, WAIT_LIMIT_NS);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { if (lane == 0) note_fail(p, 0, t, kb, 0); break; }
+        const uint32_t a_dst = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
+        const uint32_t b_dst = ASTAT ? ptx::smem_u32(ring + NA * C::A_BYTES + stage * C::B_BYTES) : a_dst + C::A_BYTES;
+        if (ASTAT) (void)a_dst;
         const uint32_t full_local = ptx::smem_u32(&c.full[stage]);
         // pairs: the bytes of both CTAs' loads are counted on the leader's full barrier
         const uint32_t full_leader = CG == 2 ? ptx::mapa(full_local, 0) : full_local;
@@ -474,7 +540,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           else ptx::tma_load_2d(dst, tm, bar, x, y);
         };
         if (lane == 0) {
-          if (rank == 0) ptx::mbar_arrive_expect_tx(bar, CG * C::STAGE_BYTES + C::SF_BYTES);
+          if (rank == 0) ptx::mbar_arrive_expect_tx(bar, ASTAT ? CG * C::B_BYTES : CG * C::STAGE_BYTES + C::SF_BYTES);
           if constexpr (C::MX) {
             // the stage's scale-factor tiles, A then B (512 bytes each), straight into the
             // arrangement the MMA issuer's tcgen05.cp reads
@@ -494,8 +560,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::bulk_load(sf_dst, p.sfa + (a_mn * p.nka + a_kg) * 512, 512, full_local);
             ptx::bulk_load(sf_dst + 512, p.sfb + (b_mn * p.nkb + b_kg) * 512, 512, full_local);
           }
-          // ---- A
-          if constexpr (MT::A_MN) {
+          // ---- A (A stationary: loaded above, into its own slot)
+          if constexpr (ASTAT) {
+          } else if constexpr (MT::A_MN) {
 #pragma unroll
             for (int i = 0; i < BM / C::BOX_MN; ++i) {
               if (tail) ld(a_dst + i * C::BOX_BYTES, &tmAT, tl.mcol0 + i * C::BOX_MN, tl.e * C::KBLK);
@@ -565,7 +632,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // this stage's full barrier completes (or has completed) the phase of this pass
         armed |= 1u << stage;
         if (phase) armed_par |= 1u << stage; else armed_par &= ~(1u << stage);
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+        if (++stage == SB) { stage = 0; phase ^= 1; }
       }
     }
     // Drain: every TMA fill this warp issued must land before the CTA may exit, also after
@@ -574,10 +641,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // before the stage was refilled.  (Pairs: the leader's full barriers count the peer's
     // bytes too.)
     if (lane == 0) {
-      for (int s = 0; s < C::STAGES; ++s)
+      for (int s = 0; s < 8; ++s) {
         if (rank == 0 && ((armed >> s) & 1u))
           if (!ptx::mbar_wait(ptx::smem_u32(&c.full[s]), (armed_par >> s) & 1u, nullptr, WAIT_LIMIT_NS))
             note_fail(p, 0, 0, s, 2);
+        if (rank == 0 && ((a_armed >> s) & 1u))
+          if (!ptx::mbar_wait(ptx::smem_u32(&c.afull[s]), (a_armed_par >> s) & 1u, nullptr, WAIT_LIMIT_NS))
+            note_fail(p, 0, 0, s, 2);
+      }
     }
   } else if (warp == 1) {
     // ================================================================ MMA issuer
@@ -598,11 +669,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ok = ptx::mbar_wait(ptx::smem_u32(&c.never), 0, abort_flag, p.stall_ns);
         if (!ok) note_fail(p, 1, 0, 0, 3);
       }
-      for (int t = tile0; t < ntiles && ok; t += tstep, ++it) {
+      uint32_t a_ph = 0;   // A stationary: per A slot, the parity of its next fill
+      for (;; ++it) {
+        const int t = nth_tile<BN>(it, p, tile0, tstep, ntiles, strips);
+        if (t < 0 || !ok) break;
         Tile tl;
         get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
         const int acc = it & 1;
         const uint32_t aph = (it >> 1) & 1;
+        // A stationary: the strip's first tile waits for A, its last releases A's slots (every
+        // tile, when A streams)
+        const int nt_strip = ASTAT ? p.N / BN : 1;
+        const bool a_res = strips && tl.num_kb <= NA;
+        const bool wait_a = ASTAT && (!a_res || it % nt_strip == 0);
+        const bool release_a = ASTAT && (!a_res || it % nt_strip == nt_strip - 1);
         ok = ptx::mbar_wait(ptx::smem_u32(&c.tempty[acc]), aph ^ 1, abort_flag, WAIT_LIMIT_NS);
         if (!ok) { note_fail(p, 1, t, 0, 0); break; }
         ptx::tc_fence_after();
@@ -613,12 +693,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         for (int kb = 0; kb < tl.num_kb; ++kb) {
+          int as = 0;
+          if constexpr (ASTAT) {
+            as = a_res ? kb : kb % NA;
+            if (wait_a) {
+              ok = ptx::mbar_wait(ptx::smem_u32(&c.afull[as]), (a_ph >> as) & 1u, abort_flag, WAIT_LIMIT_NS);
+              if (!ok) { note_fail(p, 1, t, kb, 1); break; }
+              a_ph ^= 1u << as;
+            }
+          }
           // loaded bytes and commit arrivals are ordered by the barrier itself
           ok = ptx::mbar_wait(ptx::smem_u32(&c.full[stage]), phase, abort_flag, WAIT_LIMIT_NS);
           if (!ok) { note_fail(p, 1, t, kb, 1); break; }
           ptx::tc_fence_after();
-          const uint32_t a_addr = ptx::smem_u32(ring + stage * C::STAGE_BYTES);
-          const uint32_t b_addr = a_addr + C::A_BYTES;
+          const uint32_t a_addr = ASTAT ? ptx::smem_u32(ring + as * C::A_BYTES)
+                                        : ptx::smem_u32(ring + stage * C::STAGE_BYTES);
+          const uint32_t b_addr = ASTAT ? ptx::smem_u32(ring + NA * C::A_BYTES + stage * C::B_BYTES)
+                                        : a_addr + C::A_BYTES;
           uint32_t sfa_t = 0, sfb_t = 0;
           if constexpr (C::MX) {
             // scales of this stage into TMEM columns 2*BN (A) and 2*BN + 4 (B)
@@ -655,7 +746,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.empty[stage]), 0x3);
           else ptx::tc_commit(ptx::smem_u32(&c.empty[stage]));
-          if (++stage == C::STAGES) { stage = 0; phase ^= 1; }
+          if (ASTAT && release_a) {
+            if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.aempty[as]), 0x3);
+            else ptx::tc_commit(ptx::smem_u32(&c.aempty[as]));
+          }
+          if (++stage == SB) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
         if constexpr (CG == 2) ptx::tc_commit_pair_mc(ptx::smem_u32(&c.tfull[acc]), 0x3);
@@ -676,8 +771,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - 2) >> 2;     // 0 or 1
     const int r = q * 32 + lane;          // tile row owned by this thread
     uint8_t *epi_box = extra + (warp - 2) * EPI_BOX_BYTES;       // weight gradients
-    int it = 0;
-    for (int t = tile0; t < ntiles; t += tstep, ++it) {
+    for (int it = 0;; ++it) {
+      const int t = nth_tile<BN>(it, p, tile0, tstep, ntiles, strips);
+      if (t < 0) break;
       Tile tl;
       get_tile<MODE, BN, C::KBLK, C::MX, CG>(t, p, c, offs_s, tl, rank);
       const int acc = it & 1;
@@ -978,15 +1074,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {  // weight gradients: rows q*32.. of the [M x N] block of expert e
-        // Each 32 x 64 piece goes through the warp's staging box in the layout of a
-        // 128-byte-swizzled TMA box (16-byte chunk j of row r at chunk j ^ (r % 8)); one lane
-        // then stores the box with TMA.  The box is refilled only once the store that last
+        // The warp's 32 x 128 part of the accumulator is read and rounded to bf16 first and
+        // the accumulator released, so that the MMAs of the tile after next need not wait for
+        // the stores.  Each 32 x 64 piece then goes through the warp's staging box in the
+        // layout of a 128-byte-swizzled TMA box (16-byte chunk j of row r at chunk j ^ (r % 8));
+        // one lane stores the box with TMA.  The box is refilled only once the store that last
         // used it has read it.
         static_assert(sizeof(OutT) == 2, "weight gradients are stored as bf16");
-        const int orow = tl.e * p.M + tl.mcol0 + q * 32;
-#pragma unroll 1
-        for (int cc = half * (BN / 2); cc < (half + 1) * (BN / 2); cc += 64) {
+        constexpr int PIECES = BN / 2 / 64;
+        uint4 pk[PIECES][8];
+#pragma unroll
+        for (int pc = 0; pc < PIECES; ++pc) {
           float v0[32], v1[32];
+          const int cc = half * (BN / 2) + pc * 64;
           if (tl.num_kb > 0) {
             ptx::tmem_ld32(taddr + cc, v0);
             ptx::tmem_ld32(taddr + cc + 32, v1);
@@ -994,14 +1094,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
             for (int i = 0; i < 32; ++i) { v0[i] = 0.f; v1[i] = 0.f; }
           }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) pk[pc][j] = Vec<OutT>::store(j < 4 ? &v0[8 * j] : &v1[8 * (j - 4)]);
+        }
+        // release the accumulator: one arrival per warp on the leader's barrier
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&c.tempty[acc]), 0));
+          else ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+        }
+        const int orow = tl.e * p.M + tl.mcol0 + q * 32;
+#pragma unroll
+        for (int pc = 0; pc < PIECES; ++pc) {
+          const int cc = half * (BN / 2) + pc * 64;
           uint8_t *box = epi_box;
           if (lane == 0) ptx::bulk_wait_read<0>();
           __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 w = Vec<OutT>::store(j < 4 ? &v0[8 * j] : &v1[8 * (j - 4)]);
-            *reinterpret_cast<uint4 *>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = w;
-          }
+          for (int j = 0; j < 8; ++j)
+            *reinterpret_cast<uint4 *>(box + lane * 128 + ((j ^ (lane & 7)) << 4)) = pk[pc][j];
           ptx::fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -1017,12 +1129,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      // release the accumulator: one arrival per warp on the leader's barrier
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (CG == 2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&c.tempty[acc]), 0));
-        else ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+      if constexpr (!MT::WGRAD) {
+        // release the accumulator: one arrival per warp on the leader's barrier
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (CG == 2 && rank != 0) ptx::mbar_arrive_cluster(ptx::mapa(ptx::smem_u32(&c.tempty[acc]), 0));
+          else ptx::mbar_arrive(ptx::smem_u32(&c.tempty[acc]));
+        }
       }
     }
     // weight gradients: the staging boxes stay in use until their TMA stores complete
@@ -1084,9 +1198,11 @@ static bool make_tmap(CUtensorMap *m, const void *ptr, int es, uint64_t cols, ui
   return r == CUDA_SUCCESS;
 }
 
-static int sm_count() {
-  static std::atomic<int> cache[MAX_DEVICES];
-  const int dev = device_ordinal();
+}  // namespace gg
+
+int device_sm_count() {
+  static std::atomic<int> cache[gg::MAX_DEVICES];
+  const int dev = gg::device_ordinal();
   if (dev >= 0) {
     const int n = cache[dev].load(std::memory_order_relaxed);
     if (n > 0) return n;
@@ -1097,6 +1213,9 @@ static int sm_count() {
   if (dev >= 0) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
+
+namespace gg {
+static int sm_count() { return device_sm_count(); }
 
 // Failure-detection test hook (moe_debug_set_gemm_stall_ns), 0 in normal use: process-wide,
 // read at each launch, applied to single-CTA launches only.
@@ -1119,6 +1238,23 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   if (ModeTraits<MODE>::WGRAD && !C::MX && (!at || !bt)) return MOE_ERR_INVALID_ARG;
   const CUtensorMap &out0 = o0 ? *o0 : a, &out1 = o1 ? *o1 : a;
   const CUtensorMap &atail = at ? *at : a, &btail = bt ? *bt : a;
+  // bf16 weight gradients: A slots for 1.5x the average expert's K-blocks (4..8 of the 12
+  // slots of a pair's ring), and whole strips per CTA (pair) when the average expert's A fits
+  // and there are at least two strips per CTA (pair) to balance the load; otherwise A streams
+  // tile by tile through half of the slots
+  auto set_astat = [&](int64_t units) {
+    if constexpr (ModeTraits<MODE>::WGRAD && !C::MX) {
+      const int64_t avg_rows = p.E > 0 ? (int64_t)p.P / p.E : 0;
+      const int64_t avg_kb = (avg_rows + C::KBLK - 1) / C::KBLK;
+      if constexpr (C::A_BYTES == C::B_BYTES)
+        p.na = (int)std::min<int64_t>(std::max<int64_t>((3 * avg_rows + 2 * C::KBLK - 1) / (2 * C::KBLK), 4), 8);
+      else
+        p.na = C::STAGES;
+      const int64_t nstrips = (int64_t)p.E * (p.M / C::BMP);
+      p.strips = avg_kb <= p.na && nstrips >= 2 * units;
+      if (!p.strips) p.na = C::STAGES;   // A streams with B: as many slots of each
+    }
+  };
   // the shared-memory opt-in is a per-device property of the kernel: set once per device
   // (two threads racing here both set it, which is harmless)
   static std::atomic<bool> attr_set[MAX_DEVICES];
@@ -1130,6 +1266,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
   }
   if constexpr (CG == 1) {
     const int64_t units = std::min<int64_t>(sm_count(), std::max<int64_t>(max_tiles, 1));
+    set_astat(units);
     kern<<<(unsigned)units, NUM_THREADS, SMEM, st>>>(a, b0, b1, out0, out1, atail, btail, p);
   } else {
     cudaLaunchConfig_t cfg = {};
@@ -1156,6 +1293,7 @@ static int launch(const CUtensorMap &a, const CUtensorMap &b0, const CUtensorMap
       if (dev >= 0) pairs_cache[dev].store(max_pairs, std::memory_order_relaxed);
     }
     const int64_t units = std::min<int64_t>(max_pairs, std::max<int64_t>(max_tiles, 1));
+    set_astat(units);
     cfg.gridDim = dim3((unsigned)(units * CG));
     if (cudaLaunchKernelEx(&cfg, kern, a, b0, b1, out0, out1, atail, btail, p) != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -1276,8 +1414,7 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   // (2) dWd[e] = a^T [f, rows_e] x dy_perm [rows_e, d]
   {
     // every expert's last partial K-block of a and dy_perm, zero past the expert's rows
-    if (launch_wgrad_tails(a, s.f, offsets, s.E, tail_a, st) || launch_wgrad_tails(dy_perm, s.d, offsets, s.E, tail_b, st))
-      return MOE_ERR_CUDA;
+    if (launch_wgrad_tails(a, s.f, tail_a, dy_perm, s.d, tail_b, offsets, s.E, st)) return MOE_ERR_CUDA;
     if (!make_tmap(&tAT, tail_a, ES, s.f, tail_rows, BOX_MN, KBLK) ||
         !make_tmap(&tBT, tail_b, ES, s.d, tail_rows, BOX_MN, KBLK))
       return MOE_ERR_CUDA;
@@ -1322,9 +1459,7 @@ static int bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, con
   }
   // (4) [dWg | dWu][e] = x_perm^T [d, rows_e] x dhu [rows_e, 2f]
   {
-    if (launch_wgrad_tails(x_perm, s.d, offsets, s.E, tail_a, st) ||
-        launch_wgrad_tails(dhu, 2 * s.f, offsets, s.E, tail_b, st))
-      return MOE_ERR_CUDA;
+    if (launch_wgrad_tails(x_perm, s.d, tail_a, dhu, 2 * s.f, tail_b, offsets, s.E, st)) return MOE_ERR_CUDA;
     if (!make_tmap(&tAT, tail_a, ES, s.d, tail_rows, BOX_MN, KBLK) ||
         !make_tmap(&tBT, tail_b, ES, 2 * s.f, tail_rows, BOX_MN, KBLK))
       return MOE_ERR_CUDA;
@@ -1384,8 +1519,10 @@ static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offset
                        cudaStream_t st, bool x_quantized, uint8_t *wsaved, bool wfill) {
   const WsLayout L = ws_layout(s);
   const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
-  const MxOp xq = mx_r(ws, L.xq_r, R, s.d), aq = mx_r(ws, L.aq_r, R, s.f);
-  // x_quantized: the FP8 dispatch (launch_mx_permute) already wrote xq's rows
+  // x_perm's rows in MXFP8: in the caller's saved copies when given, else in the workspace
+  const MxOp xq = wsaved ? mx_r(wsaved, mx_saved_layout(s).xq_r, R, s.d) : mx_r(ws, L.xq_r, R, s.d);
+  const MxOp aq = mx_r(ws, L.aq_r, R, s.f);
+  // x_quantized: the FP8 dispatch already wrote xq's rows
   if (!x_quantized && launch_mx_quant_rows(x_perm, P, s.d, offsets, s.E, R, xq.codes, xq.scales, st, true))
     return MOE_ERR_CUDA;
   MxOp wgu, wd;

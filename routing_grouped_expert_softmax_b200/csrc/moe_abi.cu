@@ -184,6 +184,38 @@ int moe_permute_mxfp8(const moe_config *cfg, const void *x, const int32_t *slot_
   return cuda_rc(launch_mx_permute(x, slot_of_pair, offsets, s.E, s.T, s.k, s.d, x_perm, codes, scales, S(stream)));
 }
 
+int moe_dispatch_mxfp8(const moe_config *cfg, const void *x, const int32_t *pair_of_slot, const int32_t *offsets,
+                       int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
+                       uint8_t *scales_c, moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  const Shape s = shape_of(cfg);
+  if (rows_bound < s.Ppad()) return MOE_ERR_INVALID_ARG;
+  RETURN_IF(check_ptrs({x, codes_r, codes_c}));
+  RETURN_IF(check_ptrs_or_null({x_perm}));
+  RETURN_IF(check_ptrs4({pair_of_slot, offsets, scales_r, scales_c}));
+  return cuda_rc(launch_mx_dispatch(x, pair_of_slot, offsets, s.E, s.k, s.d, rows_bound, x_perm, codes_r, scales_r,
+                                    codes_c, scales_c, S(stream), /*tiled=*/false));
+}
+
+int moe_combine_bwd_mxfp8(const moe_config *cfg, const void *dy, const void *y_perm, const int32_t *pair_of_slot,
+                          const int32_t *offsets, const float *topk_gate, int64_t rows_bound, void *dy_perm,
+                          float *dgate, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c, uint8_t *scales_c,
+                          moe_stream_t stream) {
+  RETURN_IF(check_cfg(cfg));
+  if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+  if (cfg->T == 0) return MOE_OK;
+  const Shape s = shape_of(cfg);
+  if (rows_bound < s.Ppad()) return MOE_ERR_INVALID_ARG;
+  RETURN_IF(check_ptrs({dy, y_perm, codes_r, codes_c}));
+  RETURN_IF(check_ptrs_or_null({dy_perm}));
+  RETURN_IF(check_ptrs4({pair_of_slot, offsets, topk_gate, dgate, scales_r, scales_c}));
+  return cuda_rc(launch_mx_combine_bwd(dy, y_perm, pair_of_slot, offsets, topk_gate, s.E, s.k, s.d, rows_bound,
+                                       dy_perm, dgate, codes_r, scales_r, codes_c, scales_c, S(stream),
+                                       /*tiled=*/false));
+}
+
 int moe_mx_quantize_cols(const void *src, int64_t rows, int32_t cols, const int32_t *offsets, int32_t E,
                          int64_t rows_bound, uint8_t *codes, uint8_t *scales, moe_stream_t stream) {
   if (rows < 0 || cols <= 0 || cols % 32 || (offsets && (E <= 0 || E > MAX_E))) return MOE_ERR_INVALID_ARG;
@@ -271,9 +303,13 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   RETURN_IF(check_ptrs4({sv->counts, sv->offsets}));
   if (route) RETURN_IF(check_ptrs4({w->w_router}));
   if (shared) RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down}));
-  if (s.prec == MOE_PREC_MXFP8) RETURN_IF(check_ptrs_or_null({sv->mx_saved}));
+  const bool mx = s.prec == MOE_PREC_MXFP8;
+  if (mx) RETURN_IF(check_ptrs_or_null({sv->mx_saved}));
+  // MXFP8 with the saved copies: the routed rows move as E4M3 only and x_perm is unused
+  const bool rows_fp8 = mx && sv->mx_saved;
   if (cfg->T > 0) {
-    RETURN_IF(check_ptrs({x, y, sv->x_perm, sv->a, sv->y_perm}));
+    RETURN_IF(check_ptrs({x, y, sv->a, sv->y_perm}));
+    RETURN_IF(rows_fp8 ? check_ptrs_or_null({sv->x_perm}) : check_ptrs({sv->x_perm}));
     RETURN_IF(check_ptrs_or_null({sv->hu}));
     RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, sv->pair_of_slot}));
     if (shared) {
@@ -291,18 +327,19 @@ static int layer_fwd_common(const moe_config *cfg, const moe_layer_weights *w, c
   RETURN_IF(cuda_rc(launch_build_offsets(s, sv->topk_idx, sv->counts, sv->offsets, sv->slot_of_pair,
                                          sv->pair_of_slot, bc, err, st)));
   if (cfg->T == 0) return MOE_OK;
-  const bool mx = s.prec == MOE_PREC_MXFP8;
   uint8_t *mxs = mx ? static_cast<uint8_t *>(sv->mx_saved) : nullptr;
   if (mx) {
-    // FP8 dispatch: the permute also writes x_perm's MXFP8 rows where the forward GEMM reads
-    // them, and, when the caller keeps the MXFP8 copies for the backward, its token-axis copy
-    uint8_t *xq = static_cast<uint8_t *>(ws) + L.xq_r;
     const int64_t R = s.Ppad();
     if (mxs) {
-      uint8_t *xqt = mxs + mx_saved_layout(s).xq_t;
-      RETURN_IF(cuda_rc(launch_mx_dispatch(x, sv->pair_of_slot, sv->offsets, s.E, s.k, s.d, R, sv->x_perm, xq,
-                                           xq + R * s.d, xqt, xqt + R * s.d, st)));
+      // FP8 dispatch: each routed row of x is read once and written only in MXFP8, along d
+      // for the forward GEMM and down the token axis for the backward's weight gradient
+      const MxSavedLayout M = mx_saved_layout(s);
+      uint8_t *xqr = mxs + M.xq_r, *xqt = mxs + M.xq_t;
+      RETURN_IF(cuda_rc(launch_mx_dispatch(x, sv->pair_of_slot, sv->offsets, s.E, s.k, s.d, R, nullptr, xqr,
+                                           xqr + R * s.d, xqt, xqt + R * s.d, st)));
     } else {
+      // the permute also writes x_perm's MXFP8 rows where the forward GEMM reads them
+      uint8_t *xq = static_cast<uint8_t *>(ws) + L.xq_r;
       RETURN_IF(cuda_rc(launch_mx_permute(x, sv->slot_of_pair, sv->offsets, s.E, s.T, s.k, s.d, sv->x_perm, xq,
                                           xq + R * s.d, st, /*tiled=*/true)));
     }
@@ -346,12 +383,17 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   RETURN_IF(check_ptrs4({sv->offsets}));
   if (router) RETURN_IF(check_ptrs4({w->w_router, g->dw_router}));
   if ((router || s.prec == MOE_PREC_MXFP8) && cfg->T > 0) RETURN_IF(check_ptrs4({sv->pair_of_slot}));
+  const bool mx = s.prec == MOE_PREC_MXFP8;
+  // MXFP8: dy_perm moves in MXFP8 only; with the saved copies x_perm is unused too
+  const bool rows_fp8 = mx && sv->mx_saved;
   if (shared)
     RETURN_IF(check_ptrs({w->w_shared_gate, w->w_shared_up, w->w_shared_down, g->dw_shared_gate,
                           g->dw_shared_up, g->dw_shared_down}));
   if (s.prec == MOE_PREC_MXFP8) RETURN_IF(check_ptrs_or_null({sv->mx_saved}));
   if (cfg->T > 0) {
-    RETURN_IF(check_ptrs({x, dy, g->dx, sv->x_perm, sv->a, sv->y_perm, g->dy_perm, g->dhu, g->dx_perm}));
+    RETURN_IF(check_ptrs({x, dy, g->dx, sv->a, sv->y_perm, g->dhu, g->dx_perm}));
+    RETURN_IF(rows_fp8 ? check_ptrs_or_null({sv->x_perm}) : check_ptrs({sv->x_perm}));
+    RETURN_IF(mx ? check_ptrs_or_null({g->dy_perm}) : check_ptrs({g->dy_perm}));
     RETURN_IF(check_ptrs_or_null({sv->hu}));
     RETURN_IF(check_ptrs4({sv->topk_idx, sv->topk_gate, sv->slot_of_pair, g->dgate}));
     if (shared) {
@@ -371,27 +413,27 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
     if (e == cudaSuccess && shared) e = cudaMemsetAsync(g->dw_shared_down, 0, sb, st);
     return cuda_rc(e);
   }
-  const bool mx = s.prec == MOE_PREC_MXFP8;
   if (mx) {
-    // FP8 dispatch of the backward: dy_perm's MXFP8 copies for both down-projection GEMMs come
-    // out of the combine's backward itself
+    // FP8 dispatch of the backward: dy_perm exists only as the MXFP8 copies both
+    // down-projection GEMMs read, written by the combine's backward itself
     const WsLayout L = ws_layout(s);
     uint8_t *w8 = static_cast<uint8_t *>(ws);
     const int64_t R = s.Ppad();
     uint8_t *dyq = w8 + L.dyq_r, *dyqt = w8 + L.dyq_t;
     RETURN_IF(cuda_rc(launch_mx_combine_bwd(dy, sv->y_perm, sv->pair_of_slot, sv->offsets, sv->topk_gate, s.E, s.k,
-                                            s.d, R, g->dy_perm, g->dgate, dyq, dyq + R * s.d, dyqt, dyqt + R * s.d,
+                                            s.d, R, nullptr, g->dgate, dyq, dyq + R * s.d, dyqt, dyqt + R * s.d,
                                             st)));
   } else {
     RETURN_IF(cuda_rc(launch_combine_bwd(s, dy, sv->y_perm, sv->slot_of_pair, sv->topk_gate, g->dy_perm,
                                          g->dgate, st)));
   }
   // recompute: [h | u] = x_perm [Wg | Wu] into dhu, where the SwiGLU backward then runs in place
-  uint8_t *mxs = s.prec == MOE_PREC_MXFP8 ? static_cast<uint8_t *>(sv->mx_saved) : nullptr;
+  uint8_t *mxs = mx ? static_cast<uint8_t *>(sv->mx_saved) : nullptr;
   const void *hu = sv->hu;
   if (!hu) {
+    // with the saved copies the forward's MXFP8 rows of x_perm are read again as they are
     RETURN_IF(launch_grouped_fwd(s, sv->x_perm, sv->offsets, w->w_gate, w->w_up, w->w_down, g->dhu, nullptr,
-                                 nullptr, ws, st, false, mxs, /*wfill=*/false));
+                                 nullptr, ws, st, /*x_quantized=*/rows_fp8, mxs, /*wfill=*/false));
     hu = g->dhu;
   }
   RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, hu, sv->a, sv->offsets, w->w_gate, w->w_up,
@@ -420,10 +462,11 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
   char *wsc = static_cast<char *>(ws);
   void *w_rt = wsc + L.w_rt;
   RETURN_IF(cuda_rc(launch_router_transpose(s, w->w_router, w_rt, st)));
+  // dW_r = x^T dz over the routed rows: x_perm's rows, or x's rows through pair_of_slot
   RETURN_IF(cuda_rc(launch_router_wgrad_grouped(s, sv->x_perm, sv->pair_of_slot, sv->offsets, g->dgate,
                                                 sv->topk_gate, reinterpret_cast<float *>(wsc + L.dz_slot),
                                                 reinterpret_cast<float *>(wsc + L.rg_partial), g->dw_router,
-                                                st)));
+                                                st, rows_fp8 ? x : nullptr)));
   // dx = sum_j dx_perm[slot(t,j)] + dz W_r^T in one pass
   return cuda_rc(launch_unpermute_sum(s, g->dx_perm, sv->slot_of_pair, g->dgate, sv->topk_gate, sv->topk_idx,
                                       w_rt, shared, g->dx, st));

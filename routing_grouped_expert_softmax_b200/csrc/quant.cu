@@ -486,14 +486,15 @@ __global__ void __launch_bounds__(256) mx_permute_kernel(const bf16 *__restrict_
 //   backward (BWD = true):  dy_perm[s] = bf16(g dY[t])    (src = dY), dgate = <dY[t], y_perm[s]>
 // and in the same pass the row in MXFP8 along d (codes_r, blocks of 32 columns; may be null)
 // and down the token axis (codes_c, blocks of 32 rows of the expert-padded layout), scales in
-// the GEMMs' tile layout.  Pad rows are zeros.
+// the GEMMs' tile layout (tiled) or plain ([rows][d/32] and [rows/32][d]).  out_perm may be
+// null (the bf16 rows are not written).  Pad rows are zeros.
 constexpr int CB_CHUNK = 256;
 template <bool BWD>
 __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
     const bf16 *__restrict__ src, const bf16 *__restrict__ y_perm, const int32_t *__restrict__ pos,
     const int32_t *__restrict__ offsets, const float *__restrict__ gate, int E, int k, int d, int64_t nkt,
     bf16 *__restrict__ out_perm, float *__restrict__ dgate, uint8_t *__restrict__ codes_r,
-    uint8_t *__restrict__ scales_r, uint8_t *__restrict__ codes_c, uint8_t *__restrict__ scales_c) {
+    uint8_t *__restrict__ scales_r, uint8_t *__restrict__ codes_c, uint8_t *__restrict__ scales_c, bool tiled) {
   __shared__ int pre[MAX_E + 1];
   __shared__ float colmax[8][CB_CHUNK];
   __shared__ float inv_col[CB_CHUNK];
@@ -542,11 +543,11 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
             dot[i] = fmaf(fd[j], fy[j], dot[i]);
             v[i][j] = gt[i] * fd[j];
           }
-          const uint4 o = Vec<bf16>::store(v[i]);                // the stored bf16 dy_perm row
-          *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = o;
+          const uint4 o = Vec<bf16>::store(v[i]);                // the bf16 dy_perm row
+          if (out_perm) *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = o;
           Vec<bf16>::load(o, v[i]);
         } else {
-          *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = raw;   // the permute: a bit copy
+          if (out_perm) *reinterpret_cast<uint4 *>(out_perm + slot * d + c) = raw;   // a bit copy
           Vec<bf16>::load(raw, v[i]);
         }
       } else {
@@ -569,7 +570,8 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
       w.y = (uint32_t)e4m3x2(v[i][4] * inv, v[i][5] * inv) | ((uint32_t)e4m3x2(v[i][6] * inv, v[i][7] * inv) << 16);
       if (cin && codes_r) {
         *reinterpret_cast<uint2 *>(codes_r + prow[i] * d + c) = w;
-        if ((lane & 3) == 0) scales_r[sf_tiled_off(prow[i], c / 32, d / 128)] = (uint8_t)(sc + 127);
+        if ((lane & 3) == 0)
+          scales_r[tiled ? sf_tiled_off(prow[i], c / 32, d / 128) : prow[i] * (d / 32) + c / 32] = (uint8_t)(sc + 127);
       }
     }
     // down the token axis: the block's 32 rows of each column
@@ -584,7 +586,8 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
       for (int w = 0; w < 8; ++w) amax = fmaxf(amax, colmax[w][threadIdx.x]);
       const int sc = mx_scale_exp(amax);
       inv_col[threadIdx.x] = exp2_neg(sc);
-      if (c0 + (int)threadIdx.x < d) scales_c[sf_tiled_off(c0 + threadIdx.x, blk, nkt)] = (uint8_t)(sc + 127);
+      if (c0 + (int)threadIdx.x < d)
+        scales_c[tiled ? sf_tiled_off(c0 + threadIdx.x, blk, nkt) : blk * d + c0 + threadIdx.x] = (uint8_t)(sc + 127);
     }
     __syncthreads();
 #pragma unroll
@@ -611,21 +614,21 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
 cudaError_t launch_mx_combine_bwd(const void *dy, const void *y_perm, const int32_t *pos, const int32_t *offsets,
                                   const float *gate, int E, int k, int d, int64_t rows_bound, void *dy_perm,
                                   float *dgate, uint8_t *codes_r, uint8_t *scales_r, uint8_t *codes_c,
-                                  uint8_t *scales_c, cudaStream_t st) {
+                                  uint8_t *scales_c, cudaStream_t st, bool tiled) {
   if (rows_bound <= 0) return cudaSuccess;
   mx_slot_dispatch_kernel<true><<<(unsigned)((rows_bound + 31) / 32), 256, 0, st>>>(
       static_cast<const bf16 *>(dy), static_cast<const bf16 *>(y_perm), pos, offsets, gate, E, k, d,
-      (rows_bound + 127) / 128, static_cast<bf16 *>(dy_perm), dgate, codes_r, scales_r, codes_c, scales_c);
+      (rows_bound + 127) / 128, static_cast<bf16 *>(dy_perm), dgate, codes_r, scales_r, codes_c, scales_c, tiled);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mx_dispatch(const void *x, const int32_t *pos, const int32_t *offsets, int E, int k, int d,
                                int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r,
-                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st) {
+                               uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st, bool tiled) {
   if (rows_bound <= 0) return cudaSuccess;
   mx_slot_dispatch_kernel<false><<<(unsigned)((rows_bound + 31) / 32), 256, 0, st>>>(
       static_cast<const bf16 *>(x), nullptr, pos, offsets, nullptr, E, k, d, (rows_bound + 127) / 128,
-      static_cast<bf16 *>(x_perm), nullptr, codes_r, scales_r, codes_c, scales_c);
+      static_cast<bf16 *>(x_perm), nullptr, codes_r, scales_r, codes_c, scales_c, tiled);
   return cudaGetLastError();
 }
 

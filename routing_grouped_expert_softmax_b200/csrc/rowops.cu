@@ -9,6 +9,9 @@
 //
 // Every kernel gives one warp to one token and moves its rows as 16-byte vectors
 // (8 bf16 or 4 fp32 per lane per access), so each row access is fully coalesced.
+#include <algorithm>
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
@@ -56,8 +59,9 @@ __global__ void __launch_bounds__(ROW_THREADS) permute_kernel(const uint4 *__res
   }
 }
 
-// y[t] = sum_j g[t,j] * y_perm[slot(t,j)]   (fp32 accumulation)
-template <typename T>
+// y[t] = sum_j g[t,j] * y_perm[slot(t,j)]   (fp32 accumulation).  KC >= k: all k rows'
+// vectors of a pass are loaded before the first is used, so k loads are in flight at once.
+template <typename T, int KC>
 __global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__restrict__ y_perm,
                                                               const int32_t *__restrict__ sop,
                                                               const float *__restrict__ gate,
@@ -67,10 +71,18 @@ __global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__res
   const int lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * ROW_WARPS + (threadIdx.x >> 5);
   if (t >= Tn) return;
-  int64_t my_slot = lane_slot(sop, t, k);
-  float my_g = lane < k ? gate[t * k + lane] : 0.f;
+  const int my_slot = lane < k ? sop[t * k + lane] : 0;
+  const float my_g = lane < k ? gate[t * k + lane] : 0.f;
+  int slot[KC];
+  float g[KC];
+#pragma unroll
+  for (int j = 0; j < KC; ++j) {
+    slot[j] = __shfl_sync(0xffffffffu, my_slot, j);
+    g[j] = __shfl_sync(0xffffffffu, my_g, j);
+  }
   for (int v0 = 0; v0 < nv; v0 += 64) {
     float acc[2][N];
+    uint4 raw[2][KC];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int v = v0 + u * 32 + lane;
@@ -80,29 +92,24 @@ __global__ void __launch_bounds__(ROW_THREADS) combine_kernel(const uint4 *__res
 #pragma unroll
         for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
       }
-    }
 #pragma unroll
-    for (int j = 0; j < MAX_K; ++j) {
-      if (j < k) {
-        int64_t slot = __shfl_sync(0xffffffffu, my_slot, j);
-        float g = __shfl_sync(0xffffffffu, my_g, j);
-        const uint4 *src = y_perm + slot * nv;
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          int v = v0 + u * 32 + lane;
-          if (v < nv) {
-            float f[N];
-            Vec<T>::load(__ldg(src + v), f);
-#pragma unroll
-            for (int i = 0; i < N; ++i) acc[u][i] = fmaf(g, f[i], acc[u][i]);
-          }
-        }
-      }
+      for (int j = 0; j < KC; ++j)
+        raw[u][j] = (j < k && v < nv) ? __ldg(y_perm + (int64_t)slot[j] * nv + v) : make_uint4(0, 0, 0, 0);
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      int v = v0 + u * 32 + lane;
-      if (v < nv) y[t * nv + v] = Vec<T>::store(acc[u]);
+      const int v = v0 + u * 32 + lane;
+      if (v >= nv) continue;
+#pragma unroll
+      for (int j = 0; j < KC; ++j) {
+        if (j < k) {
+          float f[N];
+          Vec<T>::load(raw[u][j], f);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[u][i] = fmaf(g[j], f[i], acc[u][i]);
+        }
+      }
+      y[t * nv + v] = Vec<T>::store(acc[u]);
     }
   }
 }
@@ -238,6 +245,139 @@ __global__ void __launch_bounds__(ROW_THREADS) unpermute_sum_kernel(
   }
 }
 
+// The same sum with the router term, by column slices: a block owns 32 vectors (512 bytes)
+// of every row and first stages that slice of W_r^T for all E experts in shared memory, so
+// a router weight is read from L2 once per block instead of once per routed pair.  A warp
+// takes two tokens per pass (2k row loads in flight); the terms are added in the order of
+// unpermute_sum_kernel, so the two kernels give the same bits.
+constexpr int US_THREADS = 256;
+constexpr int US_WARPS = US_THREADS / 32;
+template <typename T, int KC>
+__global__ void __launch_bounds__(US_THREADS) unpermute_sum_router_kernel(
+    const uint4 *__restrict__ dx_perm, const int32_t *__restrict__ sop,
+    const float *__restrict__ dgate, const float *__restrict__ gate, const int32_t *__restrict__ idx,
+    const uint4 *__restrict__ w_rt, bool accumulate, uint4 *__restrict__ dx, int64_t Tn, int k,
+    int nv, int E) {
+  extern __shared__ uint4 w_slice[];   // [E][32]
+  constexpr int N = Vec<T>::N;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int v0 = blockIdx.y * 32;
+  const int v = v0 + lane;
+  const bool vin = v < nv;             // (nv % 32 != 0 only for bf16 rows of d % 256 == 128)
+  // a token pair's metadata, lane j < k holding pair j's: slot, expert, gate, gate gradient;
+  // the next pair's is loaded while this pair's rows are in flight
+  struct Meta {
+    int slot[2], e[2];
+    float g[2], dg[2];
+  };
+  auto load_meta = [&](int64_t t0, Meta &m) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int64_t t = t0 + u < Tn ? t0 + u : t0;
+      const bool on = lane < k;
+      m.slot[u] = (dx_perm && on) ? sop[t * k + lane] : 0;
+      m.e[u] = on ? idx[t * k + lane] : 0;
+      m.g[u] = on ? gate[t * k + lane] : 0.f;
+      m.dg[u] = on ? dgate[t * k + lane] : 0.f;
+    }
+  };
+  const int64_t stride = (int64_t)gridDim.x * US_WARPS * 2;
+  int64_t t0 = ((int64_t)blockIdx.x * US_WARPS + warp) * 2;
+  Meta cur{};
+  if (t0 < Tn) load_meta(t0, cur);
+  for (int i = threadIdx.x; i < E * 32; i += US_THREADS) {
+    const int vv = v0 + (i & 31);
+    if (vv < nv) w_slice[i] = __ldg(w_rt + (int64_t)(i >> 5) * nv + vv);
+  }
+  __syncthreads();
+  for (; t0 < Tn; t0 += stride) {
+    const int nt = t0 + 1 < Tn ? 2 : 1;
+    int slot[2][KC], e[2][KC];
+    float dz[2][KC];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      // dz_j = g_j (dg_j - sum_i g_i dg_i), the sum in i order (as token_dz)
+      float g[KC], dg[KC], inner = 0.f;
+#pragma unroll
+      for (int j = 0; j < KC; ++j) {
+        slot[u][j] = __shfl_sync(0xffffffffu, cur.slot[u], j);
+        e[u][j] = __shfl_sync(0xffffffffu, cur.e[u], j);
+        g[j] = __shfl_sync(0xffffffffu, cur.g[u], j);
+        dg[j] = __shfl_sync(0xffffffffu, cur.dg[u], j);
+        if (j < k) inner = fmaf(g[j], dg[j], inner);
+      }
+#pragma unroll
+      for (int j = 0; j < KC; ++j) dz[u][j] = (j < k) ? g[j] * (dg[j] - inner) : 0.f;
+    }
+    float acc[2][N];
+    uint4 raw[2][KC];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (vin && u < nt && accumulate) {
+        Vec<T>::load(dx[(t0 + u) * nv + v], acc[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) acc[u][i] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < KC; ++j)
+        raw[u][j] = (vin && dx_perm && j < k && u < nt) ? __ldg(dx_perm + (int64_t)slot[u][j] * nv + v)
+                                                        : make_uint4(0, 0, 0, 0);
+    }
+    if (t0 + stride < Tn) load_meta(t0 + stride, cur);
+    if (!vin) continue;
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (u >= nt) break;
+#pragma unroll
+      for (int j = 0; j < KC; ++j) {
+        if (j < k) {
+          float f[N];
+          if (dx_perm) {
+            Vec<T>::load(raw[u][j], f);
+#pragma unroll
+            for (int i = 0; i < N; ++i) acc[u][i] += f[i];
+          }
+          Vec<T>::load(w_slice[e[u][j] * 32 + lane], f);
+#pragma unroll
+          for (int i = 0; i < N; ++i) acc[u][i] = fmaf(dz[u][j], f[i], acc[u][i]);
+        }
+      }
+      dx[(t0 + u) * nv + v] = Vec<T>::store(acc[u]);
+    }
+  }
+}
+
+template <typename T, int KC>
+static cudaError_t launch_unpermute_sum_router(const uint4 *a, const int32_t *sop, const float *dgate,
+                                               const float *gate, const int32_t *idx, const uint4 *w,
+                                               bool accumulate, uint4 *o, int64_t T_, int k, int nv, int E,
+                                               cudaStream_t st) {
+  // column slices of 32 vectors; enough token groups to fill every SM at the occupancy the
+  // staged W_r^T slice ([E][512 bytes]) allows
+  const int nslices = (nv + 31) / 32;
+  const int smem = E * 32 * 16;
+  auto kern = unpermute_sum_router_kernel<T, KC>;
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+  }
+  // resident blocks per SM at this E (registers and the staged slice decide), cached per E
+  static std::atomic<int> occ_cache[MAX_E + 1];
+  int per_sm = occ_cache[E].load(std::memory_order_relaxed);
+  if (per_sm <= 0) {
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, US_THREADS, smem) != cudaSuccess || per_sm <= 0)
+      per_sm = 1;
+    occ_cache[E].store(per_sm, std::memory_order_relaxed);
+  }
+  const int64_t pairs = (T_ + 1) / 2;
+  const int64_t gx = std::max<int64_t>(1, std::min<int64_t>((device_sm_count() * per_sm + nslices - 1) / nslices,
+                                                            (pairs + US_WARPS - 1) / US_WARPS));
+  kern<<<dim3((unsigned)gx, (unsigned)nslices), US_THREADS, smem, st>>>(a, sop, dgate, gate, idx, w, accumulate, o,
+                                                                        T_, k, nv, E);
+  return cudaGetLastError();
+}
+
 // w_rt[e][i] = W_r[i][e] (same storage type), 32x32 tiles through shared memory.
 template <typename T>
 __global__ void router_transpose_kernel(const T *__restrict__ w_r, T *__restrict__ w_rt, int d,
@@ -329,7 +469,7 @@ cudaError_t launch_transpose_batched(const float *src, float *dst, int B, int R,
 // belongs to that expert; a second kernel adds an expert's chunks in order.
 // ---------------------------------------------------------------------------------------
 constexpr int RG_ROWS = 64;
-constexpr int RG_THREADS = 128;  // x 2 columns = 256 columns per block
+constexpr int RG_THREADS = 128;  // x one 16-byte vector each
 
 // dz_slot[s] = g (dg - sum_j' g_j' dg_j') of the pair in slot s
 __global__ void router_dz_slot_kernel(const int32_t *__restrict__ pos, const float *__restrict__ dgate,
@@ -371,10 +511,14 @@ __device__ int chunk_prefix(const int32_t *offsets, int E, int *prefix) {
   return __shfl_sync(0xffffffffu, incl, 31);
 }
 
+// x_perm rows in slot order, or (pos != nullptr) the layer input's rows x[pos[slot] / k].
+// Thread v owns one 16-byte vector (8 bf16 or 4 fp32 columns) of the rows; each column's
+// sum runs over the chunk's rows in order.
 template <typename T>
 __global__ void __launch_bounds__(RG_THREADS) router_wgrad_grouped_kernel(
-    const T *__restrict__ x_perm, const float *__restrict__ dz_slot, const int32_t *__restrict__ offsets,
-    float *__restrict__ partial, int E, int d) {
+    const uint4 *__restrict__ x_perm, const float *__restrict__ dz_slot, const int32_t *__restrict__ offsets,
+    float *__restrict__ partial, int E, int d, const int32_t *__restrict__ pos, int k) {
+  constexpr int N = Vec<T>::N;
   __shared__ int prefix[MAX_E + 1];
   if (threadIdx.x < 32) chunk_prefix(offsets, E, prefix);
   __syncthreads();
@@ -388,31 +532,40 @@ __global__ void __launch_bounds__(RG_THREADS) router_wgrad_grouped_kernel(
   const int e = lo;
   const int r0 = offsets[e] + (q - prefix[e]) * RG_ROWS;
   const int r1 = min(offsets[e + 1], r0 + RG_ROWS);
-  const int c = (blockIdx.y * RG_THREADS + threadIdx.x) * 2;
-  if (c >= d) return;
-  float a0 = 0.f, a1 = 0.f;
+  const int nv = d / N;
+  const int v = blockIdx.y * RG_THREADS + threadIdx.x;
+  if (v >= nv) return;
+  auto row_of = [&](int slot) -> int64_t { return pos ? (int64_t)(pos[slot] / k) : (int64_t)slot; };
+  float a[N];
+#pragma unroll
+  for (int i = 0; i < N; ++i) a[i] = 0.f;
   int r = r0;
   for (; r + 4 <= r1; r += 4) {
-    float z[4], x0[4], x1[4];
+    float z[4];
+    uint4 raw[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       z[u] = dz_slot[r + u];
-      x0[u] = to_f(x_perm[(int64_t)(r + u) * d + c]);
-      x1[u] = to_f(x_perm[(int64_t)(r + u) * d + c + 1]);
+      raw[u] = __ldg(x_perm + row_of(r + u) * nv + v);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      a0 = fmaf(z[u], x0[u], a0);
-      a1 = fmaf(z[u], x1[u], a1);
+      float f[N];
+      Vec<T>::load(raw[u], f);
+#pragma unroll
+      for (int i = 0; i < N; ++i) a[i] = fmaf(z[u], f[i], a[i]);
     }
   }
   for (; r < r1; ++r) {
-    float z = dz_slot[r];
-    a0 = fmaf(z, to_f(x_perm[(int64_t)r * d + c]), a0);
-    a1 = fmaf(z, to_f(x_perm[(int64_t)r * d + c + 1]), a1);
+    const float z = dz_slot[r];
+    float f[N];
+    Vec<T>::load(__ldg(x_perm + row_of(r) * nv + v), f);
+#pragma unroll
+    for (int i = 0; i < N; ++i) a[i] = fmaf(z, f[i], a[i]);
   }
-  partial[(int64_t)q * d + c] = a0;
-  partial[(int64_t)q * d + c + 1] = a1;
+  float4 *out = reinterpret_cast<float4 *>(partial + (int64_t)q * d + (int64_t)v * N);
+#pragma unroll
+  for (int i = 0; i < N; i += 4) out[i / 4] = make_float4(a[i], a[i + 1], a[i + 2], a[i + 3]);
 }
 
 // dW_r[c][e] = sum of expert e's chunk partials, in chunk order (0 for an empty expert).
@@ -432,17 +585,21 @@ __global__ void router_wgrad_grouped_reduce_kernel(const float *__restrict__ par
 
 cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, const int32_t *pos,
                                         const int32_t *offsets, const float *dgate, const float *gate,
-                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st) {
+                                        float *dz_slot, float *partial, float *dw_r, cudaStream_t st,
+                                        const void *x) {
+  const void *rows = x ? x : x_perm;
+  const int32_t *rpos = x ? pos : nullptr;
   const int64_t P = s.P();
   router_dz_slot_kernel<<<(unsigned)((P + 255) / 256), 256, 0, st>>>(pos, dgate, gate, dz_slot, P, s.k);
   const int64_t max_chunks = (P + RG_ROWS - 1) / RG_ROWS + s.E;
-  dim3 grid((unsigned)max_chunks, (unsigned)((s.d / 2 + RG_THREADS - 1) / RG_THREADS));
+  const int nv = s.d * s.es() / 16;
+  dim3 grid((unsigned)max_chunks, (unsigned)((nv + RG_THREADS - 1) / RG_THREADS));
   if (s.dtype == MOE_BF16)
-    router_wgrad_grouped_kernel<bf16><<<grid, RG_THREADS, 0, st>>>(static_cast<const bf16 *>(x_perm), dz_slot,
-                                                                   offsets, partial, s.E, s.d);
+    router_wgrad_grouped_kernel<bf16><<<grid, RG_THREADS, 0, st>>>(static_cast<const uint4 *>(rows), dz_slot,
+                                                                   offsets, partial, s.E, s.d, rpos, s.k);
   else
-    router_wgrad_grouped_kernel<float><<<grid, RG_THREADS, 0, st>>>(static_cast<const float *>(x_perm), dz_slot,
-                                                                    offsets, partial, s.E, s.d);
+    router_wgrad_grouped_kernel<float><<<grid, RG_THREADS, 0, st>>>(static_cast<const uint4 *>(rows), dz_slot,
+                                                                    offsets, partial, s.E, s.d, rpos, s.k);
   dim3 g2((unsigned)((s.d + 255) / 256), (unsigned)s.E);
   router_wgrad_grouped_reduce_kernel<<<g2, 256, 0, st>>>(partial, offsets, dw_r, s.E, s.d);
   return cudaGetLastError();
@@ -451,17 +608,23 @@ cudaError_t launch_router_wgrad_grouped(const Shape &s, const void *x_perm, cons
 // ---------------------------------------------------------------------------------------
 // Tail buffers of the bf16 weight-gradient GEMMs, which reduce over each expert's rows in
 // K-blocks of 64: the expert's last, partial block is copied into its own 64 rows with zeros
-// after the expert's rows, so that the GEMM loads it like any other block.  One block per
-// (row i of the tail, expert e).
+// after the expert's rows, so that the GEMM loads it like any other block.  The GEMM reads
+// only the 16-row slices that hold expert rows, so rows from the next multiple of 16 on are
+// left as they are.  One block per (row i of the tail, expert e, operand: A or B).
 // ---------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) wgrad_tail_kernel(const uint4 *__restrict__ src, int nv,
-                                                         const int32_t *__restrict__ offsets,
-                                                         uint4 *__restrict__ tails) {
+__global__ void __launch_bounds__(128) wgrad_tail_kernel(const uint4 *__restrict__ src_a, int nv_a,
+                                                         uint4 *__restrict__ tails_a,
+                                                         const uint4 *__restrict__ src_b, int nv_b,
+                                                         uint4 *__restrict__ tails_b,
+                                                         const int32_t *__restrict__ offsets) {
   const int i = blockIdx.x, e = blockIdx.y;
   const int lo = offsets[e], cnt = offsets[e + 1] - lo;
   const int full = cnt / WGRAD_TAIL_ROWS * WGRAD_TAIL_ROWS, v = cnt - full;
-  if (v == 0) return;                        // no partial block: the tail rows are never read
-  uint4 *dst = tails + ((int64_t)e * WGRAD_TAIL_ROWS + i) * nv;
+  if (v == 0 || i >= (v + 15) / 16 * 16) return;   // rows the GEMM never reads
+  const bool b = blockIdx.z == 1;
+  const uint4 *src = b ? src_b : src_a;
+  const int nv = b ? nv_b : nv_a;
+  uint4 *dst = (b ? tails_b : tails_a) + ((int64_t)e * WGRAD_TAIL_ROWS + i) * nv;
   if (i < v) {
     const uint4 *row = src + ((int64_t)lo + full + i) * nv;
     for (int c = threadIdx.x; c < nv; c += 128) dst[c] = __ldg(row + c);
@@ -470,10 +633,12 @@ __global__ void __launch_bounds__(128) wgrad_tail_kernel(const uint4 *__restrict
   }
 }
 
-cudaError_t launch_wgrad_tails(const void *src, int C, const int32_t *offsets, int E, void *tails, cudaStream_t st) {
-  dim3 grid(WGRAD_TAIL_ROWS, (unsigned)E);
-  wgrad_tail_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4 *>(src), C * 2 / 16, offsets,
-                                          static_cast<uint4 *>(tails));
+cudaError_t launch_wgrad_tails(const void *src_a, int C_a, void *tails_a, const void *src_b, int C_b, void *tails_b,
+                               const int32_t *offsets, int E, cudaStream_t st) {
+  dim3 grid(WGRAD_TAIL_ROWS, (unsigned)E, 2);
+  wgrad_tail_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4 *>(src_a), C_a * 2 / 16,
+                                          static_cast<uint4 *>(tails_a), static_cast<const uint4 *>(src_b),
+                                          C_b * 2 / 16, static_cast<uint4 *>(tails_b), offsets);
   return cudaGetLastError();
 }
 
@@ -495,10 +660,14 @@ cudaError_t launch_unpermute_combine(const Shape &s, const void *y_perm, const i
   int nv = s.d * s.es() / 16;
   auto yp = static_cast<const uint4 *>(y_perm);
   auto yo = static_cast<uint4 *>(y);
-  if (s.dtype == MOE_BF16)
-    combine_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
-  else
-    combine_kernel<float><<<row_grid(s.T), ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+  const dim3 grid(row_grid(s.T));
+  if (s.dtype == MOE_BF16) {
+    if (s.k <= 4) combine_kernel<bf16, 4><<<grid, ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+    else combine_kernel<bf16, MAX_K><<<grid, ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+  } else {
+    if (s.k <= 4) combine_kernel<float, 4><<<grid, ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+    else combine_kernel<float, MAX_K><<<grid, ROW_THREADS, 0, st>>>(yp, sop, gate, yo, s.T, s.k, nv, accumulate);
+  }
   return cudaGetLastError();
 }
 
@@ -537,6 +706,17 @@ cudaError_t launch_unpermute_sum(const Shape &s, const void *dx_perm, const int3
   auto a = static_cast<const uint4 *>(dx_perm);
   auto w = static_cast<const uint4 *>(w_rt);
   auto o = static_cast<uint4 *>(dx);
+  if (w) {
+    if (s.dtype == MOE_BF16)
+      return s.k <= 4 ? launch_unpermute_sum_router<bf16, 4>(a, sop, dgate, gate, idx, w, accumulate, o, s.T, s.k,
+                                                              nv, s.E, st)
+                      : launch_unpermute_sum_router<bf16, MAX_K>(a, sop, dgate, gate, idx, w, accumulate, o, s.T,
+                                                                 s.k, nv, s.E, st);
+    return s.k <= 4 ? launch_unpermute_sum_router<float, 4>(a, sop, dgate, gate, idx, w, accumulate, o, s.T, s.k, nv,
+                                                             s.E, st)
+                    : launch_unpermute_sum_router<float, MAX_K>(a, sop, dgate, gate, idx, w, accumulate, o, s.T,
+                                                                s.k, nv, s.E, st);
+  }
   if (s.dtype == MOE_BF16)
     unpermute_sum_kernel<bf16><<<row_grid(s.T), ROW_THREADS, 0, st>>>(a, sop, dgate, gate, idx, w,
                                                                       accumulate, o, s.T, s.k, nv);

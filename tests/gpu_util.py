@@ -135,7 +135,8 @@ def check_layer(y, saved, grads, fwd, bwd, f, tol, tol_combine, tag=""):
     metadata and the permuted rows, the stated tolerances for floating point)."""
     for key in ("counts", "offsets", "slot_of_pair", "pair_of_slot"):
         assert np.array_equal(host(saved[key]), fwd[key]), key
-    assert np.array_equal(host(saved["x_perm"]), fwd["x_perm"])
+    if saved.get("x_perm") is not None:      # (None: the rows moved in MXFP8 only)
+        assert np.array_equal(host(saved["x_perm"]), fwd["x_perm"])
     assert np.max(np.abs(host(saved["topk_gate"]) - fwd["gate"])) <= 1e-5
     if saved.get("hu") is not None:
         hu = host(saved["hu"])
@@ -152,7 +153,8 @@ def check_layer(y, saved, grads, fwd, bwd, f, tol, tol_combine, tag=""):
             check(shu[:, f:], fwd["shared_u"], tol, tag + "shared_u")
     if grads is None:
         return
-    check(host(grads["dy_perm"]), bwd["dy_perm"], tol_combine, tag + "dy_perm")
+    if grads.get("dy_perm") is not None:
+        check(host(grads["dy_perm"]), bwd["dy_perm"], tol_combine, tag + "dy_perm")
     check(host(grads["dgate"]), bwd["dgate"], tol, tag + "dgate")
     dhu = host(grads["dhu"])
     check(dhu[:, :f], bwd["dh"], tol, tag + "dh")

@@ -98,8 +98,8 @@ def test_gemm_algorithmic_bytes_and_binding_roof():
 def test_launch_count():
     sys.path.insert(0, ROOT)
     import bench
-    assert bench.count_launches("router") == 18
-    assert bench.count_launches("uniform") == 13
+    assert bench.count_launches("router") == 20
+    assert bench.count_launches("uniform") == 15
     assert bench.count_launches("router", "mxfp8") == 22
-    assert bench.count_launches("router", "native", shared=True) == 26
-    assert bench.count_launches("router", "native", recompute=True) == 19
+    assert bench.count_launches("router", "native", shared=True) == 30
+    assert bench.count_launches("router", "native", recompute=True) == 21

@@ -85,9 +85,10 @@ def _mx_sampled(inp, y, saved, grads, zg, routed):
     hu, dhu = host(saved["hu"])[full_slot], host(grads["dhu"])[full_slot]
     rows = dict(h=(hu[:, :f], fwd["h"]), u=(hu[:, f:], fwd["u"]), a=(host(saved["a"])[full_slot], fwd["a"]),
                 y_perm=(host(saved["y_perm"])[full_slot], fwd["y_perm"]),
-                dy_perm=(host(grads["dy_perm"])[full_slot], bwd["dy_perm"]),
                 dh=(dhu[:, :f], bwd["dh"]), du=(dhu[:, f:], bwd["du"]),
                 dx_perm=(host(grads["dx_perm"])[full_slot], bwd["dx_perm"]))
+    if grads["dy_perm"] is not None:      # (None: dy_perm moved in MXFP8 only)
+        rows["dy_perm"] = (host(grads["dy_perm"])[full_slot], bwd["dy_perm"])
     for n, (g_rows, o_rows) in rows.items():
         check(g_rows, o_rows[sub_slot], TOL_MX, f"mxfp8 full-size sampled {n}")
     # three experts' weight gradients from their own rows (k = 1 sub-batches, same gates)

@@ -137,6 +137,84 @@ def test_permute_mxfp8_is_the_permute_and_the_row_quantiser(T, d, E, k):
     assert np.all(hc[~valid] == 0xAB) and np.all(hs[~valid] == 0xAB)
 
 
+def _both_orientations(bound, d):
+    import torch
+    u8 = dict(dtype=torch.uint8, device="cuda")
+    return (torch.full((bound, d), 0xAB, **u8), torch.full((bound, d // 32), 0xAB, **u8),
+            torch.full((bound, d), 0xAB, **u8), torch.full(((bound + 31) // 32, d), 0xAB, **u8))
+
+
+def _check_both_orientations(rows, offsets, cr, sr, cc, sc):
+    """codes/scales along d and down the padded token axis bit for bit as the oracle's OCP MX
+    rule on the expert-padded layout of `rows` (pad rows: zero codes, scale byte 0); the rows
+    past the last expert's 128-row block untouched."""
+    pv = _padded(rows, offsets)
+    n = pv.shape[0]
+    rc, rs, _ = ref.mx_quantize(pv, axis=1)
+    tc, ts, _ = ref.mx_quantize(pv, axis=0)
+    hcr, hsr, hcc, hsc = host(cr), host(sr), host(cc), host(sc)
+    assert np.array_equal(hcr[:n], rc) and np.array_equal(hsr[:n], rs)
+    assert np.array_equal(hcc[:n], tc) and np.array_equal(hsc[:n // 32], ts)
+    assert np.all(hcr[n:] == 0xAB) and np.all(hsr[n:] == 0xAB)
+    assert np.all(hcc[n:] == 0xAB) and np.all(hsc[n // 32:] == 0xAB)
+
+
+@pytest.mark.parametrize("T,d,E,k,bf16_copy", [(300, 256, 8, 2, True), (1000, 2048, 128, 4, False),
+                                               (77, 128, 5, 3, True), (513, 1024, 16, 8, False)])
+def test_dispatch_mxfp8_writes_both_orientations(T, d, E, k, bf16_copy):
+    """FP8 dispatch from x itself: each routed row read once through pair_of_slot and written
+    in MXFP8 along d and down the padded token axis, bit for bit as the oracle quantises its
+    own permute; the bf16 copy, when asked for, bit for bit as the oracle's permute."""
+    import torch
+    idx, _ = gen.uniform_random_routing(T, E, k, seed=T + 1)
+    counts, offsets, sop, pos = ref.routing_metadata(idx, E)
+    x = _special_data(T, d, T + 2)
+    cfg = moe.config(T, d, E, k, 128)
+    bound = T * k + 127 * E
+    xp = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda") if bf16_copy else None
+    cr, sr, cc, sc = _both_orientations(bound, d)
+    moe.moe_dispatch_mxfp8(cfg, dev(x, "bf16"), dev_i32(pos), dev_i32(offsets), bound, xp, cr, sr, cc, sc)
+    xpr = ref.permute(x, pos, k)
+    if bf16_copy:
+        assert np.array_equal(host(xp), xpr)
+    _check_both_orientations(xpr, offsets, cr, sr, cc, sc)
+
+
+@pytest.mark.parametrize("T,d,E,k", [(300, 256, 8, 2), (1000, 2048, 128, 4), (77, 128, 5, 3)])
+def test_combine_bwd_mxfp8_against_oracle(T, d, E, k):
+    """The combine's backward dispatched in MXFP8: dgate against the oracle within fp32
+    rounding, the bf16 dy_perm and both MXFP8 orientations of it bit for bit.  The rounding of
+    g * dY to bf16 decides the codes, so the oracle takes that product in the kernel's float32
+    (its working precision for this call) before rounding it to bf16."""
+    import torch
+    idx, gate = gen.uniform_random_routing(T, E, k, seed=T + 3)
+    counts, offsets, sop, pos = ref.routing_metadata(idx, E)
+    rng = np.random.default_rng(T)
+    gate = (gate * rng.uniform(0.2, 1.8, gate.shape)).astype(np.float32)
+    dY = _special_data(T, d, T + 4)
+    y_perm = grid(rng.standard_normal((T * k, d), dtype=np.float32), "bf16")
+    cfg = moe.config(T, d, E, k, 128)
+    bound = T * k + 127 * E
+    dyp = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    dgate = torch.empty(T, k, dtype=torch.float32, device="cuda")
+    cr, sr, cc, sc = _both_orientations(bound, d)
+    moe.moe_combine_bwd_mxfp8(cfg, dev(dY, "bf16"), dev(y_perm, "bf16"), dev_i32(pos), dev_i32(offsets),
+                              dev_f32(gate), bound, dyp, dgate, cr, sr, cc, sc)
+    with ref.working_precision(np.float32):
+        r_dyp, _ = ref.combine_bwd(dY, y_perm, sop, gate)
+    _, r_dg = ref.combine_bwd(dY, y_perm, sop, gate)
+    r_dyp = ref.bf16_rne(r_dyp)
+    assert np.array_equal(host(dyp), r_dyp)
+    assert rel_err(host(dgate), r_dg) <= 1e-4
+    _check_both_orientations(r_dyp, offsets, cr, sr, cc, sc)
+    # without the bf16 copy: the same codes
+    cr2, sr2, cc2, sc2 = _both_orientations(bound, d)
+    moe.moe_combine_bwd_mxfp8(cfg, dev(dY, "bf16"), dev(y_perm, "bf16"), dev_i32(pos), dev_i32(offsets),
+                              dev_f32(gate), bound, None, dgate, cr2, sr2, cc2, sc2)
+    for a_, b_ in ((cr, cr2), (sr, sr2), (cc, cc2), (sc, sc2)):
+        assert torch.equal(a_, b_)
+
+
 # ------------------------------------------------------------------ grouped GEMMs
 
 MX_CASES = [

@@ -99,6 +99,9 @@ def test_recompute_against_oracle_and_saving_path(T, d, E, k, f, shared, prec):
     # and bit for bit against the path that keeps h | u
     assert np.array_equal(host(y0), host(y1))
     for n in ("a", "y_perm", "x_perm") + (("shared_a",) if shared else ()):
+        if s0[n] is None:             # x_perm: the MXFP8 layer moves the rows in MXFP8 only
+            assert s1[n] is None, n
+            continue
         assert np.array_equal(host(s0[n]), host(s1[n])), n
     names = ["dx", "dw_router", "dw_gate", "dw_up", "dw_down", "dhu", "dx_perm", "dgate"]
     if shared:
