@@ -297,8 +297,11 @@ __global__ void __launch_bounds__(WQ_THREADS) mx_quant_weights_kernel(
   const int64_t r0 = (int64_t)blockIdx.y * WQ_ROWS;
   const int CO = gu ? 2 * C : C;
   // (1) the tile, 16-byte pieces (8 tile columns of one chunk each): every load of the thread
-  // in flight at once, then the shared-memory stores
+  // in flight at once, then the shared-memory stores.  Piece q of thread t is row t/vpr +
+  // q*(WQ_THREADS/vpr), columns 8*(t%vpr)..+7, so the four pieces of a 32-column block of a
+  // row sit in four adjacent lanes: the row scales come from the registers, by two shuffles.
   constexpr int vpr = NC / 8, NLD = WQ_ROWS * vpr / WQ_THREADS;
+  constexpr int nb = NC / 32;
   uint4 ld[NLD];
 #pragma unroll
   for (int q = 0; q < NLD; ++q) {
@@ -310,10 +313,25 @@ __global__ void __launch_bounds__(WQ_THREADS) mx_quant_weights_kernel(
   for (int q = 0; q < NLD; ++q) {
     const int idx = t + q * WQ_THREADS, row = idx / vpr, j = (idx - row * vpr) * 8;
     *reinterpret_cast<uint4 *>(tile + row * pitch + j) = ld[q];
+    float v[8];
+    Vec<bf16>::load(ld[q], v);
+    float amax = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    if ((t & 3) == 0) {
+      const int b = j / 32;
+      const int sc = mx_scale_exp(amax);
+      inv_r[row * nb + b] = exp2_neg(sc);
+      const int kb = m.rcol(j) / 32;                                    // K-block along the row
+      const int ti = gu ? m.tensor(j) : (j >> 7);                       // which staged tile
+      st_r[ti * 512 + 16 * (row & 31) + 4 * (row >> 5) + (kb & 3)] = (uint8_t)(sc + 127);
+    }
   }
   __syncthreads();
-  // (2) scales.  Column blocks: 4 row groups x NC columns, two adjacent columns per task
-  // (32 paired loads); row blocks: 128 rows x NC/32, 32 values as 4 vectors per task.
+  // (2) column scales: 4 row groups x NC columns, two adjacent columns per task (32 paired
+  // loads)
   for (int u = t; u < 2 * NC; u += WQ_THREADS) {
     const int grp = u / (NC / 2), j = 2 * (u - grp * (NC / 2));
     float a0 = 0.f, a1 = 0.f;
@@ -331,23 +349,6 @@ __global__ void __launch_bounds__(WQ_THREADS) mx_quant_weights_kernel(
       st_c[((j + h) >> 7) * 512 + 16 * (mn & 31) + 4 * (mn >> 5) + grp] = (uint8_t)(sc + 127);
     }
   }
-  constexpr int nb = NC / 32;
-  for (int u = t; u < WQ_ROWS * nb; u += WQ_THREADS) {
-    const int row = u / nb, b = u - row * nb, j = 32 * b;
-    float amax = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      float v[8];
-      Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j + 8 * i), v);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
-    }
-    const int sc = mx_scale_exp(amax);
-    inv_r[row * nb + b] = exp2_neg(sc);
-    const int kb = m.rcol(j) / 32;                                      // K-block along the row
-    const int ti = gu ? m.tensor(j) : (j >> 7);                         // which staged tile
-    st_r[ti * 512 + 16 * (row & 31) + 4 * (row >> 5) + (kb & 3)] = (uint8_t)(sc + 127);
-  }
   __syncthreads();
   // (3) the staged scale tiles, whole, with 16-byte stores
   for (int u = t; u < 2 * (NC / 128) * 32; u += WQ_THREADS) {
@@ -362,15 +363,24 @@ __global__ void __launch_bounds__(WQ_THREADS) mx_quant_weights_kernel(
           reinterpret_cast<const uint4 *>(st_r + ti * 512)[q];
     }
   }
-  // (4) codes: 16 tile columns of one row per task, in both orientations
-  constexpr int vr = NC / 16;
-  for (int u = t; u < WQ_ROWS * vr; u += WQ_THREADS) {
-    const int row = u / vr, j0 = (u - row * vr) * 16, grp = row >> 5;
+  // (4) codes in both orientations: thread t takes 16 tile columns of RPT consecutive rows of
+  // one 32-row group, so that the 16 column scales it needs are read once for all of them
+  constexpr int TPR = NC / 16, RPT = WQ_ROWS * TPR / WQ_THREADS;
+  static_assert(32 % RPT == 0, "a thread's rows lie in one row group");
+  const int j0 = (t % TPR) * 16, row0 = (t / TPR) * RPT, grp = row0 >> 5;
+  float ic[16];
+#pragma unroll
+  for (int i = 0; i < 16; i += 4) {
+    const float4 f = *reinterpret_cast<const float4 *>(inv_c + grp * NC + j0 + i);
+    ic[i] = f.x; ic[i + 1] = f.y; ic[i + 2] = f.z; ic[i + 3] = f.w;
+  }
+#pragma unroll
+  for (int rr = 0; rr < RPT; ++rr) {
+    const int row = row0 + rr;
     float v[16];
     Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j0), v);
     Vec<bf16>::load(*reinterpret_cast<const uint4 *>(tile + row * pitch + j0 + 8), v + 8);
     const float ir = inv_r[row * nb + j0 / 32];
-    const float *ic = inv_c + grp * NC + j0;
     uint32_t wc[4], wr[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -490,7 +500,7 @@ __global__ void __launch_bounds__(256) mx_permute_kernel(const bf16 *__restrict_
 // null (the bf16 rows are not written).  Pad rows are zeros.
 constexpr int CB_CHUNK = 256;
 template <bool BWD>
-__global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
+__global__ void __launch_bounds__(256, 2) mx_slot_dispatch_kernel(
     const bf16 *__restrict__ src, const bf16 *__restrict__ y_perm, const int32_t *__restrict__ pos,
     const int32_t *__restrict__ offsets, const float *__restrict__ gate, int E, int k, int d, int64_t nkt,
     bf16 *__restrict__ out_perm, float *__restrict__ dgate, uint8_t *__restrict__ codes_r,
@@ -511,33 +521,58 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
     if (pre[mid] <= g) lo = mid; else hi = mid;
   }
   const int cnt = offsets[lo + 1] - offsets[lo];
-  int64_t prow[4], tok[4], pair[4];
+  int prow[4], tok[4], pair[4];   // (row and slot counts stay below 2^31)
   float gt[4], dot[4];
   bool valid[4];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    prow[i] = blk * 32 + warp * 4 + i;
-    const int64_t local = prow[i] - (int64_t)pre[lo] * 128;
+    prow[i] = (int)blk * 32 + warp * 4 + i;
+    const int local = prow[i] - pre[lo] * 128;
     valid[i] = local < cnt;
-    const int64_t slot = offsets[lo] + (valid[i] ? local : 0);
+    const int slot = offsets[lo] + (valid[i] ? local : 0);
     pair[i] = valid[i] ? pos[slot] : 0;
     tok[i] = pair[i] / k;
     gt[i] = (BWD && valid[i]) ? gate[pair[i]] : 0.f;
     dot[i] = 0.f;
   }
-  for (int c0 = 0; c0 < d; c0 += CB_CHUNK) {
+  // The rows' 16-byte pieces of chunk c0 + CB_CHUNK are loaded while chunk c0 is quantised
+  // (its three block barriers would otherwise leave no load in flight).
+  int slot_of[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) slot_of[i] = offsets[lo] + (prow[i] - pre[lo] * 128);
+  uint4 nx[4], ny[4] = {};
+  auto fetch = [&](int c0n) {
+    const int cn = c0n + lane * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const bool on = valid[i] && cn < d;
+      nx[i] = on ? __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)tok[i] * d + cn)) : make_uint4(0, 0, 0, 0);
+      if constexpr (BWD)
+        ny[i] = on ? __ldg(reinterpret_cast<const uint4 *>(y_perm + (int64_t)slot_of[i] * d + cn))
+                   : make_uint4(0, 0, 0, 0);
+    }
+  };
+  // the forward's blocks take one chunk each (grid.y = chunks); the backward's blocks walk the
+  // whole row, whose dot product with y_perm gives dgate
+  const int c_lo = BWD ? 0 : (int)blockIdx.y * CB_CHUNK, c_hi = BWD ? d : min(d, c_lo + CB_CHUNK);
+  fetch(c_lo);
+  for (int c0 = c_lo; c0 < c_hi; c0 += CB_CHUNK) {
     const int c = c0 + lane * 8;
     const bool cin = c < d;       // d % 128 == 0: a 32-column block is wholly in or out
+    uint4 cx[4], cy[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { cx[i] = nx[i]; cy[i] = ny[i]; }
+    if (BWD && c0 + CB_CHUNK < c_hi) fetch(c0 + CB_CHUNK);
     float v[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int64_t slot = offsets[lo] + (prow[i] - (int64_t)pre[lo] * 128);
+      const int64_t slot = slot_of[i];
       if (valid[i] && cin) {
-        const uint4 raw = __ldg(reinterpret_cast<const uint4 *>(src + tok[i] * d + c));
+        const uint4 raw = cx[i];
         if constexpr (BWD) {
           float fd[8], fy[8];
           Vec<bf16>::load(raw, fd);
-          Vec<bf16>::load(__ldg(reinterpret_cast<const uint4 *>(y_perm + slot * d + c)), fy);
+          Vec<bf16>::load(cy[i], fy);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             dot[i] = fmaf(fd[j], fy[j], dot[i]);
@@ -569,9 +604,10 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
       w.x = (uint32_t)e4m3x2(v[i][0] * inv, v[i][1] * inv) | ((uint32_t)e4m3x2(v[i][2] * inv, v[i][3] * inv) << 16);
       w.y = (uint32_t)e4m3x2(v[i][4] * inv, v[i][5] * inv) | ((uint32_t)e4m3x2(v[i][6] * inv, v[i][7] * inv) << 16);
       if (cin && codes_r) {
-        *reinterpret_cast<uint2 *>(codes_r + prow[i] * d + c) = w;
+        *reinterpret_cast<uint2 *>(codes_r + (int64_t)prow[i] * d + c) = w;
         if ((lane & 3) == 0)
-          scales_r[tiled ? sf_tiled_off(prow[i], c / 32, d / 128) : prow[i] * (d / 32) + c / 32] = (uint8_t)(sc + 127);
+          scales_r[tiled ? sf_tiled_off(prow[i], c / 32, d / 128) : (int64_t)prow[i] * (d / 32) + c / 32] =
+              (uint8_t)(sc + 127);
       }
     }
     // down the token axis: the block's 32 rows of each column
@@ -596,7 +632,7 @@ __global__ void __launch_bounds__(256) mx_slot_dispatch_kernel(
       uint2 w;
       w.x = (uint32_t)e4m3x2(v[i][0] * iv[0], v[i][1] * iv[1]) | ((uint32_t)e4m3x2(v[i][2] * iv[2], v[i][3] * iv[3]) << 16);
       w.y = (uint32_t)e4m3x2(v[i][4] * iv[4], v[i][5] * iv[5]) | ((uint32_t)e4m3x2(v[i][6] * iv[6], v[i][7] * iv[7]) << 16);
-      if (cin) *reinterpret_cast<uint2 *>(codes_c + prow[i] * d + c) = w;
+      if (cin) *reinterpret_cast<uint2 *>(codes_c + (int64_t)prow[i] * d + c) = w;
     }
     __syncthreads();   // colmax and inv_col are rewritten by the next chunk
   }
@@ -626,7 +662,8 @@ cudaError_t launch_mx_dispatch(const void *x, const int32_t *pos, const int32_t 
                                int64_t rows_bound, void *x_perm, uint8_t *codes_r, uint8_t *scales_r,
                                uint8_t *codes_c, uint8_t *scales_c, cudaStream_t st, bool tiled) {
   if (rows_bound <= 0) return cudaSuccess;
-  mx_slot_dispatch_kernel<false><<<(unsigned)((rows_bound + 31) / 32), 256, 0, st>>>(
+  const dim3 grid((unsigned)((rows_bound + 31) / 32), (unsigned)((d + CB_CHUNK - 1) / CB_CHUNK));
+  mx_slot_dispatch_kernel<false><<<grid, 256, 0, st>>>(
       static_cast<const bf16 *>(x), nullptr, pos, offsets, nullptr, E, k, d, (rows_bound + 127) / 128,
       static_cast<bf16 *>(x_perm), nullptr, codes_r, scales_r, codes_c, scales_c, tiled);
   return cudaGetLastError();

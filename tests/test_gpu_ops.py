@@ -107,6 +107,7 @@ def test_route_topk(T, d, E, k, dtype, bias):
     (300, 128, 192, 6, False, 0),      # the second half of a 256-column tile is ragged
     (2000, 512, 128, 1, False, 0),
     (300, 128, 36, 4, False, 2),       # the CUDA-core router
+    (20000, 256, 128, 4, True, 1),     # more 128-token tiles than CTA clusters: several per cluster
 ])
 def test_route_topk_selects_exactly_on_its_own_logits(T, d, E, k, bias, nan_rows):
     """Given the fp32 logits the router wrote, the selection is unique: on every row the
