@@ -175,6 +175,7 @@ struct Ctrl {
   uint64_t xempty[4];     // router: ... and have been merged
   uint32_t tmem_base;
   int abort;
+  int strips;             // A-stationary weight gradients: every expert's A fits its slots
   union {
     int prefix[MAX_E + 1];  // exclusive prefix of 128-row blocks per expert
     float bias[MAX_E];      // router: the logit bias (0 past E)
@@ -365,14 +366,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // tf32 operands are only ever K-major: the fp32 forward reads pre-transposed weights
   constexpr bool FWD_B_KMAJOR = (sizeof(T) == 4) && (MODE == FWD_GU || MODE == FWD_DOWN);
   constexpr bool B_MN = MT::B_MN && !FWD_B_KMAJOR;
-  // A stationary (bf16 weight gradients): the ring memory holds NA A slots and then SB B
-  // slots instead of STAGES (A | B) stages.  CTA pairs hold 128 rows of A and 128 columns of
-  // B per CTA, slots of the same size, so the split is the host's choice (p.na); single CTAs
-  // keep STAGES of each.
-  constexpr bool ASTAT = MT::WGRAD && !C::MX;
-  const int NA = ASTAT ? (C::A_BYTES == C::B_BYTES ? p.na : C::STAGES) : 0;
-  const int SB = ASTAT ? (C::A_BYTES == C::B_BYTES ? 2 * C::STAGES - NA : C::STAGES) : C::STAGES;
-  const bool strips = ASTAT && p.strips;
+  constexpr bool ASTAT = MT::WGRAD && !C::MX;   // A stationary (bf16 weight gradients), below
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ring = smem;                                   // STAGES x (A | B)
@@ -445,6 +439,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if constexpr (SMEM_OFFS) {
     if (warp == 3)
       for (int i = lane; i <= p.E; i += 32) offs_smem[i] = p.offsets[i];
+    if (ASTAT && warp == 3) {
+      // strips only when every expert's K-blocks fit the A slots: a strip of an expert that
+      // streams A would hold its whole row of tiles on one CTA (pair) and stall the others
+      __syncwarp();
+      int mx = 0;
+      for (int e = lane; e < p.E; e += 32) mx = max(mx, offs_smem[e + 1] - offs_smem[e]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      if (lane == 0) c.strips = p.strips && (mx + C::KBLK - 1) / C::KBLK <= p.na;
+    }
   }
   if (warp == 2 && (!MT::WGRAD || C::MX) && MODE != ROUTER) {
     // per-expert 128-row block counts, exclusive prefix: lane l owns experts 8l..8l+7
@@ -478,6 +482,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   ptx::tc_fence_after();
   const uint32_t tmem_base = c.tmem_base;
   const int ntiles = total_tiles<MODE, BN, CG>(p, c);
+  // A stationary (bf16 weight gradients): the ring memory holds NA A slots and then SB B
+  // slots instead of STAGES (A | B) stages.  With strips, CTA pairs (whose A and B slots are
+  // the same size) split the ring's slots by the host's choice (p.na); otherwise, and for
+  // single CTAs, STAGES of each.
+  const bool strips = ASTAT && c.strips;
+  const int NA = ASTAT ? ((C::A_BYTES == C::B_BYTES && strips) ? p.na : C::STAGES) : 0;
+  const int SB = ASTAT ? 2 * C::STAGES - NA : C::STAGES;
 
   if (warp == 0) {
     // ================================================================ producer
