@@ -361,7 +361,9 @@ typedef struct moe_layer_grads {
   void *dy_perm;     /* [P,d] intermediate; unused (may be NULL) with MOE_PREC_MXFP8, where the
                         combine's backward writes it in MXFP8 only */
   float *dgate;      /* [T,k] intermediate */
-  void *dhu;         /* [P,2f] intermediate (also holds recomputed h | u) */
+  void *dhu;         /* [P,2f] intermediate (also holds recomputed h | u); with MOE_PREC_MXFP8
+                        [dh | du] is kept in MXFP8 only and dhu holds no defined values after
+                        the call (it is still required: the recompute's scratch) */
   void *dx_perm;     /* [P,d] intermediate */
   void *dw_shared_gate; /* [d,f] with a shared expert */
   void *dw_shared_up;   /* [d,f] */

@@ -280,6 +280,6 @@ int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, 
                        const void *a, const int32_t *offsets, const void *w_gate,
                        const void *w_up, const void *w_down, void *dhu, void *dx_perm,
                        void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st,
-                       const uint8_t *wsaved = nullptr, bool dy_quantized = false);
+                       const uint8_t *wsaved = nullptr, bool dy_quantized = false, bool keep_dhu = true);
 
 }  // namespace moe

@@ -1058,8 +1058,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
           }
           const int col = tl.n_blk * BN + cc;
-          store_slab(dhu + srow * 2 * p.f + col, 2 * p.f, nvalid, dh);
-          store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
+          if (dhu) {   // (the MXFP8 layer keeps [dh | du] in MXFP8 only)
+            store_slab(dhu + srow * 2 * p.f + col, 2 * p.f, nvalid, dh);
+            store_slab(dhu + srow * 2 * p.f + p.f + col, 2 * p.f, nvalid, du);
+          }
           if constexpr (C::MX) {
             if (p.q_row_codes) {
               // the gate/up GEMMs' operand: the stored bf16 [dh | du] in MXFP8 along 2f (for the
@@ -1590,7 +1592,7 @@ static int mx_fwd_impl(const Shape &s, const void *x_perm, const int32_t *offset
 static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu, const void *a,
                        const int32_t *offsets, const void *w_gate, const void *w_up, const void *w_down, void *dhu,
                        void *dx_perm, void *dw_gate, void *dw_up, void *dw_down, void *ws, cudaStream_t st,
-                       const uint8_t *wsaved, bool dy_quantized) {
+                       const uint8_t *wsaved, bool dy_quantized, bool keep_dhu) {
   const WsLayout L = ws_layout(s);
   const int64_t P = s.P(), R = s.Ppad(), ed = (int64_t)s.E * s.d, ef = (int64_t)s.E * s.f;
   const int nkt = (int)((R + 127) / 128);   // K groups of the token-axis operands
@@ -1618,7 +1620,8 @@ static int mx_bwd_impl(const Shape &s, const void *dy_perm, const void *x_perm, 
     return MOE_ERR_CUDA;
   if (!make_tmap(&tA, dyq.codes, 1, s.d, R, 128, BM) || !make_tmap(&tB, wdr.codes, 1, s.d, ef, 128, 128))
     return MOE_ERR_CUDA;
-  p.K = s.d; p.N = s.f; p.out0 = dhu; p.aux = hu;
+  // keep_dhu: [dh | du] in bf16 as well (nothing in the MXFP8 backward reads it)
+  p.K = s.d; p.N = s.f; p.out0 = keep_dhu ? dhu : nullptr; p.aux = hu;
   p.sfa = dyq.scales; p.nka = s.d / 128; p.sfb = wdr.scales; p.nkb = s.d / 128;
   // the epilogue also writes [dh | du] in MXFP8 in both orientations the gate/up GEMMs read
   p.q_row_codes = dhuq.codes; p.q_row_scales = dhuq.scales; p.nk_row = 2 * s.f / 128;
@@ -1682,13 +1685,14 @@ int launch_grouped_fwd(const Shape &s, const void *x_perm, const int32_t *offset
 int launch_grouped_bwd(const Shape &s, const void *dy_perm, const void *x_perm, const void *hu,
                        const void *a, const int32_t *offsets, const void *w_gate, const void *w_up,
                        const void *w_down, void *dhu, void *dx_perm, void *dw_gate, void *dw_up,
-                       void *dw_down, void *ws, cudaStream_t st, const uint8_t *wsaved, bool dy_quantized) {
+                       void *dw_down, void *ws, cudaStream_t st, const uint8_t *wsaved, bool dy_quantized,
+                       bool keep_dhu) {
   // The weight-gradient GEMMs reduce over tokens, which makes both operands MN-major;
   // tf32 MMAs take K-major operands only, so the fp32 backward is not offered.
   if (s.dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (s.prec == MOE_PREC_MXFP8)
     return gg::mx_bwd_impl(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm, dw_gate,
-                           dw_up, dw_down, ws, st, wsaved, dy_quantized);
+                           dw_up, dw_down, ws, st, wsaved, dy_quantized, keep_dhu);
   return gg::bwd_impl<bf16>(s, dy_perm, x_perm, hu, a, offsets, w_gate, w_up, w_down, dhu, dx_perm,
                             dw_gate, dw_up, dw_down, ws, st);
 }

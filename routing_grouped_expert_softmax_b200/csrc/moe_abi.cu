@@ -436,8 +436,10 @@ int moe_layer_bwd(const moe_config *cfg, const moe_layer_weights *w, const void 
                                  nullptr, ws, st, /*x_quantized=*/rows_fp8, mxs, /*wfill=*/false));
     hu = g->dhu;
   }
+  // MXFP8: [dh | du] is kept in MXFP8 only (g->dhu serves as the recompute's scratch)
   RETURN_IF(launch_grouped_bwd(s, g->dy_perm, sv->x_perm, hu, sv->a, sv->offsets, w->w_gate, w->w_up,
-                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st, mxs, mx));
+                               w->w_down, g->dhu, g->dx_perm, g->dw_gate, g->dw_up, g->dw_down, ws, st, mxs, mx,
+                               /*keep_dhu=*/!mx));
   if (shared) {
     // one group of all tokens: its dy is dY itself (weight 1) and its dx, in token order,
     // is written to dx, to which the routed experts' rows are then added

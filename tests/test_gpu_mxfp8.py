@@ -323,7 +323,7 @@ def test_mx_layer_against_oracle_and_bf16_path(T, d, E, k, f, skew):
     y, sv, g = outs["mxfp8"]
     zg = check_logits_and_routing(inp, sv)
     fwd, bwd_fn = gpu_decided_oracle(inp, zg, mx=True)
-    check_layer(y, sv, g, fwd, bwd_fn(fwd), f, TOL_MX, TOL_MX, tag="mxfp8 ")
+    check_layer(y, sv, g, fwd, bwd_fn(fwd), f, TOL_MX, TOL_MX, tag="mxfp8 ", dhu=False)
     # and MXFP8 stays close to the bf16 path (quantisation error only)
     ybf, _, gbf = outs["native"]
     assert 0 < rel_err(host(y), host(ybf)) <= 0.1
