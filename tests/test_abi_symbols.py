@@ -141,3 +141,59 @@ def test_debug_stall_hook_validates_its_limit(lib):
     assert lib.moe_debug_set_gemm_stall_ns(2_000_000_000) == moe.MOE_ERR_INVALID_ARG
     assert lib.moe_debug_set_gemm_stall_ns(1_000_000) == moe.MOE_OK
     assert lib.moe_debug_set_gemm_stall_ns(0) == moe.MOE_OK
+
+
+def test_dispatch_mxfp8_host_validation(lib):
+    cfg = moe.config(16, 128, 8, 2, 128)
+    bound = 16 * 2 + 127 * 8
+    # (cfg, x, pair_of_slot, offsets, rows_bound, x_perm, codes_r, scales_r, codes_c, scales_c, stream)
+    c32 = moe.config(16, 128, 8, 2, 128, dtype="f32")
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(c32), 16, 16, 16, bound, None, 16, 16, 16, 16, None) \
+        == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(cfg), 16, 16, 16, bound - 1, None, 16, 16, 16, 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(cfg), 16, 16, 16, bound, 24, 16, 16, 16, 16, None) \
+        == moe.MOE_ERR_INVALID_ARG                                   # x_perm, when given, 16-byte aligned
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(cfg), 16, 16, 16, bound, None, None, 16, 16, 16, None) \
+        == moe.MOE_ERR_INVALID_ARG                                   # both orientations are outputs
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(cfg), 16, 16, 16, bound, None, 16, 16, 16, 6, None) \
+        == moe.MOE_ERR_INVALID_ARG                                   # scales 4-byte aligned
+    c0 = moe.config(0, 128, 8, 2, 128)
+    assert lib.moe_dispatch_mxfp8(ctypes.byref(c0), None, None, None, 0, None, None, None, None, None, None) \
+        == moe.MOE_OK
+    # (cfg, dy, y_perm, pair_of_slot, offsets, topk_gate, rows_bound, dy_perm, dgate, codes_r, scales_r,
+    #  codes_c, scales_c, stream)
+    assert lib.moe_combine_bwd_mxfp8(ctypes.byref(c32), 16, 16, 16, 16, 16, bound, None, 16, 16, 16, 16, 16,
+                                     None) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_combine_bwd_mxfp8(ctypes.byref(cfg), 16, 16, 16, 16, 16, bound - 1, None, 16, 16, 16, 16, 16,
+                                     None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_combine_bwd_mxfp8(ctypes.byref(cfg), 16, 16, 16, 16, 16, bound, None, None, 16, 16, 16, 16,
+                                     None) == moe.MOE_ERR_INVALID_ARG  # dgate is an output
+    assert lib.moe_combine_bwd_mxfp8(ctypes.byref(c0), None, None, None, None, None, 0, None, None, None, None,
+                                     None, None, None) == moe.MOE_OK
+
+
+def test_layer_bf16_rows_are_optional_only_in_mxfp8(lib):
+    w = moe.LayerWeights(16, None, 16, 16, 16, None, None, None)
+    # bf16 layer: x_perm is required
+    cfg = moe.config(16, 128, 8, 2, 128)
+    fields = {n: 16 for n in moe.SAVED_FIELDS}
+    fields["x_perm"] = None
+    fields["mx_saved"] = None
+    sv = moe.LayerSaved(*[fields[n] for n in moe.SAVED_FIELDS])
+    assert lib.moe_layer_fwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    # MXFP8 without the saved copies: the forward writes x_perm, so it is required too
+    cmx = moe.config(16, 128, 8, 2, 128, prec="mxfp8")
+    assert lib.moe_layer_fwd(ctypes.byref(cmx), ctypes.byref(w), 16, 16, ctypes.byref(sv), 16, None) \
+        == moe.MOE_ERR_INVALID_ARG
+    # bf16 backward: dy_perm is required (MXFP8 keeps it in MXFP8 only)
+    fields = {n: 16 for n in moe.SAVED_FIELDS}
+    sv = moe.LayerSaved(*[fields[n] for n in moe.SAVED_FIELDS])
+    gf = {n: 16 for n in moe.GRAD_FIELDS}
+    gf["dy_perm"] = None
+    for n in ("dw_shared_gate", "dw_shared_up", "dw_shared_down", "shared_dhu"):
+        gf[n] = None
+    g = moe.LayerGrads(*[gf[n] for n in moe.GRAD_FIELDS])
+    assert lib.moe_layer_bwd(ctypes.byref(cfg), ctypes.byref(w), 16, 16, ctypes.byref(sv), ctypes.byref(g), 16,
+                             None) == moe.MOE_ERR_INVALID_ARG
